@@ -1,0 +1,170 @@
+/*
+ * mimo_attn.h — C ABI of the MiMo-V2-Flash hybrid attention layer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * One layer of the decoder's attention, as the pages describe it:
+ *   - "Add Xiaomi MiMo-V2" (huggingface/transformers pull request 45144),
+ *     section "Additional useful info": partial RoPE over the leading third
+ *     of the QK head dim; a RoPE base that differs between sliding-window
+ *     (SWA) and global (GA) layers; a KV-head count that differs between
+ *     them (GQA); a V head dim decoupled from the QK head dim; V rescaled by
+ *     sqrt(hidden_size / (num_attention_heads * v_head_dim)); a gpt-oss-style
+ *     attention sink on SWA layers only.
+ *   - "feat(models): add Xiaomi MiMo v2 (mimo_v2_flash) text model support"
+ *     (lablup/mlxcel issue 842), section "Architecture, verified against
+ *     upstream": hybrid_layer_pattern[idx] == 1 selects a sliding layer with
+ *     a window of sliding_window_size; the RoPE base is swa_rope_theta on
+ *     sliding layers and rope_theta otherwise; the rotated width is
+ *     int(partial_rotary_factor * head_dim). Section "Implementation plan":
+ *     sliding layers keep a rotating (ring) KV cache.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are dense, row-major, in device memory (cudaMalloc or torch),
+ *     in the element type given by `dtype` unless stated otherwise. The
+ *     caller owns every buffer; the library never allocates device memory
+ *     on these calls and keeps no pointer after a call returns.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream) and never synchronises.
+ *   - Arguments are checked on the host before any launch. A bad argument
+ *     returns a non-zero status and launches nothing. A failed launch
+ *     returns MIMO_ATTN_ERR_CUDA. Conditions only the device can see
+ *     (kv_lens out of range, a pipeline wait that timed out) set the
+ *     device error word read by mimo_attn_get_device_error(); nothing traps.
+ *   - Base pointers of bf16 tensors must be 16-byte aligned (TMA rule).
+ */
+#ifndef MIMO_ATTN_H
+#define MIMO_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MIMO_ATTN_OK = 0,
+    MIMO_ATTN_ERR_INVALID_ARG = 1,  /* shape, pointer or value check failed */
+    MIMO_ATTN_ERR_UNSUPPORTED = 2,  /* valid, but no kernel handles it (e.g. dims > 256) */
+    MIMO_ATTN_ERR_WORKSPACE = 3,    /* workspace missing or smaller than the size query says */
+    MIMO_ATTN_ERR_CUDA = 4          /* a CUDA runtime call or launch failed */
+} mimo_attn_status;
+
+/* Layer kind = the layer's hybrid_layer_pattern entry (lablup/mlxcel issue
+ * 842, "Architecture, verified against upstream"). */
+typedef enum { MIMO_ATTN_GLOBAL = 0, MIMO_ATTN_SWA = 1 } mimo_attn_layer_type;
+
+/* Element type of q, k, v, out and the caches. */
+typedef enum { MIMO_ATTN_BF16 = 0, MIMO_ATTN_FP32 = 1 } mimo_attn_dtype;
+
+/* Per-layer parameters (host struct; read during the call only). */
+typedef struct {
+    int32_t layer_type;    /* mimo_attn_layer_type */
+    int32_t num_q_heads;   /* Hq */
+    int32_t num_kv_heads;  /* Hkv; Hq % Hkv == 0; query head h reads KV head h / (Hq/Hkv) */
+    int32_t qk_dim;        /* Dqk, even, <= 256 */
+    int32_t v_dim;         /* Dv, <= 256 (decoupled from Dqk, PR 45144) */
+    int32_t rotary_dim;    /* r = int(partial_rotary_factor * qk_dim); even, 0 <= r <= Dqk */
+    int32_t window;        /* SWA: keys visible to query i are i-window+1 .. i; ignored for GLOBAL */
+    int32_t hidden_size;   /* V scale = sqrt(hidden_size / (Hq * Dv)); must be > 0 */
+    double rope_theta;     /* base of this layer: swa_rope_theta (SWA) or rope_theta (GLOBAL); > 0 */
+    float softmax_scale;   /* 0 selects 1/sqrt(Dqk) */
+    const float *sinks;    /* device [Hq] fp32 sink logits, one per query head; SWA only
+                              (must be NULL for GLOBAL, PR 45144); NULL = no sink */
+} mimo_attn_layer;
+
+/* Rotated width helper: int(partial_rotary_factor * qk_dim), the rule of
+ * lablup/mlxcel issue 842 ("Architecture, verified against upstream"); the
+ * factor is taken as a double because upstream types it as an int but uses
+ * it as a multiplier. Returns -1 for a negative or non-finite product. */
+int mimo_attn_rotary_dim(double partial_rotary_factor, int qk_dim);
+
+/* Bytes of workspace mimo_attn_prefill needs for this layer and shape
+ * (the rotated keys when they are not written into a global cache). The
+ * value does not depend on whether caches are passed; 0 means none. */
+size_t mimo_attn_prefill_workspace_size(const mimo_attn_layer *layer, int dtype,
+                                        int batch, int seq);
+
+/* Prefill: one layer's attention over a whole prompt.
+ *   q   [batch, seq, Hq,  Dqk]  unrotated queries
+ *   k   [batch, seq, Hkv, Dqk]  unrotated keys
+ *   v   [batch, seq, Hkv, Dv]
+ *   positions: device int32 [seq] RoPE positions, or NULL for 0..seq-1.
+ *              Masking always uses the sequence index (causal, window).
+ *   out [batch, seq, Hq, Dv]    out[b,i,h] = Vscale * sum_j p_ij v_j, with
+ *              p the softmax over the visible keys j (GLOBAL: j <= i; SWA:
+ *              i-window < j <= i) plus, on SWA with sinks, the sink term
+ *              exp(sink[h]) in the denominator only.
+ *   k_cache, v_cache: optional (both NULL or both set). GLOBAL: linear caches
+ *              [batch, cache_capacity, Hkv, D] with cache_capacity >= seq;
+ *              slots 0..seq-1 receive the rotated keys and the values.
+ *              SWA: ring caches [batch, window, Hkv, D], cache_capacity ==
+ *              window; token i (for i >= seq - window) lands in slot
+ *              i mod window.
+ *   workspace: device buffer of at least mimo_attn_prefill_workspace_size()
+ *              bytes (may be NULL when that size is 0), 256-byte aligned.
+ * Errors: MIMO_ATTN_ERR_INVALID_ARG for null required pointers, batch or
+ * seq < 0, Hq % Hkv != 0, odd or out-of-range rotary_dim, window < 1 on SWA,
+ * sinks on GLOBAL, a cache capacity that breaks the rules above, theta <= 0,
+ * misaligned bf16 pointers; MIMO_ATTN_ERR_UNSUPPORTED for dims > 256;
+ * MIMO_ATTN_ERR_WORKSPACE for a short workspace. batch == 0 or seq == 0 is
+ * a no-op returning MIMO_ATTN_OK. */
+mimo_attn_status mimo_attn_prefill(const mimo_attn_layer *layer, int dtype, int batch, int seq,
+                                   const void *q, const void *k, const void *v,
+                                   const int32_t *positions, void *out,
+                                   void *k_cache, void *v_cache, int cache_capacity,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace mimo_attn_decode needs (split-KV partial results) for
+ * this layer, batch and cache capacity. */
+size_t mimo_attn_decode_workspace_size(const mimo_attn_layer *layer, int dtype, int batch,
+                                       int cache_capacity);
+
+/* Decode: one new token per sequence, attending to its cache.
+ *   q     [batch, Hq, Dqk], k_new [batch, Hkv, Dqk], v_new [batch, Hkv, Dv], unrotated.
+ *   kv_lens: device int32 [batch]; L_b counts the new token (L_b >= 1), so the
+ *          new token's position is L_b - 1. GLOBAL needs L_b <= cache_capacity.
+ *   k_cache, v_cache (required, updated in place):
+ *          GLOBAL: linear [batch, cache_capacity, Hkv, D]; slot p holds the
+ *          rotated key / value of position p (p < L_b - 1 already filled).
+ *          SWA: ring [batch, window, Hkv, D] with cache_capacity == window;
+ *          slot p mod window holds position p.
+ *          The call writes the new token's rotated key and value into slot
+ *          L_b - 1 (GLOBAL) or (L_b - 1) mod window (SWA).
+ *   out   [batch, Hq, Dv]: attention of the new token over positions
+ *          0..L_b-1 (GLOBAL) or max(0, L_b-window)..L_b-1 (SWA), with the
+ *          sink and V scale as in mimo_attn_prefill.
+ *   workspace: at least mimo_attn_decode_workspace_size() bytes, 256-byte aligned.
+ * A kv_lens entry out of range sets MIMO_ATTN_DEVERR_KV_LEN in the device
+ * error word and leaves that sequence's output and cache untouched. */
+mimo_attn_status mimo_attn_decode(const mimo_attn_layer *layer, int dtype, int batch,
+                                  const void *q, const void *k_new, const void *v_new,
+                                  const int32_t *kv_lens, void *k_cache, void *v_cache,
+                                  int cache_capacity, void *out, void *workspace,
+                                  size_t workspace_bytes, void *stream);
+
+/* Device error word bits (sticky until read). */
+#define MIMO_ATTN_DEVERR_KV_LEN 0x1u   /* a kv_lens entry was out of range */
+#define MIMO_ATTN_DEVERR_TIMEOUT 0x2u  /* a kernel pipeline wait hit its iteration limit */
+
+/* Reads and clears the device error word of the current device
+ * (synchronises the device). Returns MIMO_ATTN_OK and stores the bits in
+ * *bits, or MIMO_ATTN_ERR_CUDA. */
+mimo_attn_status mimo_attn_get_device_error(uint32_t *bits);
+
+/* Static description of a status code. */
+const char *mimo_attn_status_string(mimo_attn_status status);
+
+/* Test hook: while non-zero, every launching entry point returns
+ * MIMO_ATTN_ERR_CUDA after its argument checks, without launching. Lets the
+ * host-side error path be tested without provoking a GPU fault. */
+void mimo_attn_debug_fail_launches(int enable);
+
+/* Version string of the library. */
+const char *mimo_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MIMO_ATTN_H */

@@ -1,0 +1,187 @@
+"""fp64 CPU oracle for the MiMo-V2-Flash hybrid attention layer.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` are the only
+callers. The CUDA library never imports, links or runs anything here, and
+nothing here imports the CUDA library.
+
+The arithmetic lives in ``mimo_oracle.c`` (plain C, double precision, plain
+loops). This module compiles it with gcc when needed, loads it with ctypes
+and marshals numpy arrays; the composition helpers below only chain the C
+steps in the pages' order (rotate Q and K at their positions, then attend),
+see "Add Xiaomi MiMo-V2" (huggingface/transformers PR 45144), section
+"Additional useful info", and "feat(models): add Xiaomi MiMo v2
+(mimo_v2_flash) text model support" (lablup/mlxcel issue 842), section
+"Architecture, verified against upstream".
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mimo_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+GLOBAL = 0
+SWA = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile mimo_oracle.c into liboracle.so next to it (gcc, -O2)."""
+    if force or not os.path.exists(_LIB_PATH) or (
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    ):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-Wall", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        dp = ctypes.POINTER(ctypes.c_double)
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        lib.oracle_rope.argtypes = [dp, dp, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_double, dp]
+        lib.oracle_rope.restype = ctypes.c_int
+        lib.oracle_prefill_rows.argtypes = [dp, i64p, ctypes.c_int64, dp, dp, ctypes.c_int64,
+                                            ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int64, ctypes.c_double, ctypes.c_int,
+                                            ctypes.c_double, ctypes.c_double, dp]
+        lib.oracle_prefill_rows.restype = ctypes.c_int
+        lib.oracle_decode.argtypes = [dp, ctypes.c_int, dp, dp, dp, dp, ctypes.c_int64,
+                                      ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_double, ctypes.c_int, ctypes.c_int64,
+                                      ctypes.c_double, dp, ctypes.c_double, dp]
+        lib.oracle_decode.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def default_softmax_scale(qk_dim: int) -> float:
+    """1/sqrt(qk_dim): the pages name no scale; the standard one is the reading."""
+    return 1.0 / math.sqrt(qk_dim)
+
+
+def v_scale(hidden_size: int, num_q_heads: int, v_dim: int) -> float:
+    """The V rescale factor sqrt(hidden / (Hq * v_dim)) (PR 45144, Additional useful info)."""
+    return math.sqrt(hidden_size / (num_q_heads * v_dim))
+
+
+def rope(x, rotary_dim: int, theta: float, pos) -> np.ndarray:
+    """Partial RoPE of the rows of x ([n, dim]) at positions pos ([n])."""
+    x = _f64(x)
+    squeeze = x.ndim == 1
+    if squeeze:
+        x = x[None, :]
+    n, dim = x.shape
+    p = _f64(np.broadcast_to(np.asarray(pos, dtype=np.float64), (n,)))
+    y = np.empty_like(x)
+    rc = _load().oracle_rope(_ptr(x), _ptr(y), n, dim, int(rotary_dim), float(theta), _ptr(p))
+    if rc != 0:
+        raise ValueError("oracle_rope: bad rotary_dim")
+    return y[0] if squeeze else y
+
+
+def prefill_rows(q_rot, rows: Sequence[int], k_rot, v, layer_type: int, window: int,
+                 softmax_scale: float, sink: Optional[float], vscale: float) -> np.ndarray:
+    """Output rows of one (batch, query head): q_rot [n, Dqk] at indices rows,
+    against rotated keys k_rot [S, Dqk] and values v [S, Dv]."""
+    q_rot = _f64(q_rot)
+    k_rot = _f64(k_rot)
+    v = _f64(v)
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    n = r.shape[0]
+    seq, qk_dim = k_rot.shape
+    v_dim = v.shape[1]
+    out = np.empty((n, v_dim), dtype=np.float64)
+    has_sink = sink is not None
+    rc = _load().oracle_prefill_rows(
+        _ptr(q_rot), r.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n, _ptr(k_rot), _ptr(v),
+        seq, qk_dim, v_dim, int(layer_type), int(window), float(softmax_scale), int(has_sink),
+        float(sink) if has_sink else 0.0, float(vscale), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_prefill_rows: bad argument")
+    return out
+
+
+def decode(q, k_new, v_new, k_cache, v_cache, L: int, rotary_dim: int, theta: float,
+           layer_type: int, window: int, softmax_scale: float, sinks, vscale: float):
+    """One decode step of one (batch, KV head). q: [n_q, Dqk] unrotated query
+    heads of the group; k_new [Dqk], v_new [Dv] unrotated; k_cache [cap, Dqk]
+    (rotated keys), v_cache [cap, Dv]. Returns (out [n_q, Dv], k_cache', v_cache')
+    with the new token written into its slot."""
+    q = _f64(q)
+    if q.ndim == 1:
+        q = q[None, :]
+    n_q, qk_dim = q.shape
+    k_new = _f64(k_new)
+    v_new = _f64(v_new)
+    kc = np.array(k_cache, dtype=np.float64, copy=True, order="C")
+    vc = np.array(v_cache, dtype=np.float64, copy=True, order="C")
+    cap = kc.shape[0]
+    v_dim = vc.shape[1]
+    out = np.empty((n_q, v_dim), dtype=np.float64)
+    s = None if sinks is None else _f64(sinks)
+    rc = _load().oracle_decode(
+        _ptr(q), n_q, _ptr(k_new), _ptr(v_new), _ptr(kc), _ptr(vc), cap, int(L), qk_dim, v_dim,
+        int(rotary_dim), float(theta), int(layer_type), int(window), float(softmax_scale),
+        None if s is None else _ptr(s), float(vscale), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_decode: bad argument")
+    return out, kc, vc
+
+
+def prefill_layer(q, k, v, *, layer_type: int, num_kv_heads: int, rotary_dim: int, theta: float,
+                  window: int, sinks, hidden_size: int, softmax_scale: Optional[float] = None,
+                  positions=None, rows=None, heads=None, batches=None):
+    """Whole-layer prefill in the pages' order: rotate Q and K (partial RoPE at
+    each token's position), then attend per (batch, query head) row.
+
+    q [B, S, Hq, Dqk], k [B, S, Hkv, Dqk], v [B, S, Hkv, Dv] (any float dtype,
+    converted to double). rows/heads/batches restrict the computed outputs
+    (the result holds NaN elsewhere). Returns out [B, S, Hq, Dv] in float64.
+    """
+    q = np.asarray(q)
+    k = np.asarray(k)
+    v = np.asarray(v)
+    B, S, Hq, Dqk = q.shape
+    Dv = v.shape[3]
+    G = Hq // num_kv_heads
+    scale = default_softmax_scale(Dqk) if softmax_scale is None else softmax_scale
+    vs = v_scale(hidden_size, Hq, Dv)
+    pos = np.arange(S, dtype=np.float64) if positions is None else _f64(positions)
+    rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
+    heads = range(Hq) if heads is None else heads
+    batches = range(B) if batches is None else batches
+    out = np.full((B, S, Hq, Dv), np.nan, dtype=np.float64)
+    for b in batches:
+        k_rot = {}
+        for h in heads:
+            kv = h // G
+            if kv not in k_rot:
+                k_rot[kv] = rope(k[b, :, kv, :], rotary_dim, theta, pos)
+            q_rot = rope(q[b, rows, h, :], rotary_dim, theta, pos[rows])
+            sink = None if sinks is None else float(np.asarray(sinks)[h])
+            out[b, rows, h, :] = prefill_rows(q_rot, rows, k_rot[kv], v[b, :, kv, :], layer_type,
+                                              window, scale, sink, vs)
+    return out

@@ -1,0 +1,321 @@
+"""Pins of the fp64 oracle to facts that do not come from the oracle itself.
+
+Each test ties one step of the oracle to a closed form, an invariant the pages
+or the mathematics fix, or a library routine it must reduce to (torch SDPA in
+float64, torch.softmax). The plausible mistakes each one catches are named in
+its docstring. No GPU is used.
+
+Pages: "Add Xiaomi MiMo-V2" (huggingface/transformers PR 45144), section
+"Additional useful info"; "feat(models): add Xiaomi MiMo v2 (mimo_v2_flash)
+text model support" (lablup/mlxcel issue 842), section "Architecture,
+verified against upstream".
+"""
+import cmath
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+
+RNG = np.random.default_rng(1234)
+
+
+def rnd(*shape):
+    return RNG.standard_normal(shape)
+
+
+# ---------------------------------------------------------------- RoPE pins
+
+def test_rope_rotary_dim_zero_is_identity():
+    """rotary_dim 0 leaves Q/K untouched (an invariant the layer's config fixes)."""
+    x = rnd(7, 48)
+    y = oracle.rope(x, 0, 1e4, np.arange(7) * 37.0)
+    assert np.array_equal(x, y)
+
+
+def test_rope_position_zero_is_identity():
+    x = rnd(5, 192)
+    y = oracle.rope(x, 64, 5e6, np.zeros(5))
+    assert np.array_equal(x, y)
+
+
+def test_rope_preserves_pair_norms():
+    """A rotation keeps |(x_j, x_{j+r/2})| and leaves dims >= r alone; catches a
+    scale error or a wrong partner index."""
+    x = rnd(9, 192)
+    pos = RNG.integers(0, 40000, 9).astype(np.float64)
+    y = oracle.rope(x, 64, 1e4, pos)
+    half = 32
+    nx = x[:, :half] ** 2 + x[:, half:64] ** 2
+    ny = y[:, :half] ** 2 + y[:, half:64] ** 2
+    np.testing.assert_allclose(ny, nx, rtol=1e-13, atol=1e-13)
+    assert np.array_equal(x[:, 64:], y[:, 64:])
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)
+
+
+@pytest.mark.parametrize("r,theta", [(64, 1e4), (16, 1e6), (64, 5e6), (2, 10.0)])
+def test_rope_position_one_closed_form(r, theta):
+    """At position 1, pair j turns by theta^(-2j/r): written as a complex product
+    (a + i b) * exp(i * phi) with cmath. Catches a wrong sign, a wrong pairing
+    (interleaved vs half-split) or a frequency denominator other than r."""
+    dim = max(r, 8) + 6
+    x = rnd(dim)
+    y = oracle.rope(x, r, theta, 1.0)
+    half = r // 2
+    for j in range(half):
+        z = complex(x[j], x[j + half]) * cmath.exp(1j * theta ** (-2.0 * j / r))
+        assert abs(y[j] - z.real) < 1e-14 and abs(y[j + half] - z.imag) < 1e-14
+    assert np.array_equal(y[r:], x[r:])
+
+
+def test_rope_relative_position_property():
+    """<R(p)q, R(s)k> depends only on p - s (shift all positions by c)."""
+    q = rnd(192)
+    k = rnd(192)
+    for p, s, c in [(5, 2, 100), (3000, 17, 12345), (0, 0, 7)]:
+        a = oracle.rope(q, 64, 1e4, p) @ oracle.rope(k, 64, 1e4, s)
+        b = oracle.rope(q, 64, 1e4, p + c) @ oracle.rope(k, 64, 1e4, s + c)
+        assert abs(a - b) < 1e-10
+
+
+def test_rope_rejects_odd_or_oversized_rotary_dim():
+    with pytest.raises(ValueError):
+        oracle.rope(rnd(8), 3, 1e4, 1.0)
+    with pytest.raises(ValueError):
+        oracle.rope(rnd(8), 10, 1e4, 1.0)
+
+
+# ------------------------------------------------------- attention pins
+
+def _layer(q, k, v, **kw):
+    return oracle.prefill_layer(q, k, v, **kw)
+
+
+def _sdpa(q, k, v, mask=None, causal=False, scale=None):
+    """torch SDPA in float64; q [B,S,Hq,D] layout converted to [B,H,S,D]."""
+    tq, tk, tv = (torch.from_numpy(np.ascontiguousarray(a)).permute(0, 2, 1, 3) for a in (q, k, v))
+    o = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, is_causal=causal, scale=scale,
+                                       enable_gqa=True)
+    return o.permute(0, 2, 1, 3).numpy()
+
+
+@pytest.mark.parametrize("B,S,Hq,Hkv,D,Dv", [(1, 37, 4, 1, 48, 32), (2, 64, 8, 2, 24, 40),
+                                            (1, 1, 2, 2, 16, 8)])
+def test_global_layer_matches_sdpa_causal(B, S, Hq, Hkv, D, Dv):
+    """Global layer, rotary 0, V scale 1, no sink == torch SDPA(is_causal, GQA).
+    Catches a mask off by one, a transposed operand, a wrong softmax scale
+    (SDPA's default is 1/sqrt(D)) and a wrong KV-head mapping (SDPA's GQA
+    repeats each KV head for consecutive query heads)."""
+    q, k, v = rnd(B, S, Hq, D), rnd(B, S, Hkv, D), rnd(B, S, Hkv, Dv)
+    out = _layer(q, k, v, layer_type=0, num_kv_heads=Hkv, rotary_dim=0, theta=1e4, window=0,
+                 sinks=None, hidden_size=Hq * Dv)
+    ref = _sdpa(q, k, v, causal=True)
+    np.testing.assert_allclose(out, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_rotated_global_layer_matches_sdpa_on_rotated_inputs():
+    """With rotary on, the layer equals SDPA on pre-rotated q/k (RoPE is pinned
+    above), so rotation happens at each token's own position."""
+    B, S, Hq, Hkv, D, Dv = 1, 50, 4, 2, 48, 16
+    q, k, v = rnd(B, S, Hq, D), rnd(B, S, Hkv, D), rnd(B, S, Hkv, Dv)
+    pos = np.arange(S, dtype=np.float64)
+    qr = np.stack([oracle.rope(q[0, :, h], 16, 1e6, pos) for h in range(Hq)], axis=1)[None]
+    kr = np.stack([oracle.rope(k[0, :, h], 16, 1e6, pos) for h in range(Hkv)], axis=1)[None]
+    out = _layer(q, k, v, layer_type=0, num_kv_heads=Hkv, rotary_dim=16, theta=1e6, window=0,
+                 sinks=None, hidden_size=Hq * Dv)
+    np.testing.assert_allclose(out, _sdpa(qr, kr, v, causal=True), rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("S,W", [(64, 16), (33, 1), (20, 7), (5, 9)])
+def test_swa_layer_without_sink_matches_sdpa_band_mask(S, W):
+    """Sliding window, no sink == SDPA with the band mask 0 <= i-j < W (W keys
+    including the query). Catches a window of W+1 or W-1 keys."""
+    B, Hq, Hkv, D, Dv = 1, 4, 2, 48, 32
+    q, k, v = rnd(B, S, Hq, D), rnd(B, S, Hkv, D), rnd(B, S, Hkv, Dv)
+    i = torch.arange(S)[:, None]
+    j = torch.arange(S)[None, :]
+    mask = (j <= i) & (i - j < W)
+    out = _layer(q, k, v, layer_type=1, num_kv_heads=Hkv, rotary_dim=0, theta=1e4, window=W,
+                 sinks=None, hidden_size=Hq * Dv)
+    np.testing.assert_allclose(out, _sdpa(q, k, v, mask=mask), rtol=1e-11, atol=1e-12)
+
+
+def test_window_at_least_seq_with_minus_inf_sink_equals_global():
+    """Invariant: window >= seq_len and a -inf sink reduce SWA to global attention."""
+    B, S, Hq, Hkv, D, Dv = 2, 40, 4, 2, 48, 32
+    q, k, v = rnd(B, S, Hq, D), rnd(B, S, Hkv, D), rnd(B, S, Hkv, Dv)
+    common = dict(num_kv_heads=Hkv, rotary_dim=16, theta=1e4, hidden_size=256)
+    g = _layer(q, k, v, layer_type=0, window=0, sinks=None, **common)
+    for W in (S, S + 5):
+        s = _layer(q, k, v, layer_type=1, window=W, sinks=np.full(Hq, -np.inf), **common)
+        np.testing.assert_allclose(s, g, rtol=1e-13, atol=1e-14)
+
+
+def test_sink_matches_softmax_over_augmented_scores():
+    """The sink joins the denominator only: softmax over [scores, sink] with
+    the sink column dropped (torch.softmax in float64). Catches a sink that
+    is scaled by the softmax scale, given a value, or left out."""
+    S, D, Dv, W = 30, 16, 8, 6
+    q, k, v = rnd(1, S, 1, D), rnd(1, S, 1, D), rnd(1, S, 1, Dv)
+    sink = np.array([0.7])
+    out = _layer(q, k, v, layer_type=1, num_kv_heads=1, rotary_dim=0, theta=1e4, window=W,
+                 sinks=sink, hidden_size=Dv)
+    tq, tk, tv = (torch.from_numpy(a[0, :, 0]) for a in (q, k, v))
+    scores = tq @ tk.T / math.sqrt(D)
+    i = torch.arange(S)[:, None]
+    j = torch.arange(S)[None, :]
+    scores = scores.masked_fill(~((j <= i) & (i - j < W)), float("-inf"))
+    aug = torch.cat([scores, torch.full((S, 1), 0.7, dtype=torch.float64)], dim=1)
+    p = torch.softmax(aug, dim=1)[:, :S]
+    np.testing.assert_allclose(out[0, :, 0], (p @ tv).numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_minus_inf_sink_is_plain_softmax():
+    S, D, Dv = 25, 48, 32
+    q, k, v = rnd(1, S, 2, D), rnd(1, S, 1, D), rnd(1, S, 1, Dv)
+    kw = dict(layer_type=1, num_kv_heads=1, rotary_dim=16, theta=1e4, window=8, hidden_size=64)
+    a = _layer(q, k, v, sinks=np.full(2, -np.inf), **kw)
+    b = _layer(q, k, v, sinks=None, **kw)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_single_key_closed_form():
+    """One KV position: o = beta * v without a sink, and
+    o = beta * v * e^x / (e^x + e^s) with one, x = <q~, k~> / sqrt(D)."""
+    D, Dv, Hq = 48, 32, 4
+    q, k, v = rnd(1, 1, Hq, D), rnd(1, 1, 1, D), rnd(1, 1, 1, Dv)
+    hidden = 1000
+    beta = math.sqrt(hidden / (Hq * Dv))
+    out = _layer(q, k, v, layer_type=0, num_kv_heads=1, rotary_dim=16, theta=1e4, window=0,
+                 sinks=None, hidden_size=hidden)
+    for h in range(Hq):
+        np.testing.assert_allclose(out[0, 0, h], beta * v[0, 0, 0], rtol=1e-14)
+    sinks = np.array([0.3, -2.0, 4.0, 0.0])
+    out = _layer(q, k, v, layer_type=1, num_kv_heads=1, rotary_dim=16, theta=1e4, window=3,
+                 sinks=sinks, hidden_size=hidden)
+    for h in range(Hq):
+        x = float(q[0, 0, h] @ k[0, 0, 0]) / math.sqrt(D)  # position 0: no rotation
+        w = math.exp(x) / (math.exp(x) + math.exp(sinks[h]))
+        np.testing.assert_allclose(out[0, 0, h], beta * w * v[0, 0, 0], rtol=1e-12)
+
+
+def test_zero_query_closed_form():
+    """q = 0 gives equal scores: o = beta * sum(v_visible) / (n + e^s)."""
+    S, D, Dv, W = 12, 16, 4, 5
+    q = np.zeros((1, S, 1, D))
+    k, v = rnd(1, S, 1, D), rnd(1, S, 1, Dv)
+    s = 1.3
+    out = _layer(q, k, v, layer_type=1, num_kv_heads=1, rotary_dim=8, theta=1e4, window=W,
+                 sinks=np.array([s]), hidden_size=4 * Dv)
+    beta = 2.0
+    for i in range(S):
+        lo = max(0, i - W + 1)
+        n = i - lo + 1
+        ref = beta * v[0, lo:i + 1, 0].sum(axis=0) / (n + math.exp(s))
+        np.testing.assert_allclose(out[0, i, 0], ref, rtol=1e-13, atol=1e-15)
+
+
+def test_v_scale_multiplies_output():
+    """hidden = Hq*Dv gives beta = 1; any other hidden scales the output by
+    sqrt(hidden/(Hq*Dv)) (a multiplication, not a division)."""
+    S, Hq, D, Dv = 20, 4, 48, 32
+    q, k, v = rnd(1, S, Hq, D), rnd(1, S, 2, D), rnd(1, S, 2, Dv)
+    kw = dict(layer_type=1, num_kv_heads=2, rotary_dim=16, theta=1e4, window=7,
+              sinks=np.array([0.1, 0.2, -0.3, 1.0]))
+    a = _layer(q, k, v, hidden_size=Hq * Dv, **kw)
+    b = _layer(q, k, v, hidden_size=9 * Hq * Dv, **kw)
+    np.testing.assert_allclose(b, 3.0 * a, rtol=1e-12, atol=1e-14)
+    assert oracle.v_scale(4096, 64, 128) == pytest.approx(math.sqrt(0.5))
+    assert oracle.v_scale(256, 4, 32) == pytest.approx(math.sqrt(2.0))
+
+
+def test_gqa_equals_replicated_mha():
+    """Replicating each KV head G times (contiguous grouping) and running MHA
+    gives the GQA result; catches a strided (h % Hkv) head mapping."""
+    S, Hq, Hkv, D, Dv = 24, 8, 2, 32, 16
+    q, k, v = rnd(1, S, Hq, D), rnd(1, S, Hkv, D), rnd(1, S, Hkv, Dv)
+    kw = dict(layer_type=1, rotary_dim=16, theta=1e4, window=9, sinks=rnd(Hq), hidden_size=512)
+    a = _layer(q, k, v, num_kv_heads=Hkv, **kw)
+    G = Hq // Hkv
+    b = _layer(q, np.repeat(k, G, axis=2), np.repeat(v, G, axis=2), num_kv_heads=Hq, **kw)
+    np.testing.assert_allclose(a, b, rtol=1e-14, atol=1e-15)
+
+
+def test_positions_shift_leaves_output_unchanged():
+    """Shifting every RoPE position by c changes nothing (relative property)."""
+    S, Hq, D, Dv = 30, 2, 48, 8
+    q, k, v = rnd(1, S, Hq, D), rnd(1, S, 1, D), rnd(1, S, 1, Dv)
+    kw = dict(layer_type=0, num_kv_heads=1, rotary_dim=16, theta=1e4, window=0, sinks=None,
+              hidden_size=64)
+    a = _layer(q, k, v, **kw)
+    b = _layer(q, k, v, positions=np.arange(S) + 4321.0, **kw)
+    np.testing.assert_allclose(a, b, rtol=1e-9, atol=1e-10)
+
+
+# ---------------------------------------------------------------- decode pins
+
+def _rotated_cache(k, v, L, cap, layer_type, window, r, theta):
+    """Cache holding positions 0..L-2 of k (rotated) / v, laid out per the
+    cache rule: slot p (global) or p mod window (ring)."""
+    kc = rnd(cap, k.shape[1])  # stale garbage in unused slots
+    vc = rnd(cap, v.shape[1])
+    for p in range(L - 1):
+        slot = p % window if layer_type == 1 else p
+        kc[slot] = oracle.rope(k[p], r, theta, p)
+        vc[slot] = v[p]
+    return kc, vc
+
+
+@pytest.mark.parametrize("layer_type,L,W", [(0, 1, 0), (0, 37, 0), (1, 1, 8), (1, 5, 8),
+                                           (1, 8, 8), (1, 9, 8), (1, 30, 8)])
+def test_decode_equals_prefill_last_row(layer_type, L, W):
+    """Decode of token L-1 equals row L-1 of prefill over L tokens. For the
+    ring this pins the W-slot ring (new token + W-1 previous) to the W-key
+    window of prefill."""
+    Hq, D, Dv, r, theta = 4, 48, 32, 16, 1e4
+    q, k, v = rnd(1, L, Hq, D), rnd(1, L, 1, D), rnd(1, L, 1, Dv)
+    sinks = rnd(Hq) if layer_type == 1 else None
+    pre = _layer(q, k, v, layer_type=layer_type, num_kv_heads=1, rotary_dim=r, theta=theta,
+                 window=W, sinks=sinks, hidden_size=256)
+    cap = W if layer_type == 1 else L + 3
+    kc, vc = _rotated_cache(k[0, :, 0], v[0, :, 0], L, cap, layer_type, W, r, theta)
+    out, kc2, vc2 = oracle.decode(q[0, L - 1], k[0, L - 1, 0], v[0, L - 1, 0], kc, vc, L, r, theta,
+                                  layer_type, W, 1 / math.sqrt(D), sinks, oracle.v_scale(256, Hq, Dv))
+    np.testing.assert_allclose(out, pre[0, L - 1], rtol=1e-12, atol=1e-13)
+    slot = (L - 1) % W if layer_type == 1 else L - 1
+    np.testing.assert_allclose(kc2[slot], oracle.rope(k[0, L - 1, 0], r, theta, L - 1), rtol=1e-15)
+    assert np.array_equal(vc2[slot], v[0, L - 1, 0])
+    others = [s for s in range(cap) if s != slot]
+    assert np.array_equal(kc2[others], kc[others]) and np.array_equal(vc2[others], vc[others])
+
+
+def test_decode_ring_slot_permutation_invariance():
+    """Softmax is order-free: permuting the ring slots that hold the W-1 older
+    positions leaves the output unchanged."""
+    W, L, D, Dv = 16, 50, 48, 32
+    q, kn, vn = rnd(2, D), rnd(D), rnd(Dv)
+    kc, vc = rnd(W, D), rnd(W, Dv)
+    args = (L, 16, 1e4, 1, W, 1 / math.sqrt(D), np.array([0.2, -1.0]), 0.5)
+    a, _, _ = oracle.decode(q, kn, vn, kc, vc, *args)
+    new_slot = (L - 1) % W
+    others = [s for s in range(W) if s != new_slot]
+    perm = list(others)
+    RNG.shuffle(perm)
+    kc2, vc2 = kc.copy(), vc.copy()
+    kc2[others] = kc[perm]
+    vc2[others] = vc[perm]
+    b, _, _ = oracle.decode(q, kn, vn, kc2, vc2, *args)
+    np.testing.assert_allclose(a, b, rtol=1e-13, atol=1e-14)
+
+
+def test_decode_rejects_bad_lengths():
+    D, Dv = 8, 4
+    with pytest.raises(ValueError):
+        oracle.decode(rnd(1, D), rnd(D), rnd(Dv), rnd(4, D), rnd(4, Dv), 5, 4, 1e4, 0, 0, 1.0, None, 1.0)
+    with pytest.raises(ValueError):
+        oracle.decode(rnd(1, D), rnd(D), rnd(Dv), rnd(4, D), rnd(4, Dv), 0, 4, 1e4, 0, 0, 1.0, None, 1.0)
+    with pytest.raises(ValueError):  # ring capacity must equal the window
+        oracle.decode(rnd(1, D), rnd(D), rnd(Dv), rnd(4, D), rnd(4, Dv), 3, 4, 1e4, 1, 5, 1.0, None, 1.0)
