@@ -1,0 +1,292 @@
+// C ABI of the MiMo-V2-Flash attention library (declared in include/mimo_attn.h).
+//
+// Host side only: argument checks (all before any launch), per-layer
+// parameter resolution (softmax scale, V scale sqrt(hidden/(Hq*Dv)), RoPE
+// inverse frequencies theta^(-2j/r) in double precision), workspace layout,
+// and the launches. No device memory is allocated here.
+#include "../../include/mimo_attn.h"
+#include "kernels.cuh"
+
+#include <math.h>
+#include <string.h>
+
+namespace {
+
+// Device error word: sticky bits set by kernels (kv_lens out of range, wait
+// timeouts). One copy per device, read by mimo_attn_get_device_error().
+__device__ unsigned g_device_error;
+
+int g_fail_launches = 0;
+
+constexpr int kMaxDevices = 64;
+unsigned *g_err_ptr[kMaxDevices];
+
+unsigned *device_error_ptr()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return nullptr;
+    if (g_err_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess)
+            return nullptr;
+        g_err_ptr[dev] = static_cast<unsigned *>(p);
+    }
+    return g_err_ptr[dev];
+}
+
+size_t elem_size(int dtype) { return dtype == MIMO_ATTN_BF16 ? 2 : 4; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validates the per-layer struct; fills the resolved arguments.
+mimo_attn_status resolve_layer(const mimo_attn_layer *layer, int dtype, mimo::LayerArgs *out)
+{
+    if (layer == nullptr)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (dtype != MIMO_ATTN_BF16 && dtype != MIMO_ATTN_FP32)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    const mimo_attn_layer &l = *layer;
+    if (l.layer_type != MIMO_ATTN_GLOBAL && l.layer_type != MIMO_ATTN_SWA)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (l.num_q_heads < 1 || l.num_kv_heads < 1 || l.num_q_heads % l.num_kv_heads != 0)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (l.qk_dim < 2 || l.v_dim < 1 || (l.qk_dim % 2) != 0)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (l.rotary_dim < 0 || l.rotary_dim > l.qk_dim || (l.rotary_dim % 2) != 0)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (l.layer_type == MIMO_ATTN_SWA && l.window < 1)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (l.layer_type == MIMO_ATTN_GLOBAL && l.sinks != nullptr)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (l.hidden_size < 1 || !(l.rope_theta > 0.0) || !isfinite(l.rope_theta))
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (!(l.softmax_scale >= 0.f) || !isfinite(l.softmax_scale))
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (l.qk_dim > 256 || l.v_dim > 256)
+        return MIMO_ATTN_ERR_UNSUPPORTED;
+
+    mimo::LayerArgs &L = *out;
+    memset(&L, 0, sizeof(L));
+    L.layer_type = l.layer_type;
+    L.Hq = l.num_q_heads;
+    L.Hkv = l.num_kv_heads;
+    L.G = l.num_q_heads / l.num_kv_heads;
+    L.Dqk = l.qk_dim;
+    L.Dv = l.v_dim;
+    L.window = l.layer_type == MIMO_ATTN_SWA ? l.window : 0;
+    const double scale = l.softmax_scale > 0.f ? (double)l.softmax_scale : 1.0 / sqrt((double)l.qk_dim);
+    L.scale_log2 = (float)(scale * 1.4426950408889634074);
+    L.v_scale = (float)sqrt((double)l.hidden_size / ((double)l.num_q_heads * (double)l.v_dim));
+    L.sinks = l.sinks;
+    L.rope.rotary_dim = l.rotary_dim;
+    L.rope.half = l.rotary_dim / 2;
+    for (int j = 0; j < L.rope.half; ++j)
+        L.rope.inv_freq[j] = pow(l.rope_theta, -2.0 * (double)j / (double)l.rotary_dim);
+    return MIMO_ATTN_OK;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+} // namespace
+
+extern "C" {
+
+int mimo_attn_rotary_dim(double partial_rotary_factor, int qk_dim)
+{
+    const double r = partial_rotary_factor * (double)qk_dim;
+    if (!isfinite(r) || r < 0.0 || r > 2147483647.0)
+        return -1;
+    return (int)r;  // truncation toward zero: Python int() of a non-negative float
+}
+
+size_t mimo_attn_prefill_workspace_size(const mimo_attn_layer *layer, int dtype, int batch, int seq)
+{
+    mimo::LayerArgs L;
+    if (resolve_layer(layer, dtype, &L) != MIMO_ATTN_OK || batch < 0 || seq < 0)
+        return 0;
+    return round_up((size_t)batch * seq * L.Hkv * L.Dqk * elem_size(dtype), 256);
+}
+
+mimo_attn_status mimo_attn_prefill(const mimo_attn_layer *layer, int dtype, int batch, int seq,
+                                   const void *q, const void *k, const void *v,
+                                   const int32_t *positions, void *out, void *k_cache,
+                                   void *v_cache, int cache_capacity, void *workspace,
+                                   size_t workspace_bytes, void *stream)
+{
+    mimo::LayerArgs L;
+    mimo_attn_status st = resolve_layer(layer, dtype, &L);
+    if (st != MIMO_ATTN_OK)
+        return st;
+    if (batch < 0 || seq < 0)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if ((k_cache == nullptr) != (v_cache == nullptr))
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    const bool has_cache = k_cache != nullptr;
+    if (has_cache) {
+        if (L.layer_type == MIMO_ATTN_SWA && cache_capacity != L.window)
+            return MIMO_ATTN_ERR_INVALID_ARG;
+        if (L.layer_type == MIMO_ATTN_GLOBAL && cache_capacity < seq)
+            return MIMO_ATTN_ERR_INVALID_ARG;
+    }
+    if (batch == 0 || seq == 0)
+        return MIMO_ATTN_OK;
+    if (q == nullptr || k == nullptr || v == nullptr || out == nullptr)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (dtype == MIMO_ATTN_BF16 &&
+        !(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out) && aligned16(k_cache) &&
+          aligned16(v_cache) && aligned16(workspace)))
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    // Rotated keys go straight into a global cache; otherwise to the workspace.
+    const bool keys_in_cache = has_cache && L.layer_type == MIMO_ATTN_GLOBAL;
+    const size_t need = keys_in_cache ? 0 : mimo_attn_prefill_workspace_size(layer, dtype, batch, seq);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+        return MIMO_ATTN_ERR_WORKSPACE;
+    if (g_fail_launches)
+        return MIMO_ATTN_ERR_CUDA;
+    unsigned *err = device_error_ptr();
+    if (err == nullptr)
+        return MIMO_ATTN_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    mimo::KprepArgs kp;
+    memset(&kp, 0, sizeof(kp));
+    kp.k = k;
+    kp.v = v;
+    kp.positions = positions;
+    kp.dst_k = keys_in_cache ? k_cache : workspace;
+    kp.dst_rows = keys_in_cache ? cache_capacity : seq;
+    if (has_cache && L.layer_type == MIMO_ATTN_SWA) {
+        kp.ring_k = k_cache;
+        kp.ring_v = v_cache;
+    }
+    if (keys_in_cache) {
+        kp.lin_v = v_cache;
+        kp.lin_rows = cache_capacity;
+    }
+    kp.B = batch;
+    kp.S = seq;
+    kp.Hkv = L.Hkv;
+    kp.Dqk = L.Dqk;
+    kp.Dv = L.Dv;
+    kp.window = L.layer_type == MIMO_ATTN_SWA ? L.window : 0;
+    kp.rope = L.rope;
+    if (mimo::launch_kprep(kp, dtype, s) != cudaSuccess)
+        return MIMO_ATTN_ERR_CUDA;
+
+    mimo::PrefillArgs pa;
+    pa.q = q;
+    pa.krot = kp.dst_k;
+    pa.krot_rows = kp.dst_rows;
+    pa.v = v;
+    pa.positions = positions;
+    pa.out = out;
+    pa.B = batch;
+    pa.S = seq;
+    pa.err = err;
+    cudaError_t e;
+    if (dtype == MIMO_ATTN_BF16 && mimo::prefill_tc_supported(L))
+        e = mimo::launch_prefill_tc(L, pa, s);
+    else
+        e = mimo::launch_prefill_simt(L, pa, dtype, s);
+    return e == cudaSuccess ? MIMO_ATTN_OK : MIMO_ATTN_ERR_CUDA;
+}
+
+size_t mimo_attn_decode_workspace_size(const mimo_attn_layer *layer, int dtype, int batch,
+                                       int cache_capacity)
+{
+    mimo::LayerArgs L;
+    if (resolve_layer(layer, dtype, &L) != MIMO_ATTN_OK || batch < 0 || cache_capacity < 1)
+        return 0;
+    const int splits = mimo::decode_max_splits(L, dtype, cache_capacity);
+    if (splits <= 1)
+        return 0;
+    return round_up((size_t)batch * L.Hq * splits * (L.Dv + 2) * sizeof(float), 256);
+}
+
+mimo_attn_status mimo_attn_decode(const mimo_attn_layer *layer, int dtype, int batch,
+                                  const void *q, const void *k_new, const void *v_new,
+                                  const int32_t *kv_lens, void *k_cache, void *v_cache,
+                                  int cache_capacity, void *out, void *workspace,
+                                  size_t workspace_bytes, void *stream)
+{
+    mimo::LayerArgs L;
+    mimo_attn_status st = resolve_layer(layer, dtype, &L);
+    if (st != MIMO_ATTN_OK)
+        return st;
+    if (batch < 0 || cache_capacity < 1)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (L.layer_type == MIMO_ATTN_SWA && cache_capacity != L.window)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (batch == 0)
+        return MIMO_ATTN_OK;
+    if (q == nullptr || k_new == nullptr || v_new == nullptr || kv_lens == nullptr ||
+        k_cache == nullptr || v_cache == nullptr || out == nullptr)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (dtype == MIMO_ATTN_BF16 &&
+        !(aligned16(q) && aligned16(k_new) && aligned16(v_new) && aligned16(k_cache) &&
+          aligned16(v_cache) && aligned16(out)))
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    const size_t need = mimo_attn_decode_workspace_size(layer, dtype, batch, cache_capacity);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+        return MIMO_ATTN_ERR_WORKSPACE;
+    if (g_fail_launches)
+        return MIMO_ATTN_ERR_CUDA;
+    unsigned *err = device_error_ptr();
+    if (err == nullptr)
+        return MIMO_ATTN_ERR_CUDA;
+
+    mimo::DecodeArgs da;
+    da.q = q;
+    da.k_new = k_new;
+    da.v_new = v_new;
+    da.kv_lens = kv_lens;
+    da.k_cache = k_cache;
+    da.v_cache = v_cache;
+    da.cap = cache_capacity;
+    da.out = out;
+    da.partial = static_cast<float *>(workspace);
+    da.max_splits = mimo::decode_max_splits(L, dtype, cache_capacity);
+    da.chunk = mimo::decode_chunk_keys(L, dtype);
+    da.B = batch;
+    da.err = err;
+    cudaError_t e = mimo::launch_decode(L, da, dtype, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MIMO_ATTN_OK : MIMO_ATTN_ERR_CUDA;
+}
+
+mimo_attn_status mimo_attn_get_device_error(uint32_t *bits)
+{
+    if (bits == nullptr)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    unsigned host = 0;
+    const unsigned zero = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpyFromSymbol(&host, g_device_error, sizeof(host)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+        return MIMO_ATTN_ERR_CUDA;
+    *bits = host;
+    return MIMO_ATTN_OK;
+}
+
+const char *mimo_attn_status_string(mimo_attn_status status)
+{
+    switch (status) {
+    case MIMO_ATTN_OK:
+        return "ok";
+    case MIMO_ATTN_ERR_INVALID_ARG:
+        return "invalid argument";
+    case MIMO_ATTN_ERR_UNSUPPORTED:
+        return "unsupported configuration";
+    case MIMO_ATTN_ERR_WORKSPACE:
+        return "workspace missing or too small";
+    case MIMO_ATTN_ERR_CUDA:
+        return "CUDA error";
+    }
+    return "unknown status";
+}
+
+void mimo_attn_debug_fail_launches(int enable) { g_fail_launches = enable != 0; }
+
+const char *mimo_attn_version(void) { return "mimo_attn 0.1.0 (sm_100a)"; }
+
+} // extern "C"

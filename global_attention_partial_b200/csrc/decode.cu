@@ -1,0 +1,593 @@
+// Decode attention of one MiMo-V2-Flash layer: one new token per sequence.
+//
+// bf16, Dqk 192, Dv 128, G <= 16 query heads per KV head: split-KV kernel.
+//   grid (split, kv head, batch); 4 warps. The CTA rotates the G query heads
+//   of its KV group at position L-1 (partial RoPE) into shared memory; the CTA
+//   whose key range holds the new token's slot also rotates the new key,
+//   writes key and value into the cache slot (L-1 for a global cache,
+//   (L-1) mod window for a sliding-window ring) and uses its own copy.
+//   K/V tiles of 64 keys stream through a two-stage cp.async pipeline with
+//   16-byte coalesced loads; each warp takes 16 keys of a tile and runs
+//   S = Q K^T and O += P V on mma.sync m16n8k16 (query heads on M, keys on
+//   N), with the row max / sum reduced by warp shuffles. Warps are merged
+//   through shared memory; a sequence with one split is finished in place
+//   (sink folded, V scale applied), otherwise the (m, l, O) partials go to the
+//   workspace and a combine kernel merges them.
+// Other dtypes / dims: a CUDA-core path (one warp per query head) after a
+// separate new-token write.
+#include "kernels.cuh"
+
+#include <math.h>
+
+namespace mimo {
+namespace {
+
+constexpr int kDqk = 192;
+constexpr int kDv = 128;
+constexpr int kThreads = 128;
+constexpr int kTileKeys = 64;
+constexpr int kStages = 2;
+constexpr int kKStride = kDqk + 8;  // elements; 400-byte rows keep ldmatrix conflict-free
+constexpr int kVStride = kDv + 8;   // 272-byte rows
+constexpr int kQStride = kDqk + 8;
+constexpr int kChunkKeys = 1024;    // keys per split on global layers
+constexpr int kStageElems = kTileKeys * (kKStride + kVStride);
+constexpr int kSmemBytes = (16 * kQStride + kStages * kStageElems + kDqk + kDv) * 2;
+
+struct DecodeSmem {
+    float wm[4][16];
+    float wl[4][16];
+    float o[16][kDv];
+};
+
+__device__ __forceinline__ int visible_count(int layer_type, int Lb, int window)
+{
+    return layer_type == 1 ? min(Lb, window) : Lb;
+}
+
+__device__ __forceinline__ bool kv_len_ok(int layer_type, int Lb, int cap)
+{
+    return Lb >= 1 && (layer_type == 1 || Lb <= cap);
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+    decode_mma_kernel(const __grid_constant__ LayerArgs L, const __grid_constant__ DecodeArgs a)
+{
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    __nv_bfloat16 *sQ = reinterpret_cast<__nv_bfloat16 *>(smem_raw);
+    __nv_bfloat16 *sStage = sQ + 16 * kQStride;
+    __nv_bfloat16 *sKnew = sStage + kStages * kStageElems;
+    __nv_bfloat16 *sVnew = sKnew + kDqk;
+    __shared__ DecodeSmem red;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int split = blockIdx.x;
+    const int kvh = blockIdx.y;
+    const int b = blockIdx.z;
+    const int Lb = __ldg(a.kv_lens + b);
+    if (!kv_len_ok(L.layer_type, Lb, a.cap)) {
+        if (split == 0 && kvh == 0 && tid == 0)
+            atomicOr(a.err, kErrKvLen);
+        return;
+    }
+    const int n_vis = visible_count(L.layer_type, Lb, L.window);
+    const int nsplit = (n_vis + a.chunk - 1) / a.chunk;
+    if (split >= nsplit)
+        return;
+    const int key_begin = split * a.chunk;
+    const int key_end = min(n_vis, key_begin + a.chunk);
+    const int slot_new = L.layer_type == 1 ? (Lb - 1) % L.window : Lb - 1;
+    const bool owns_new = slot_new >= key_begin && slot_new < key_end;
+    const double pos = (double)(Lb - 1);
+    const int G = L.G;
+    const int half = L.rope.half;
+
+    const size_t kv_row = (size_t)L.Hkv;  // rows of the cache are [slot][Hkv][D]
+    const __nv_bfloat16 *kc = reinterpret_cast<const __nv_bfloat16 *>(a.k_cache) +
+                              ((size_t)b * a.cap * kv_row + kvh) * kDqk;
+    const __nv_bfloat16 *vc = reinterpret_cast<const __nv_bfloat16 *>(a.v_cache) +
+                              ((size_t)b * a.cap * kv_row + kvh) * kDv;
+
+    // Query heads of this KV group, rotated at position L-1 (rows >= G are 0).
+    {
+        const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(a.q) +
+                                  ((size_t)b * L.Hq + (size_t)kvh * G) * kDqk;
+        for (int idx = tid; idx < 16 * kDqk; idx += kThreads) {
+            const int r = idx / kDqk;
+            const int e = idx - r * kDqk;
+            float y = 0.f;
+            if (r < G) {
+                const __nv_bfloat16 *qr = qg + (size_t)r * kDqk;
+                if (e < L.rope.rotary_dim) {
+                    const int j = e < half ? e : e - half;
+                    float c, s;
+                    rope_cos_sin(pos, L.rope.inv_freq[j], c, s);
+                    const float xa = __bfloat162float(qr[j]);
+                    const float xb = __bfloat162float(qr[j + half]);
+                    y = e < half ? xa * c - xb * s : xb * c + xa * s;
+                } else {
+                    y = __bfloat162float(qr[e]);
+                }
+            }
+            sQ[r * kQStride + e] = __float2bfloat16_rn(y);
+        }
+    }
+    // New token: rotate k, write k and v into the cache slot, keep a copy.
+    if (owns_new) {
+        const __nv_bfloat16 *kn = reinterpret_cast<const __nv_bfloat16 *>(a.k_new) +
+                                  ((size_t)b * L.Hkv + kvh) * kDqk;
+        const __nv_bfloat16 *vn = reinterpret_cast<const __nv_bfloat16 *>(a.v_new) +
+                                  ((size_t)b * L.Hkv + kvh) * kDv;
+        __nv_bfloat16 *kdst = reinterpret_cast<__nv_bfloat16 *>(a.k_cache) +
+                              (((size_t)b * a.cap + slot_new) * kv_row + kvh) * kDqk;
+        __nv_bfloat16 *vdst = reinterpret_cast<__nv_bfloat16 *>(a.v_cache) +
+                              (((size_t)b * a.cap + slot_new) * kv_row + kvh) * kDv;
+        for (int e = tid; e < kDqk; e += kThreads) {
+            float y;
+            if (e < L.rope.rotary_dim) {
+                const int j = e < half ? e : e - half;
+                float c, s;
+                rope_cos_sin(pos, L.rope.inv_freq[j], c, s);
+                const float xa = __bfloat162float(kn[j]);
+                const float xb = __bfloat162float(kn[j + half]);
+                y = e < half ? xa * c - xb * s : xb * c + xa * s;
+            } else {
+                y = __bfloat162float(kn[e]);
+            }
+            const __nv_bfloat16 yb = __float2bfloat16_rn(y);
+            sKnew[e] = yb;
+            kdst[e] = yb;
+        }
+        for (int e = tid; e < kDv; e += kThreads) {
+            const __nv_bfloat16 x = vn[e];
+            sVnew[e] = x;
+            vdst[e] = x;
+        }
+    }
+    __syncthreads();
+
+    // Query fragments (A operand, 16 heads x 192) for the 12 k-steps.
+    uint32_t qa[12][4];
+    {
+        const int mi = lane >> 3;
+        const int r = (lane & 7) + (mi & 1) * 8;
+        const uint32_t base = smem_u32(sQ) + (uint32_t)(r * kQStride + (mi >> 1) * 8) * 2u;
+#pragma unroll
+        for (int ks = 0; ks < 12; ++ks)
+            ldmatrix_x4(base + ks * 32, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
+    }
+
+    const int n_tiles = (key_end - key_begin + kTileKeys - 1) / kTileKeys;
+    auto issue = [&](int t) {
+        __nv_bfloat16 *st = sStage + (t % kStages) * kStageElems;
+        const int base_key = key_begin + t * kTileKeys;
+        for (int c = tid; c < kTileKeys * 40; c += kThreads) {
+            const int r = c / 40;
+            const int ch = c - r * 40;
+            const int key = base_key + r;
+            const bool valid = key < key_end && key != slot_new;
+            const int ks = valid ? key : key_begin;
+            if (ch < 24) {
+                cp_async16(st + r * kKStride + ch * 8, kc + (size_t)ks * kv_row * kDqk + ch * 8,
+                           valid ? 16u : 0u);
+            } else {
+                const int cv = ch - 24;
+                cp_async16(st + kTileKeys * kKStride + r * kVStride + cv * 8,
+                           vc + (size_t)ks * kv_row * kDv + cv * 8, valid ? 16u : 0u);
+            }
+        }
+    };
+#pragma unroll
+    for (int s = 0; s < kStages - 1; ++s) {
+        if (s < n_tiles)
+            issue(s);
+        cp_async_commit();
+    }
+
+    const int g = lane >> 2;  // row (head) g and g + 8
+    const int tq = lane & 3;
+    float m0 = -INFINITY, m1 = -INFINITY;  // running max of rows g, g+8 (base 2)
+    float l0 = 0.f, l1 = 0.f;              // this thread's partial sums
+    float o[16][4];
+#pragma unroll
+    for (int d = 0; d < 16; ++d)
+        o[d][0] = o[d][1] = o[d][2] = o[d][3] = 0.f;
+
+    for (int t = 0; t < n_tiles; ++t) {
+        cp_async_wait<kStages - 2>();
+        __syncthreads();
+        __nv_bfloat16 *st = sStage + (t % kStages) * kStageElems;
+        const int base_key = key_begin + t * kTileKeys;
+        if (owns_new && slot_new >= base_key && slot_new < base_key + kTileKeys) {
+            const int r = slot_new - base_key;
+            if (tid < 24)
+                *reinterpret_cast<uint4 *>(st + r * kKStride + tid * 8) =
+                    *reinterpret_cast<const uint4 *>(sKnew + tid * 8);
+            else if (tid < 40)
+                *reinterpret_cast<uint4 *>(st + kTileKeys * kKStride + r * kVStride + (tid - 24) * 8) =
+                    *reinterpret_cast<const uint4 *>(sVnew + (tid - 24) * 8);
+            __syncthreads();
+        }
+        if (t + kStages - 1 < n_tiles)
+            issue(t + kStages - 1);
+        cp_async_commit();
+
+        const int kb = warp * 16;  // this warp's 16 keys within the tile
+        if (base_key + kb >= key_end)
+            continue;
+        // S = Q K^T for 16 heads x 16 keys.
+        float s_acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        {
+            const int mi = lane >> 3;
+            const int key = kb + (mi >> 1) * 8 + (lane & 7);
+            const uint32_t base = smem_u32(st) + (uint32_t)(key * kKStride + (mi & 1) * 8) * 2u;
+#pragma unroll
+            for (int ks = 0; ks < 12; ++ks) {
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4(base + ks * 32, b0, b1, b2, b3);
+                mma_bf16_16816(s_acc[0], qa[ks], b0, b1);
+                mma_bf16_16816(s_acc[1], qa[ks], b2, b3);
+            }
+        }
+        // Scale, mask keys past the end of the range, online softmax.
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int key = base_key + kb + nt * 8 + 2 * tq + e;
+                const bool valid = key < key_end;
+                s_acc[nt][e] = valid ? s_acc[nt][e] * L.scale_log2 : -INFINITY;
+                s_acc[nt][2 + e] = valid ? s_acc[nt][2 + e] * L.scale_log2 : -INFINITY;
+                mx0 = fmaxf(mx0, s_acc[nt][e]);
+                mx1 = fmaxf(mx1, s_acc[nt][2 + e]);
+            }
+        }
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        const float mn0 = fmaxf(m0, mx0);
+        const float mn1 = fmaxf(m1, mx1);
+        const float c0 = (mn0 == -INFINITY) ? 1.f : exp2f(m0 - mn0);
+        const float c1 = (mn1 == -INFINITY) ? 1.f : exp2f(m1 - mn1);
+        const float u0 = (mn0 == -INFINITY) ? 0.f : mn0;
+        const float u1 = (mn1 == -INFINITY) ? 0.f : mn1;
+        m0 = mn0;
+        m1 = mn1;
+        float p[2][4];
+        float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            p[nt][0] = exp2f(s_acc[nt][0] - u0);
+            p[nt][1] = exp2f(s_acc[nt][1] - u0);
+            p[nt][2] = exp2f(s_acc[nt][2] - u1);
+            p[nt][3] = exp2f(s_acc[nt][3] - u1);
+            rs0 += p[nt][0] + p[nt][1];
+            rs1 += p[nt][2] + p[nt][3];
+        }
+        l0 = l0 * c0 + rs0;
+        l1 = l1 * c1 + rs1;
+#pragma unroll
+        for (int d = 0; d < 16; ++d) {
+            o[d][0] *= c0;
+            o[d][1] *= c0;
+            o[d][2] *= c1;
+            o[d][3] *= c1;
+        }
+        uint32_t pa[4];
+        pa[0] = pack_bf16x2(p[0][0], p[0][1]);
+        pa[1] = pack_bf16x2(p[0][2], p[0][3]);
+        pa[2] = pack_bf16x2(p[1][0], p[1][1]);
+        pa[3] = pack_bf16x2(p[1][2], p[1][3]);
+        // O += P V over these 16 keys.
+        {
+            const int mi = lane >> 3;
+            const int key = kb + (mi & 1) * 8 + (lane & 7);
+            const uint32_t base = smem_u32(st + kTileKeys * kKStride) +
+                                  (uint32_t)(key * kVStride + (mi >> 1) * 8) * 2u;
+#pragma unroll
+            for (int dp = 0; dp < 8; ++dp) {
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4_trans(base + dp * 32, b0, b1, b2, b3);
+                mma_bf16_16816(o[2 * dp], pa, b0, b1);
+                mma_bf16_16816(o[2 * dp + 1], pa, b2, b3);
+            }
+        }
+    }
+    cp_async_wait<0>();
+
+    // Merge the four warps.
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    if (tq == 0) {
+        red.wm[warp][g] = m0;
+        red.wm[warp][g + 8] = m1;
+        red.wl[warp][g] = l0;
+        red.wl[warp][g + 8] = l1;
+    }
+    for (int idx = tid; idx < 16 * kDv; idx += kThreads)
+        (&red.o[0][0])[idx] = 0.f;
+    __syncthreads();
+    float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        M0 = fmaxf(M0, red.wm[w][g]);
+        M1 = fmaxf(M1, red.wm[w][g + 8]);
+    }
+    const float f0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M0);
+    const float f1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M1);
+    for (int w = 0; w < 4; ++w) {
+        if (warp == w) {
+#pragma unroll
+            for (int d = 0; d < 16; ++d) {
+                const int col = d * 8 + 2 * tq;
+                red.o[g][col] += o[d][0] * f0;
+                red.o[g][col + 1] += o[d][1] * f0;
+                red.o[g + 8][col] += o[d][2] * f1;
+                red.o[g + 8][col + 1] += o[d][3] * f1;
+            }
+        }
+        __syncthreads();
+    }
+
+    // Row r = query head kvh*G + r; thread -> (row, 16 columns).
+    for (int idx = tid; idx < G * (kDv / 16); idx += kThreads) {
+        const int r = idx / (kDv / 16);
+        const int c0 = (idx % (kDv / 16)) * 16;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+            M = fmaxf(M, red.wm[w][r]);
+        float Ls = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+            Ls += (red.wm[w][r] == -INFINITY) ? 0.f : red.wl[w][r] * exp2f(red.wm[w][r] - M);
+        const int h = kvh * G + r;
+        if (nsplit == 1) {
+            float scale;
+            if (L.sinks != nullptr) {
+                const float s2 = __ldg(L.sinks + h) * kLog2e;
+                const float mf = fmaxf(M, s2);
+                const float al = exp2f(M - mf);
+                scale = al * L.v_scale / (Ls * al + exp2f(s2 - mf));
+            } else {
+                scale = L.v_scale / Ls;
+            }
+            __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.out) + ((size_t)b * L.Hq + h) * kDv + c0;
+            uint4 w0, w1;
+            w0.x = pack_bf16x2(red.o[r][c0 + 0] * scale, red.o[r][c0 + 1] * scale);
+            w0.y = pack_bf16x2(red.o[r][c0 + 2] * scale, red.o[r][c0 + 3] * scale);
+            w0.z = pack_bf16x2(red.o[r][c0 + 4] * scale, red.o[r][c0 + 5] * scale);
+            w0.w = pack_bf16x2(red.o[r][c0 + 6] * scale, red.o[r][c0 + 7] * scale);
+            w1.x = pack_bf16x2(red.o[r][c0 + 8] * scale, red.o[r][c0 + 9] * scale);
+            w1.y = pack_bf16x2(red.o[r][c0 + 10] * scale, red.o[r][c0 + 11] * scale);
+            w1.z = pack_bf16x2(red.o[r][c0 + 12] * scale, red.o[r][c0 + 13] * scale);
+            w1.w = pack_bf16x2(red.o[r][c0 + 14] * scale, red.o[r][c0 + 15] * scale);
+            reinterpret_cast<uint4 *>(dst)[0] = w0;
+            reinterpret_cast<uint4 *>(dst)[1] = w1;
+        } else {
+            float *part = a.partial + (((size_t)b * L.Hq + h) * a.max_splits + split) * (kDv + 2);
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                part[c0 + c] = red.o[r][c0 + c];
+            if (c0 == 0) {
+                part[kDv] = M;
+                part[kDv + 1] = Ls;
+            }
+        }
+    }
+}
+
+// Merges the split partials of one (batch, query head): log-sum-exp merge,
+// sink folded into the denominator, V scale applied.
+template <typename T>
+__global__ void decode_combine_kernel(const __grid_constant__ LayerArgs L, const __grid_constant__ DecodeArgs a)
+{
+    const int h = blockIdx.x;
+    const int b = blockIdx.y;
+    const int Lb = __ldg(a.kv_lens + b);
+    if (!kv_len_ok(L.layer_type, Lb, a.cap))
+        return;
+    const int n_vis = visible_count(L.layer_type, Lb, L.window);
+    const int nsplit = (n_vis + a.chunk - 1) / a.chunk;
+    if (nsplit <= 1)
+        return;
+    const float *part = a.partial + ((size_t)b * L.Hq + h) * a.max_splits * (L.Dv + 2);
+    float M = -INFINITY;
+    for (int s = 0; s < nsplit; ++s)
+        M = fmaxf(M, part[(size_t)s * (L.Dv + 2) + L.Dv]);
+    float s2 = -INFINITY;
+    if (L.sinks != nullptr) {
+        s2 = __ldg(L.sinks + h) * kLog2e;
+        M = fmaxf(M, s2);
+    }
+    float Ls = (L.sinks != nullptr) ? exp2f(s2 - M) : 0.f;
+    for (int s = 0; s < nsplit; ++s) {
+        const float *ps = part + (size_t)s * (L.Dv + 2);
+        Ls += ps[L.Dv + 1] * exp2f(ps[L.Dv] - M);
+    }
+    const float scale = L.v_scale / Ls;
+    for (int e = threadIdx.x; e < L.Dv; e += blockDim.x) {
+        float acc = 0.f;
+        for (int s = 0; s < nsplit; ++s) {
+            const float *ps = part + (size_t)s * (L.Dv + 2);
+            acc += ps[e] * exp2f(ps[L.Dv] - M);
+        }
+        reinterpret_cast<T *>(a.out)[((size_t)b * L.Hq + h) * L.Dv + e] = from_f32<T>(acc * scale);
+    }
+}
+
+// ------------------------------------------------------- CUDA-core path
+// Writes the new token (rotated key, value) into its cache slot.
+template <typename T>
+__global__ void decode_write_new_kernel(const __grid_constant__ LayerArgs L, const __grid_constant__ DecodeArgs a)
+{
+    const int kvh = blockIdx.x;
+    const int b = blockIdx.y;
+    const int Lb = __ldg(a.kv_lens + b);
+    if (!kv_len_ok(L.layer_type, Lb, a.cap)) {
+        if (kvh == 0 && threadIdx.x == 0)
+            atomicOr(a.err, kErrKvLen);
+        return;
+    }
+    const int slot = L.layer_type == 1 ? (Lb - 1) % L.window : Lb - 1;
+    const double pos = (double)(Lb - 1);
+    const int half = L.rope.half;
+    const T *kn = reinterpret_cast<const T *>(a.k_new) + ((size_t)b * L.Hkv + kvh) * L.Dqk;
+    const T *vn = reinterpret_cast<const T *>(a.v_new) + ((size_t)b * L.Hkv + kvh) * L.Dv;
+    T *kd = reinterpret_cast<T *>(a.k_cache) + (((size_t)b * a.cap + slot) * L.Hkv + kvh) * L.Dqk;
+    T *vd = reinterpret_cast<T *>(a.v_cache) + (((size_t)b * a.cap + slot) * L.Hkv + kvh) * L.Dv;
+    for (int e = threadIdx.x; e < L.Dqk; e += blockDim.x) {
+        float y;
+        if (e < L.rope.rotary_dim) {
+            const int j = e < half ? e : e - half;
+            float c, s;
+            rope_cos_sin(pos, L.rope.inv_freq[j], c, s);
+            const float xa = to_f32<T>(kn[j]);
+            const float xb = to_f32<T>(kn[j + half]);
+            y = e < half ? xa * c - xb * s : xb * c + xa * s;
+        } else {
+            y = to_f32<T>(kn[e]);
+        }
+        kd[e] = from_f32<T>(y);
+    }
+    for (int e = threadIdx.x; e < L.Dv; e += blockDim.x)
+        vd[e] = vn[e];
+}
+
+// One warp per (batch, query head) over the visible cache slots.
+template <typename T>
+__global__ void decode_simt_kernel(const __grid_constant__ LayerArgs L, const __grid_constant__ DecodeArgs a)
+{
+    __shared__ float qs[4][256];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int h = blockIdx.x * 4 + warp;
+    const int b = blockIdx.y;
+    if (h >= L.Hq)
+        return;
+    const int Lb = __ldg(a.kv_lens + b);
+    if (!kv_len_ok(L.layer_type, Lb, a.cap))
+        return;
+    const int n_vis = visible_count(L.layer_type, Lb, L.window);
+    const double pos = (double)(Lb - 1);
+    const int half = L.rope.half;
+    const T *q = reinterpret_cast<const T *>(a.q) + ((size_t)b * L.Hq + h) * L.Dqk;
+    for (int e = lane; e < L.Dqk; e += 32) {
+        float y;
+        if (e < L.rope.rotary_dim) {
+            const int j = e < half ? e : e - half;
+            float c, s;
+            rope_cos_sin(pos, L.rope.inv_freq[j], c, s);
+            const float xa = to_f32<T>(q[j]);
+            const float xb = to_f32<T>(q[j + half]);
+            y = e < half ? xa * c - xb * s : xb * c + xa * s;
+        } else {
+            y = to_f32<T>(q[e]);
+        }
+        qs[warp][e] = y;
+    }
+    __syncwarp();
+    const int kvh = h / L.G;
+    float m = -INFINITY, l = 0.f;
+    float acc[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+        acc[t] = 0.f;
+    for (int slot = 0; slot < n_vis; ++slot) {
+        const T *kr = reinterpret_cast<const T *>(a.k_cache) + (((size_t)b * a.cap + slot) * L.Hkv + kvh) * L.Dqk;
+        float part = 0.f;
+        for (int e = lane; e < L.Dqk; e += 32)
+            part += qs[warp][e] * to_f32<T>(kr[e]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            part += __shfl_xor_sync(0xffffffffu, part, off);
+        const float x = part * L.scale_log2;
+        const float mn = fmaxf(m, x);
+        const float c = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+        const float pj = exp2f(x - mn);
+        l = l * c + pj;
+        const T *vr = reinterpret_cast<const T *>(a.v_cache) + (((size_t)b * a.cap + slot) * L.Hkv + kvh) * L.Dv;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const int e = lane + 32 * t;
+            if (e < L.Dv)
+                acc[t] = acc[t] * c + pj * to_f32<T>(vr[e]);
+        }
+        m = mn;
+    }
+    float scale;
+    if (L.sinks != nullptr) {
+        const float s2 = __ldg(L.sinks + h) * kLog2e;
+        const float mf = fmaxf(m, s2);
+        const float al = exp2f(m - mf);
+        scale = al * L.v_scale / (l * al + exp2f(s2 - mf));
+    } else {
+        scale = L.v_scale / l;
+    }
+    T *dst = reinterpret_cast<T *>(a.out) + ((size_t)b * L.Hq + h) * L.Dv;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+        const int e = lane + 32 * t;
+        if (e < L.Dv)
+            dst[e] = from_f32<T>(acc[t] * scale);
+    }
+}
+
+bool decode_mma_supported(const LayerArgs &L, int dtype)
+{
+    return dtype == kDtypeBf16 && L.Dqk == kDqk && L.Dv == kDv && L.G >= 1 && L.G <= 16;
+}
+
+} // namespace
+
+int decode_chunk_keys(const LayerArgs &L, int dtype)
+{
+    if (!decode_mma_supported(L, dtype))
+        return 1 << 30;
+    return L.layer_type == 1 ? max(L.window, 1) : kChunkKeys;
+}
+
+int decode_max_splits(const LayerArgs &L, int dtype, int cap)
+{
+    const int chunk = decode_chunk_keys(L, dtype);
+    return (cap + chunk - 1) / chunk;
+}
+
+cudaError_t launch_decode(const LayerArgs &L, const DecodeArgs &a, int dtype, cudaStream_t stream)
+{
+    if (decode_mma_supported(L, dtype)) {
+        static bool attr_set = false;
+        if (!attr_set) {
+            cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            if (e != cudaSuccess)
+                return e;
+            attr_set = true;
+        }
+        dim3 grid(a.max_splits, L.Hkv, a.B);
+        decode_mma_kernel<<<grid, kThreads, kSmemBytes, stream>>>(L, a);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess || a.max_splits <= 1)
+            return e;
+        decode_combine_kernel<__nv_bfloat16><<<dim3(L.Hq, a.B), 128, 0, stream>>>(L, a);
+        return cudaGetLastError();
+    }
+    dim3 g1(L.Hkv, a.B);
+    dim3 g2((L.Hq + 3) / 4, a.B);
+    if (dtype == kDtypeBf16) {
+        decode_write_new_kernel<__nv_bfloat16><<<g1, 128, 0, stream>>>(L, a);
+        decode_simt_kernel<__nv_bfloat16><<<g2, 128, 0, stream>>>(L, a);
+    } else {
+        decode_write_new_kernel<float><<<g1, 128, 0, stream>>>(L, a);
+        decode_simt_kernel<float><<<g2, 128, 0, stream>>>(L, a);
+    }
+    return cudaGetLastError();
+}
+
+} // namespace mimo

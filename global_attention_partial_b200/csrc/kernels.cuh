@@ -1,0 +1,81 @@
+// Internal launch interface of the MiMo-V2-Flash attention kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace mimo {
+
+enum { kDtypeBf16 = 0, kDtypeFp32 = 1 };
+
+// Per-layer values resolved on the host from mimo_attn_layer.
+struct LayerArgs {
+    int layer_type;    // 0 global, 1 sliding window
+    int Hq, Hkv, G;    // G = Hq / Hkv query heads per KV head
+    int Dqk, Dv;
+    int window;        // sliding layers only
+    float scale_log2;  // softmax scale * log2(e): scores are kept in base-2 units
+    float v_scale;     // sqrt(hidden / (Hq * Dv))
+    const float *sinks;  // [Hq] natural-log sink logits or nullptr
+    RopeArgs rope;
+};
+
+// Rotates K at each token's position and stores it, and copies K/V into the
+// caches. dst_k receives every token (row i of [B, dst_rows, Hkv, Dqk]);
+// ring_k / ring_v (sliding-window ring, slot i mod window) receive the last
+// `window` tokens; lin_v (global value cache [B, lin_rows, Hkv, Dv]) receives
+// every token.
+struct KprepArgs {
+    const void *k;
+    const void *v;
+    const int *positions;  // nullptr: position = sequence index
+    void *dst_k;
+    long long dst_rows;
+    void *ring_k;
+    void *ring_v;
+    void *lin_v;
+    long long lin_rows;
+    int B, S, Hkv, Dqk, Dv, window;
+    RopeArgs rope;
+};
+cudaError_t launch_kprep(const KprepArgs &a, int dtype, cudaStream_t stream);
+
+// Prefill attention on CUDA cores (any dims up to 256, fp32 or bf16).
+// krot: rotated keys [B, krot_rows, Hkv, Dqk].
+struct PrefillArgs {
+    const void *q;
+    const void *krot;
+    long long krot_rows;
+    const void *v;
+    const int *positions;
+    void *out;
+    int B, S;
+    unsigned *err;
+};
+cudaError_t launch_prefill_simt(const LayerArgs &L, const PrefillArgs &a, int dtype,
+                                cudaStream_t stream);
+
+// Prefill attention on the tcgen05 tensor cores (bf16, Dqk 192, Dv 128).
+bool prefill_tc_supported(const LayerArgs &L);
+cudaError_t launch_prefill_tc(const LayerArgs &L, const PrefillArgs &a, cudaStream_t stream);
+
+// Decode. Caches: GLOBAL linear [B, cap, Hkv, D]; SWA ring [B, window, Hkv, D].
+struct DecodeArgs {
+    const void *q;
+    const void *k_new;
+    const void *v_new;
+    const int *kv_lens;
+    void *k_cache;
+    void *v_cache;
+    int cap;
+    void *out;
+    float *partial;  // workspace: [B, Hq, max_splits, Dv + 2] fp32
+    int max_splits;
+    int chunk;       // keys per split
+    int B;
+    unsigned *err;
+};
+int decode_chunk_keys(const LayerArgs &L, int dtype);
+int decode_max_splits(const LayerArgs &L, int dtype, int cap);
+cudaError_t launch_decode(const LayerArgs &L, const DecodeArgs &a, int dtype, cudaStream_t stream);
+
+} // namespace mimo

@@ -1,0 +1,175 @@
+// Key preparation and the CUDA-core prefill path of the MiMo-V2-Flash layer.
+//
+// kprep: rotates every key at its token's position (partial RoPE, computed
+// in fp32 from a double-precision angle) once per layer, and writes it where
+// the attention kernels read it (the global cache itself, or a workspace),
+// plus the caches: the global value cache, or the sliding-window ring (slot
+// i mod window for the last `window` tokens). Rotating K once per layer,
+// rather than once per (query tile, key tile) pair, keeps the rotation off
+// the attention kernels' inner loop.
+//
+// prefill_simt: one warp per query row on CUDA cores, fp32 arithmetic; the
+// path for fp32 inputs and for head dims the tensor-core kernel does not
+// take.
+#include "kernels.cuh"
+
+#include <math.h>
+
+namespace mimo {
+namespace {
+
+template <typename T>
+__global__ void kprep_kernel(const __grid_constant__ KprepArgs a)
+{
+    const int warps = blockDim.x >> 5;
+    const long long row = (long long)blockIdx.x * warps + (threadIdx.x >> 5);
+    const long long total = (long long)a.B * a.S * a.Hkv;
+    if (row >= total)
+        return;
+    const int lane = threadIdx.x & 31;
+    const int kv = (int)(row % a.Hkv);
+    const long long bi = row / a.Hkv;
+    const int i = (int)(bi % a.S);
+    const int b = (int)(bi / a.S);
+    const double pos = a.positions ? (double)__ldg(a.positions + i) : (double)i;
+    const int half = a.rope.half;
+    const T *k = reinterpret_cast<const T *>(a.k) + row * a.Dqk;
+    T *dk = reinterpret_cast<T *>(a.dst_k) + (((long long)b * a.dst_rows + i) * a.Hkv + kv) * a.Dqk;
+    const bool to_ring = a.ring_k != nullptr && a.window > 0 && i >= a.S - a.window;
+    const long long ring_off = to_ring ? ((long long)b * a.window + i % a.window) * a.Hkv + kv : 0;
+    T *rk = to_ring ? reinterpret_cast<T *>(a.ring_k) + ring_off * a.Dqk : nullptr;
+    for (int e = lane; e < a.Dqk; e += 32) {
+        float y;
+        if (e < a.rope.rotary_dim) {
+            const int j = e < half ? e : e - half;
+            float c, s;
+            rope_cos_sin(pos, a.rope.inv_freq[j], c, s);
+            const float xa = to_f32<T>(k[j]);
+            const float xb = to_f32<T>(k[j + half]);
+            y = e < half ? xa * c - xb * s : xb * c + xa * s;
+        } else {
+            y = to_f32<T>(k[e]);
+        }
+        const T yt = from_f32<T>(y);
+        dk[e] = yt;
+        if (rk)
+            rk[e] = yt;
+    }
+    T *rv = to_ring ? reinterpret_cast<T *>(a.ring_v) + ring_off * a.Dv : nullptr;
+    T *lv = a.lin_v ? reinterpret_cast<T *>(a.lin_v) + (((long long)b * a.lin_rows + i) * a.Hkv + kv) * a.Dv
+                    : nullptr;
+    if (rv || lv) {
+        const T *v = reinterpret_cast<const T *>(a.v) + row * a.Dv;
+        for (int e = lane; e < a.Dv; e += 32) {
+            const T x = v[e];
+            if (rv)
+                rv[e] = x;
+            if (lv)
+                lv[e] = x;
+        }
+    }
+}
+
+template <typename T>
+__global__ void prefill_simt_kernel(const __grid_constant__ LayerArgs L, const __grid_constant__ PrefillArgs a)
+{
+    __shared__ float qs[4][256];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int i = blockIdx.x * 4 + warp;
+    const int h = blockIdx.y;
+    const int b = blockIdx.z;
+    if (i >= a.S)
+        return;
+    const double pos = a.positions ? (double)__ldg(a.positions + i) : (double)i;
+    const int half = L.rope.half;
+    const T *q = reinterpret_cast<const T *>(a.q) + (((size_t)b * a.S + i) * L.Hq + h) * L.Dqk;
+    for (int e = lane; e < L.Dqk; e += 32) {
+        float y;
+        if (e < L.rope.rotary_dim) {
+            const int j = e < half ? e : e - half;
+            float c, s;
+            rope_cos_sin(pos, L.rope.inv_freq[j], c, s);
+            const float xa = to_f32<T>(q[j]);
+            const float xb = to_f32<T>(q[j + half]);
+            y = e < half ? xa * c - xb * s : xb * c + xa * s;
+        } else {
+            y = to_f32<T>(q[e]);
+        }
+        qs[warp][e] = y;
+    }
+    __syncwarp();
+    const int kvh = h / L.G;
+    const int lo = L.layer_type == 1 ? max(0, i - L.window + 1) : 0;
+    float m = -INFINITY, l = 0.f;
+    float acc[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+        acc[t] = 0.f;
+    for (int j = lo; j <= i; ++j) {
+        const T *kr = reinterpret_cast<const T *>(a.krot) + (((size_t)b * a.krot_rows + j) * L.Hkv + kvh) * L.Dqk;
+        float part = 0.f;
+        for (int e = lane; e < L.Dqk; e += 32)
+            part += qs[warp][e] * to_f32<T>(kr[e]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            part += __shfl_xor_sync(0xffffffffu, part, off);
+        const float x = part * L.scale_log2;
+        const float mn = fmaxf(m, x);
+        const float c = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+        const float pj = exp2f(x - mn);
+        l = l * c + pj;
+        const T *vr = reinterpret_cast<const T *>(a.v) + (((size_t)b * a.S + j) * L.Hkv + kvh) * L.Dv;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const int e = lane + 32 * t;
+            if (e < L.Dv)
+                acc[t] = acc[t] * c + pj * to_f32<T>(vr[e]);
+        }
+        m = mn;
+    }
+    float scale;
+    if (L.sinks != nullptr) {
+        const float s2 = __ldg(L.sinks + h) * kLog2e;
+        const float mf = fmaxf(m, s2);
+        const float al = exp2f(m - mf);
+        scale = al * L.v_scale / (l * al + exp2f(s2 - mf));
+    } else {
+        scale = L.v_scale / l;
+    }
+    T *dst = reinterpret_cast<T *>(a.out) + (((size_t)b * a.S + i) * L.Hq + h) * L.Dv;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+        const int e = lane + 32 * t;
+        if (e < L.Dv)
+            dst[e] = from_f32<T>(acc[t] * scale);
+    }
+}
+
+} // namespace
+
+cudaError_t launch_kprep(const KprepArgs &a, int dtype, cudaStream_t stream)
+{
+    const long long rows = (long long)a.B * a.S * a.Hkv;
+    if (rows == 0)
+        return cudaSuccess;
+    const int threads = 256;
+    const long long blocks = (rows + (threads / 32) - 1) / (threads / 32);
+    if (dtype == kDtypeBf16)
+        kprep_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, stream>>>(a);
+    else
+        kprep_kernel<float><<<(unsigned)blocks, threads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_simt(const LayerArgs &L, const PrefillArgs &a, int dtype, cudaStream_t stream)
+{
+    dim3 grid((a.S + 3) / 4, L.Hq, a.B);
+    if (dtype == kDtypeBf16)
+        prefill_simt_kernel<__nv_bfloat16><<<grid, 128, 0, stream>>>(L, a);
+    else
+        prefill_simt_kernel<float><<<grid, 128, 0, stream>>>(L, a);
+    return cudaGetLastError();
+}
+
+} // namespace mimo

@@ -38,6 +38,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define MIMO_ATTN_API __attribute__((visibility("default")))
+#else
+#define MIMO_ATTN_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -77,12 +83,12 @@ typedef struct {
  * lablup/mlxcel issue 842 ("Architecture, verified against upstream"); the
  * factor is taken as a double because upstream types it as an int but uses
  * it as a multiplier. Returns -1 for a negative or non-finite product. */
-int mimo_attn_rotary_dim(double partial_rotary_factor, int qk_dim);
+MIMO_ATTN_API int mimo_attn_rotary_dim(double partial_rotary_factor, int qk_dim);
 
 /* Bytes of workspace mimo_attn_prefill needs for this layer and shape
  * (the rotated keys when they are not written into a global cache). The
  * value does not depend on whether caches are passed; 0 means none. */
-size_t mimo_attn_prefill_workspace_size(const mimo_attn_layer *layer, int dtype,
+MIMO_ATTN_API size_t mimo_attn_prefill_workspace_size(const mimo_attn_layer *layer, int dtype,
                                         int batch, int seq);
 
 /* Prefill: one layer's attention over a whole prompt.
@@ -109,7 +115,7 @@ size_t mimo_attn_prefill_workspace_size(const mimo_attn_layer *layer, int dtype,
  * misaligned bf16 pointers; MIMO_ATTN_ERR_UNSUPPORTED for dims > 256;
  * MIMO_ATTN_ERR_WORKSPACE for a short workspace. batch == 0 or seq == 0 is
  * a no-op returning MIMO_ATTN_OK. */
-mimo_attn_status mimo_attn_prefill(const mimo_attn_layer *layer, int dtype, int batch, int seq,
+MIMO_ATTN_API mimo_attn_status mimo_attn_prefill(const mimo_attn_layer *layer, int dtype, int batch, int seq,
                                    const void *q, const void *k, const void *v,
                                    const int32_t *positions, void *out,
                                    void *k_cache, void *v_cache, int cache_capacity,
@@ -117,7 +123,7 @@ mimo_attn_status mimo_attn_prefill(const mimo_attn_layer *layer, int dtype, int 
 
 /* Bytes of workspace mimo_attn_decode needs (split-KV partial results) for
  * this layer, batch and cache capacity. */
-size_t mimo_attn_decode_workspace_size(const mimo_attn_layer *layer, int dtype, int batch,
+MIMO_ATTN_API size_t mimo_attn_decode_workspace_size(const mimo_attn_layer *layer, int dtype, int batch,
                                        int cache_capacity);
 
 /* Decode: one new token per sequence, attending to its cache.
@@ -137,7 +143,7 @@ size_t mimo_attn_decode_workspace_size(const mimo_attn_layer *layer, int dtype, 
  *   workspace: at least mimo_attn_decode_workspace_size() bytes, 256-byte aligned.
  * A kv_lens entry out of range sets MIMO_ATTN_DEVERR_KV_LEN in the device
  * error word and leaves that sequence's output and cache untouched. */
-mimo_attn_status mimo_attn_decode(const mimo_attn_layer *layer, int dtype, int batch,
+MIMO_ATTN_API mimo_attn_status mimo_attn_decode(const mimo_attn_layer *layer, int dtype, int batch,
                                   const void *q, const void *k_new, const void *v_new,
                                   const int32_t *kv_lens, void *k_cache, void *v_cache,
                                   int cache_capacity, void *out, void *workspace,
@@ -150,18 +156,18 @@ mimo_attn_status mimo_attn_decode(const mimo_attn_layer *layer, int dtype, int b
 /* Reads and clears the device error word of the current device
  * (synchronises the device). Returns MIMO_ATTN_OK and stores the bits in
  * *bits, or MIMO_ATTN_ERR_CUDA. */
-mimo_attn_status mimo_attn_get_device_error(uint32_t *bits);
+MIMO_ATTN_API mimo_attn_status mimo_attn_get_device_error(uint32_t *bits);
 
 /* Static description of a status code. */
-const char *mimo_attn_status_string(mimo_attn_status status);
+MIMO_ATTN_API const char *mimo_attn_status_string(mimo_attn_status status);
 
 /* Test hook: while non-zero, every launching entry point returns
  * MIMO_ATTN_ERR_CUDA after its argument checks, without launching. Lets the
  * host-side error path be tested without provoking a GPU fault. */
-void mimo_attn_debug_fail_launches(int enable);
+MIMO_ATTN_API void mimo_attn_debug_fail_launches(int enable);
 
 /* Version string of the library. */
-const char *mimo_attn_version(void);
+MIMO_ATTN_API const char *mimo_attn_version(void);
 
 #ifdef __cplusplus
 }
