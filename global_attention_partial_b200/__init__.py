@@ -34,6 +34,7 @@ EXPORTED = (
     "mimo_attn_prefill",
     "mimo_attn_decode_workspace_size",
     "mimo_attn_decode",
+    "mimo_attn_decode_static",
     "mimo_attn_get_device_error",
     "mimo_attn_status_string",
     "mimo_attn_debug_fail_launches",
@@ -87,6 +88,8 @@ def load() -> ctypes.CDLL:
     lib.mimo_attn_decode_workspace_size.restype = sz
     lib.mimo_attn_decode.argtypes = [lp, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
     lib.mimo_attn_decode.restype = i32
+    lib.mimo_attn_decode_static.argtypes = [lp, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp]
+    lib.mimo_attn_decode_static.restype = i32
     lib.mimo_attn_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     lib.mimo_attn_get_device_error.restype = i32
     lib.mimo_attn_status_string.argtypes = [i32]
@@ -185,6 +188,16 @@ def mimo_attn_decode(layer: mimo_attn_layer, dtype: int, batch: int, q, k_new, v
         ctypes.byref(layer), dtype, batch, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(kv_lens),
         _ptr(k_cache), _ptr(v_cache), int(cache_capacity), _ptr(out), _ptr(workspace),
         int(workspace_bytes), _stream(stream)))
+
+
+def mimo_attn_decode_static(layer: mimo_attn_layer, dtype: int, batch: int, q, k_new, v_new, kv_lens, k_cache,
+                            v_cache, cache_capacity: int, out, stream=None) -> int:
+    """Decode with no allocation at all: the split partials live in the
+    library's built-in 16 MiB scratch (see include/mimo_attn.h). For callers
+    that cannot allocate device memory; concurrent calls race on the scratch."""
+    return int(load().mimo_attn_decode_static(
+        ctypes.byref(layer), dtype, batch, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(kv_lens),
+        _ptr(k_cache), _ptr(v_cache), int(cache_capacity), _ptr(out), _stream(stream)))
 
 
 def mimo_attn_get_device_error() -> int:

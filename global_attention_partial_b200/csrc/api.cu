@@ -10,6 +10,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 namespace {
 
 // Device error word: sticky bits set by kernels (kv_lens out of range, wait
@@ -290,3 +292,60 @@ void mimo_attn_debug_fail_launches(int enable) { g_fail_launches = enable != 0; 
 const char *mimo_attn_version(void) { return "mimo_attn 0.1.0 (sm_100a)"; }
 
 } // extern "C"
+
+// ------------------------------------------------------ decode without allocation
+// mimo_attn_decode_static keeps the split-KV partial results in this
+// file-scope device array instead of a caller workspace, for callers that
+// cannot allocate device memory. The array is part of the library's device
+// image: every GPU that loads the library holds these 16 MiB until the
+// process exits. Every call shares it and it keeps the previous call's
+// contents; nothing in it needs to start at zero, because each call writes
+// every partial it later reads. Calls whose kernels overlap on the GPU (other
+// streams, other host threads) race on it.
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) float g_decode_scratch[kStaticScratchBytes / sizeof(float)];
+
+std::mutex g_scratch_mutex;
+float *g_scratch_ptr[kMaxDevices];
+
+// Device address of g_decode_scratch on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+float *static_scratch_ptr()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return nullptr;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (g_scratch_ptr[dev] == nullptr) {
+        float *ptr = nullptr;
+        if (cudaGetSymbolAddress((void **)&ptr, g_decode_scratch) != cudaSuccess)
+            return nullptr;
+        g_scratch_ptr[dev] = ptr;
+    }
+    return g_scratch_ptr[dev];
+}
+
+} // namespace
+
+extern "C" mimo_attn_status mimo_attn_decode_static(const mimo_attn_layer *layer, int dtype, int batch,
+                                                    const void *q, const void *k_new, const void *v_new,
+                                                    const int32_t *kv_lens, void *k_cache, void *v_cache,
+                                                    int cache_capacity, void *out, void *stream)
+{
+    const size_t need = mimo_attn_decode_workspace_size(layer, dtype, batch, cache_capacity);
+    if (need > kStaticScratchBytes)
+        return MIMO_ATTN_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    if (need > 0) {  // a valid layer that splits the keys: partials go to the array
+        if (g_fail_launches)
+            return MIMO_ATTN_ERR_CUDA;
+        scratch = static_scratch_ptr();
+        if (scratch == nullptr)
+            return MIMO_ATTN_ERR_CUDA;
+    }
+    return mimo_attn_decode(layer, dtype, batch, q, k_new, v_new, kv_lens, k_cache, v_cache,
+                            cache_capacity, out, scratch, need, stream);
+}

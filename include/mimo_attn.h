@@ -149,6 +149,32 @@ MIMO_ATTN_API mimo_attn_status mimo_attn_decode(const mimo_attn_layer *layer, in
                                   int cache_capacity, void *out, void *workspace,
                                   size_t workspace_bytes, void *stream);
 
+/* Decode without any allocation: the same computation, arguments and
+ * errors as mimo_attn_decode, but the split-KV partial results live in a
+ * 16 MiB scratch array built into the library instead of a caller
+ * workspace. For callers that cannot allocate device memory at all (a host
+ * program whose memory pool owns the whole device, a plugin with no
+ * allocator of its own, a loop that must not pay cudaMalloc's
+ * synchronisation). The pages have no counterpart: this is an interface
+ * convenience of this library, not a step of the layer.
+ *   - Limit: mimo_attn_decode_workspace_size(layer, dtype, batch,
+ *     cache_capacity) must be at most 16 MiB (16777216 bytes), else the call
+ *     returns MIMO_ATTN_ERR_WORKSPACE and launches nothing. (Example: 64
+ *     query heads, cache 32768, up to 15 sequences per call.)
+ *   - The array is device memory held by every GPU that loads the library,
+ *     until the process exits.
+ *   - The first call on a device looks up the array's device address there
+ *     (once per device, cached); make that first call before any stream
+ *     capture.
+ *   - All calls share the array and it keeps the last call's contents;
+ *     nothing in it has to start at zero. Calls whose kernels overlap on the
+ *     GPU (concurrent streams, several host threads) race on it: serialise
+ *     them. */
+MIMO_ATTN_API mimo_attn_status mimo_attn_decode_static(const mimo_attn_layer *layer, int dtype, int batch,
+                                         const void *q, const void *k_new, const void *v_new,
+                                         const int32_t *kv_lens, void *k_cache, void *v_cache,
+                                         int cache_capacity, void *out, void *stream);
+
 /* Device error word bits (sticky until read). */
 #define MIMO_ATTN_DEVERR_KV_LEN 0x1u   /* a kv_lens entry was out of range */
 #define MIMO_ATTN_DEVERR_TIMEOUT 0x2u  /* a kernel pipeline wait hit its iteration limit */
