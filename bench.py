@@ -405,12 +405,19 @@ def barrier(dist, local):
         dist.barrier(device_ids=[local])
 
 
-def max_over_ranks(dist, x: float) -> float:
+def max_over_ranks(dist, x: float, device="cuda") -> float:
+    """Max of x over all ranks (the step time of the slowest GPU)."""
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_value(world: int, units_per_rank: float, ms_max: float) -> float:
+    """Whole-job throughput (weak scaling): every rank processes the same
+    units; the job takes as long as the slowest rank. TFLOP/s for FLOP units."""
+    return world * units_per_rank / (ms_max * 1e-3) / 1e12
 
 
 def run_reference(args):
@@ -508,7 +515,7 @@ def main():
     pflops = w.prefill_flops() if w.do_prefill else 0.0
     dflops = w.decode_flops() if w.do_decode else 0.0
     step_flops = pflops + dflops
-    value = world * step_flops / (ms * 1e-3) / 1e12
+    value = job_value(world, step_flops, ms)
 
     parts = {}
     roofline = None
@@ -574,7 +581,7 @@ def main():
         torch.cuda.synchronize()
         barrier(dist, local)
         ms_e2e = max_over_ranks(dist, e0.elapsed_time(e1) / e2e_steps)
-        e2e = {"value": world * step_flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_value(world, step_flops, ms_e2e), "unit": "TFLOP/s",
                "h2d_bytes_per_step": host.h2d, "d2h_bytes_per_step": host.d2h, "ms_per_step": ms_e2e,
                "steps": e2e_steps}
         del host
