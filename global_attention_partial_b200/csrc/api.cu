@@ -37,6 +37,23 @@ unsigned *device_error_ptr()
     return g_err_ptr[dev];
 }
 
+int g_num_sms[kMaxDevices];
+
+// Streaming multiprocessors of the current device (cached per device).
+int num_sms()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return 148;
+    if (g_num_sms[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+            n = 148;
+        g_num_sms[dev] = n;
+    }
+    return g_num_sms[dev];
+}
+
 size_t elem_size(int dtype) { return dtype == MIMO_ATTN_BF16 ? 2 : 4; }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -107,7 +124,9 @@ size_t mimo_attn_prefill_workspace_size(const mimo_attn_layer *layer, int dtype,
     mimo::LayerArgs L;
     if (resolve_layer(layer, dtype, &L) != MIMO_ATTN_OK || batch < 0 || seq < 0)
         return 0;
-    return round_up((size_t)batch * seq * L.Hkv * L.Dqk * elem_size(dtype), 256);
+    // the RoPE cos/sin table [S, r/2], then the rotated keys [B, S, Hkv, Dqk]
+    return round_up((size_t)seq * L.rope.half * sizeof(float2), 256) +
+           round_up((size_t)batch * seq * L.Hkv * L.Dqk * elem_size(dtype), 256);
 }
 
 mimo_attn_status mimo_attn_prefill(const mimo_attn_layer *layer, int dtype, int batch, int seq,
@@ -139,9 +158,12 @@ mimo_attn_status mimo_attn_prefill(const mimo_attn_layer *layer, int dtype, int 
         !(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out) && aligned16(k_cache) &&
           aligned16(v_cache) && aligned16(workspace)))
         return MIMO_ATTN_ERR_INVALID_ARG;
-    // Rotated keys go straight into a global cache; otherwise to the workspace.
+    // Workspace: the RoPE cos/sin table [S, r/2] first, then the rotated keys
+    // (which go straight into a global cache when the caller passes one).
     const bool keys_in_cache = has_cache && L.layer_type == MIMO_ATTN_GLOBAL;
-    const size_t need = keys_in_cache ? 0 : mimo_attn_prefill_workspace_size(layer, dtype, batch, seq);
+    const bool use_swa_kernel = dtype == MIMO_ATTN_BF16 && mimo::prefill_swa_supported(L);
+    const size_t table_bytes = round_up((size_t)seq * L.rope.half * sizeof(float2), 256);
+    const size_t need = keys_in_cache ? table_bytes : mimo_attn_prefill_workspace_size(layer, dtype, batch, seq);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need))
         return MIMO_ATTN_ERR_WORKSPACE;
     if (g_fail_launches)
@@ -156,7 +178,7 @@ mimo_attn_status mimo_attn_prefill(const mimo_attn_layer *layer, int dtype, int 
     kp.k = k;
     kp.v = v;
     kp.positions = positions;
-    kp.dst_k = keys_in_cache ? k_cache : workspace;
+    kp.dst_k = keys_in_cache ? k_cache : static_cast<void *>(static_cast<char *>(workspace) + table_bytes);
     kp.dst_rows = keys_in_cache ? cache_capacity : seq;
     if (has_cache && L.layer_type == MIMO_ATTN_SWA) {
         kp.ring_k = k_cache;
@@ -172,6 +194,7 @@ mimo_attn_status mimo_attn_prefill(const mimo_attn_layer *layer, int dtype, int 
     kp.Dqk = L.Dqk;
     kp.Dv = L.Dv;
     kp.window = L.layer_type == MIMO_ATTN_SWA ? L.window : 0;
+    kp.rope_table = L.rope.half > 0 ? reinterpret_cast<float2 *>(workspace) : nullptr;
     kp.rope = L.rope;
     if (mimo::launch_kprep(kp, dtype, s) != cudaSuccess)
         return MIMO_ATTN_ERR_CUDA;
@@ -182,12 +205,15 @@ mimo_attn_status mimo_attn_prefill(const mimo_attn_layer *layer, int dtype, int 
     pa.krot_rows = kp.dst_rows;
     pa.v = v;
     pa.positions = positions;
+    pa.rope_table = kp.rope_table;
     pa.out = out;
     pa.B = batch;
     pa.S = seq;
     pa.err = err;
     cudaError_t e;
-    if (dtype == MIMO_ATTN_BF16 && mimo::prefill_tc_supported(L))
+    if (use_swa_kernel)
+        e = mimo::launch_prefill_swa(L, pa, pa.rope_table, num_sms(), s);
+    else if (dtype == MIMO_ATTN_BF16 && mimo::prefill_tc_supported(L))
         e = mimo::launch_prefill_tc(L, pa, s);
     else
         e = mimo::launch_prefill_simt(L, pa, dtype, s);

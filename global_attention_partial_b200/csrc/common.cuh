@@ -3,8 +3,8 @@
 // PTX wrappers for mbarriers, TMA tensor loads, tcgen05 (TMEM alloc, MMA,
 // commit, ld/st), cp.async, ldmatrix and mma.sync, plus the RoPE angle
 // routine shared by every kernel of the library. Every spin-wait is bounded:
-// after kWaitLimitNs of waiting it sets the device error word and reports a
-// timeout so the caller can tear down instead of hanging.
+// after kWaitLimitCycles of waiting it sets the device error word and reports
+// a timeout so the caller can tear down instead of hanging.
 #pragma once
 
 #include <cuda.h>
@@ -17,7 +17,8 @@ namespace mimo {
 constexpr int kMaxHalfRotary = 128;          // rotary_dim <= 256
 constexpr unsigned kErrKvLen = 0x1u;         // = MIMO_ATTN_DEVERR_KV_LEN
 constexpr unsigned kErrTimeout = 0x2u;       // = MIMO_ATTN_DEVERR_TIMEOUT
-constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s
+// Wait limit in SM clock cycles: ~4 s at 2 GHz, ~8 s at the lowest clocks.
+constexpr long long kWaitLimitCycles = 8000000000ll;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Partial-RoPE parameters of one layer: pair j of the first rotary_dim dims
@@ -53,6 +54,21 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
+// 2^x on the special-function unit (ex2.approx, flush-to-zero): relative
+// error ~2^-22, ample for softmax weights rounded to bf16; 2^-inf = 0.
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Branch-free test lo <= c <= hi (one unsigned compare; empty when hi < lo).
+__device__ __forceinline__ bool in_range(int c, int lo, int hi)
+{
+    return (unsigned)(c - lo) <= (unsigned)(hi - lo) && hi >= lo;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -64,12 +80,8 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p)
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t globaltimer_ns()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
+// SM cycle counter: cheap to read, used to bound every spin-wait.
+__device__ __forceinline__ long long cycles_now() { return clock64(); }
 
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
@@ -101,22 +113,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// Non-blocking probe of a phase (never suspends the thread): for polling
+// loops that must not stall on one barrier while another is ready.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}\n"
+                 : "=r"(ok)
+                 : "r"(smem_u32(bar)), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
 // Waits for the phase of `bar` with the given parity to complete. Returns
 // false (without waiting further) once *abort is set by another thread of the
-// CTA, or after kWaitLimitNs, in which case it sets *abort and the timeout
+// CTA, or after kWaitLimitCycles, in which case it sets *abort and the timeout
 // bit of the device error word.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           unsigned *err)
 {
     if (mbar_try_wait(bar, parity))
         return true;
-    uint64_t t0 = globaltimer_ns();
+    const long long t0 = cycles_now();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity))
             return true;
         if (*abort)
             return false;
-        if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+        if ((it & 255u) == 0 && cycles_now() - t0 > kWaitLimitCycles) {
             *abort = 1;
             atomicOr(err, kErrTimeout);
             return false;
@@ -128,9 +154,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 // in-flight asynchronous copies to land so the CTA never exits under them.
 __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity)
 {
-    uint64_t t0 = globaltimer_ns();
+    const long long t0 = cycles_now();
     while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs)
+        if (cycles_now() - t0 > kWaitLimitCycles)
             return;
     }
 }
@@ -283,6 +309,20 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
                  : "r"(taddr));
 }
 
+// Ties registers filled by earlier tcgen05.ld to a wait already executed
+// (tmem_wait_ld_only), so the compiler cannot read them before it.
+template <int N> __device__ __forceinline__ void tmem_tie(uint32_t (&r)[N])
+{
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+        asm volatile("" : "+r"(r[i]));
+}
+
+__device__ __forceinline__ void tmem_wait_ld_only()
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 template <int N> __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[N])
 {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
@@ -317,6 +357,16 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
 __device__ __forceinline__ void tmem_wait_st()
 {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Warpgroup register rebalancing: every warp of the warpgroup executes it.
+template <int N> __device__ __forceinline__ void setmaxnreg_inc()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N> __device__ __forceinline__ void setmaxnreg_dec()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ----------------------------------------------------- cp.async / mma.sync

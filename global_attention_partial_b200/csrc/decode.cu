@@ -84,6 +84,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int G = L.G;
     const int half = L.rope.half;
 
+    // cos/sin of the new token's position for every rotary pair, once per CTA
+    __shared__ float2 s_cs[kMaxHalfRotary];
+    for (int j = tid; j < half; j += kThreads) {
+        float c, s;
+        rope_cos_sin(pos, L.rope.inv_freq[j], c, s);
+        s_cs[j] = make_float2(c, s);
+    }
+    __syncthreads();
+
     const size_t kv_row = (size_t)L.Hkv;  // rows of the cache are [slot][Hkv][D]
     const __nv_bfloat16 *kc = reinterpret_cast<const __nv_bfloat16 *>(a.k_cache) +
                               ((size_t)b * a.cap * kv_row + kvh) * kDqk;
@@ -102,11 +111,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const __nv_bfloat16 *qr = qg + (size_t)r * kDqk;
                 if (e < L.rope.rotary_dim) {
                     const int j = e < half ? e : e - half;
-                    float c, s;
-                    rope_cos_sin(pos, L.rope.inv_freq[j], c, s);
+                    const float2 cs = s_cs[j];
                     const float xa = __bfloat162float(qr[j]);
                     const float xb = __bfloat162float(qr[j + half]);
-                    y = e < half ? xa * c - xb * s : xb * c + xa * s;
+                    y = e < half ? xa * cs.x - xb * cs.y : xb * cs.x + xa * cs.y;
                 } else {
                     y = __bfloat162float(qr[e]);
                 }
@@ -128,11 +136,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             float y;
             if (e < L.rope.rotary_dim) {
                 const int j = e < half ? e : e - half;
-                float c, s;
-                rope_cos_sin(pos, L.rope.inv_freq[j], c, s);
+                const float2 cs = s_cs[j];
                 const float xa = __bfloat162float(kn[j]);
                 const float xb = __bfloat162float(kn[j + half]);
-                y = e < half ? xa * c - xb * s : xb * c + xa * s;
+                y = e < half ? xa * cs.x - xb * cs.y : xb * cs.x + xa * cs.y;
             } else {
                 y = __bfloat162float(kn[e]);
             }
@@ -438,6 +445,13 @@ __global__ void decode_write_new_kernel(const __grid_constant__ LayerArgs L, con
     const int slot = L.layer_type == 1 ? (Lb - 1) % L.window : Lb - 1;
     const double pos = (double)(Lb - 1);
     const int half = L.rope.half;
+    __shared__ float2 s_cs[kMaxHalfRotary];
+    for (int j = threadIdx.x; j < half; j += blockDim.x) {
+        float c, s;
+        rope_cos_sin(pos, L.rope.inv_freq[j], c, s);
+        s_cs[j] = make_float2(c, s);
+    }
+    __syncthreads();
     const T *kn = reinterpret_cast<const T *>(a.k_new) + ((size_t)b * L.Hkv + kvh) * L.Dqk;
     const T *vn = reinterpret_cast<const T *>(a.v_new) + ((size_t)b * L.Hkv + kvh) * L.Dv;
     T *kd = reinterpret_cast<T *>(a.k_cache) + (((size_t)b * a.cap + slot) * L.Hkv + kvh) * L.Dqk;
@@ -446,11 +460,10 @@ __global__ void decode_write_new_kernel(const __grid_constant__ LayerArgs L, con
         float y;
         if (e < L.rope.rotary_dim) {
             const int j = e < half ? e : e - half;
-            float c, s;
-            rope_cos_sin(pos, L.rope.inv_freq[j], c, s);
+            const float2 cs = s_cs[j];
             const float xa = to_f32<T>(kn[j]);
             const float xb = to_f32<T>(kn[j + half]);
-            y = e < half ? xa * c - xb * s : xb * c + xa * s;
+            y = e < half ? xa * cs.x - xb * cs.y : xb * cs.x + xa * cs.y;
         } else {
             y = to_f32<T>(kn[e]);
         }
@@ -465,28 +478,34 @@ template <typename T>
 __global__ void decode_simt_kernel(const __grid_constant__ LayerArgs L, const __grid_constant__ DecodeArgs a)
 {
     __shared__ float qs[4][256];
+    __shared__ float2 s_cs[kMaxHalfRotary];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int h = blockIdx.x * 4 + warp;
     const int b = blockIdx.y;
-    if (h >= L.Hq)
-        return;
     const int Lb = __ldg(a.kv_lens + b);
     if (!kv_len_ok(L.layer_type, Lb, a.cap))
         return;
-    const int n_vis = visible_count(L.layer_type, Lb, L.window);
     const double pos = (double)(Lb - 1);
     const int half = L.rope.half;
+    for (int j = threadIdx.x; j < half; j += blockDim.x) {
+        float c, s;
+        rope_cos_sin(pos, L.rope.inv_freq[j], c, s);
+        s_cs[j] = make_float2(c, s);
+    }
+    __syncthreads();
+    if (h >= L.Hq)
+        return;
+    const int n_vis = visible_count(L.layer_type, Lb, L.window);
     const T *q = reinterpret_cast<const T *>(a.q) + ((size_t)b * L.Hq + h) * L.Dqk;
     for (int e = lane; e < L.Dqk; e += 32) {
         float y;
         if (e < L.rope.rotary_dim) {
             const int j = e < half ? e : e - half;
-            float c, s;
-            rope_cos_sin(pos, L.rope.inv_freq[j], c, s);
+            const float2 cs = s_cs[j];
             const float xa = to_f32<T>(q[j]);
             const float xb = to_f32<T>(q[j + half]);
-            y = e < half ? xa * c - xb * s : xb * c + xa * s;
+            y = e < half ? xa * cs.x - xb * cs.y : xb * cs.x + xa * cs.y;
         } else {
             y = to_f32<T>(q[e]);
         }

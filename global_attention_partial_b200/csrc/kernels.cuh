@@ -35,6 +35,7 @@ struct KprepArgs {
     void *lin_v;
     long long lin_rows;
     int B, S, Hkv, Dqk, Dv, window;
+    float2 *rope_table;  // [S][rotary_dim/2] (cos, sin) of each token's position, built by launch_kprep
     RopeArgs rope;
 };
 cudaError_t launch_kprep(const KprepArgs &a, int dtype, cudaStream_t stream);
@@ -47,6 +48,7 @@ struct PrefillArgs {
     long long krot_rows;
     const void *v;
     const int *positions;
+    const float2 *rope_table;  // [S][rotary_dim/2] (cos, sin), built by launch_kprep
     void *out;
     int B, S;
     unsigned *err;
@@ -57,6 +59,17 @@ cudaError_t launch_prefill_simt(const LayerArgs &L, const PrefillArgs &a, int dt
 // Prefill attention on the tcgen05 tensor cores (bf16, Dqk 192, Dv 128).
 bool prefill_tc_supported(const LayerArgs &L);
 cudaError_t launch_prefill_tc(const LayerArgs &L, const PrefillArgs &a, cudaStream_t stream);
+
+// Sliding-window prefill whose tiles need a single key span (persistent,
+// one CTA per SM); rope_table is the kprep table.
+bool prefill_swa_supported(const LayerArgs &L);
+cudaError_t launch_prefill_swa(const LayerArgs &L, const PrefillArgs &a, const float2 *rope_table,
+                               int num_sms, cudaStream_t stream);
+
+// 4-D bf16 TMA map with 128-byte swizzle over [d3][d2_alloc][d1][d0] (d0
+// innermost), of which the first d2 rows along dimension 2 are in bounds.
+bool make_bf16_map_4d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                      uint64_t d2_alloc, uint64_t d3, uint32_t b0, uint32_t b1, uint32_t b2);
 
 // Decode. Caches: GLOBAL linear [B, cap, Hkv, D]; SWA ring [B, window, Hkv, D].
 struct DecodeArgs {

@@ -1,7 +1,8 @@
 // Key preparation and the CUDA-core prefill path of the MiMo-V2-Flash layer.
 //
-// kprep: rotates every key at its token's position (partial RoPE, computed
-// in fp32 from a double-precision angle) once per layer, and writes it where
+// kprep: builds the RoPE cos/sin table of every (position, pair) once, then
+// rotates every key at its token's position (fp32 arithmetic on the table's
+// values, angles formed in double precision) once per layer, and writes it where
 // the attention kernels read it (the global cache itself, or a workspace),
 // plus the caches: the global value cache, or the sliding-window ring (slot
 // i mod window for the last `window` tokens). Rotating K once per layer,
@@ -18,6 +19,29 @@
 namespace mimo {
 namespace {
 
+// cos / sin of every (position, pair): table[i][j] for pair j of token i.
+// The inverse frequencies are staged in shared memory, so lanes that need
+// different pairs never serialise on the kernel-parameter bank.
+__global__ void rope_table_kernel(const __grid_constant__ KprepArgs a)
+{
+    __shared__ double inv_freq[kMaxHalfRotary];
+    const int half = a.rope.half;
+    for (int j = threadIdx.x; j < half; j += blockDim.x)
+        inv_freq[j] = a.rope.inv_freq[j];
+    __syncthreads();
+    const long long total = (long long)a.S * half;
+    for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < total;
+         u += (long long)gridDim.x * blockDim.x) {
+        const int i = (int)(u / half);
+        const int j = (int)(u - (long long)i * half);
+        const double pos = a.positions ? (double)__ldg(a.positions + i) : (double)i;
+        float c, s;
+        rope_cos_sin(pos, inv_freq[j], c, s);
+        a.rope_table[u] = make_float2(c, s);
+    }
+}
+
+// One warp per key row (b, i, kv); any dims / dtype. Reads cos/sin from the table.
 template <typename T>
 __global__ void kprep_kernel(const __grid_constant__ KprepArgs a)
 {
@@ -31,8 +55,8 @@ __global__ void kprep_kernel(const __grid_constant__ KprepArgs a)
     const long long bi = row / a.Hkv;
     const int i = (int)(bi % a.S);
     const int b = (int)(bi / a.S);
-    const double pos = a.positions ? (double)__ldg(a.positions + i) : (double)i;
     const int half = a.rope.half;
+    const float2 *cs = a.rope_table + (long long)i * half;
     const T *k = reinterpret_cast<const T *>(a.k) + row * a.Dqk;
     T *dk = reinterpret_cast<T *>(a.dst_k) + (((long long)b * a.dst_rows + i) * a.Hkv + kv) * a.Dqk;
     const bool to_ring = a.ring_k != nullptr && a.window > 0 && i >= a.S - a.window;
@@ -42,11 +66,10 @@ __global__ void kprep_kernel(const __grid_constant__ KprepArgs a)
         float y;
         if (e < a.rope.rotary_dim) {
             const int j = e < half ? e : e - half;
-            float c, s;
-            rope_cos_sin(pos, a.rope.inv_freq[j], c, s);
+            const float2 c = __ldg(cs + j);
             const float xa = to_f32<T>(k[j]);
             const float xb = to_f32<T>(k[j + half]);
-            y = e < half ? xa * c - xb * s : xb * c + xa * s;
+            y = e < half ? xa * c.x - xb * c.y : xb * c.x + xa * c.y;
         } else {
             y = to_f32<T>(k[e]);
         }
@@ -70,6 +93,71 @@ __global__ void kprep_kernel(const __grid_constant__ KprepArgs a)
     }
 }
 
+// bf16 rows in 16-byte units (8 elements): a lane takes either a pair of
+// rotary chunks (c, c + half/8), a pass-through K chunk, or a V chunk.
+// Needs rotary_dim % 16 == 0, Dqk % 8 == 0, Dv % 8 == 0.
+__global__ void kprep_bf16_vec_kernel(const __grid_constant__ KprepArgs a)
+{
+    const int warps = blockDim.x >> 5;
+    const long long row = (long long)blockIdx.x * warps + (threadIdx.x >> 5);
+    const long long total = (long long)a.B * a.S * a.Hkv;
+    if (row >= total)
+        return;
+    const int lane = threadIdx.x & 31;
+    const int kv = (int)(row % a.Hkv);
+    const long long bi = row / a.Hkv;
+    const int i = (int)(bi % a.S);
+    const int b = (int)(bi / a.S);
+    const int npair = a.rope.half / 8;
+    const int ncopy = (a.Dqk - a.rope.rotary_dim) / 8;
+    const bool with_v = a.ring_v != nullptr || a.lin_v != nullptr;
+    const int nv = with_v ? a.Dv / 8 : 0;
+    const bool to_ring = a.ring_k != nullptr && a.window > 0 && i >= a.S - a.window;
+    const long long ring_off = to_ring ? ((long long)b * a.window + i % a.window) * a.Hkv + kv : 0;
+    const uint4 *k = reinterpret_cast<const uint4 *>(a.k) + row * (a.Dqk / 8);
+    uint4 *dk = reinterpret_cast<uint4 *>(a.dst_k) + (((long long)b * a.dst_rows + i) * a.Hkv + kv) * (a.Dqk / 8);
+    uint4 *rk = to_ring ? reinterpret_cast<uint4 *>(a.ring_k) + ring_off * (a.Dqk / 8) : nullptr;
+    for (int u = lane; u < npair + ncopy + nv; u += 32) {
+        if (u < npair) {
+            const uint4 xa = __ldg(k + u);
+            const uint4 xb = __ldg(k + u + npair);
+            const float4 *cs = reinterpret_cast<const float4 *>(a.rope_table + (long long)i * a.rope.half + u * 8);
+            const uint32_t *pa = reinterpret_cast<const uint32_t *>(&xa);
+            const uint32_t *pb = reinterpret_cast<const uint32_t *>(&xb);
+            uint4 ya, yb;
+            uint32_t *qa = reinterpret_cast<uint32_t *>(&ya);
+            uint32_t *qb = reinterpret_cast<uint32_t *>(&yb);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float4 c = __ldg(cs + w);  // (cos, sin) of pairs 8u+2w and 8u+2w+1
+                const float2 va = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pa[w]));
+                const float2 vb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pb[w]));
+                qa[w] = pack_bf16x2(va.x * c.x - vb.x * c.y, va.y * c.z - vb.y * c.w);
+                qb[w] = pack_bf16x2(vb.x * c.x + va.x * c.y, vb.y * c.z + va.y * c.w);
+            }
+            dk[u] = ya;
+            dk[u + npair] = yb;
+            if (rk) {
+                rk[u] = ya;
+                rk[u + npair] = yb;
+            }
+        } else if (u < npair + ncopy) {
+            const int c = 2 * npair + (u - npair);
+            const uint4 x = __ldg(k + c);
+            dk[c] = x;
+            if (rk)
+                rk[c] = x;
+        } else {
+            const int c = u - npair - ncopy;
+            const uint4 x = __ldg(reinterpret_cast<const uint4 *>(a.v) + row * (a.Dv / 8) + c);
+            if (to_ring)
+                reinterpret_cast<uint4 *>(a.ring_v)[ring_off * (a.Dv / 8) + c] = x;
+            if (a.lin_v)
+                reinterpret_cast<uint4 *>(a.lin_v)[(((long long)b * a.lin_rows + i) * a.Hkv + kv) * (a.Dv / 8) + c] = x;
+        }
+    }
+}
+
 template <typename T>
 __global__ void prefill_simt_kernel(const __grid_constant__ LayerArgs L, const __grid_constant__ PrefillArgs a)
 {
@@ -81,18 +169,17 @@ __global__ void prefill_simt_kernel(const __grid_constant__ LayerArgs L, const _
     const int b = blockIdx.z;
     if (i >= a.S)
         return;
-    const double pos = a.positions ? (double)__ldg(a.positions + i) : (double)i;
     const int half = L.rope.half;
+    const float2 *cs = a.rope_table + (size_t)i * half;
     const T *q = reinterpret_cast<const T *>(a.q) + (((size_t)b * a.S + i) * L.Hq + h) * L.Dqk;
     for (int e = lane; e < L.Dqk; e += 32) {
         float y;
         if (e < L.rope.rotary_dim) {
             const int j = e < half ? e : e - half;
-            float c, s;
-            rope_cos_sin(pos, L.rope.inv_freq[j], c, s);
+            const float2 c = __ldg(cs + j);
             const float xa = to_f32<T>(q[j]);
             const float xb = to_f32<T>(q[j + half]);
-            y = e < half ? xa * c - xb * s : xb * c + xa * s;
+            y = e < half ? xa * c.x - xb * c.y : xb * c.x + xa * c.y;
         } else {
             y = to_f32<T>(q[e]);
         }
@@ -153,9 +240,18 @@ cudaError_t launch_kprep(const KprepArgs &a, int dtype, cudaStream_t stream)
     const long long rows = (long long)a.B * a.S * a.Hkv;
     if (rows == 0)
         return cudaSuccess;
+    if (a.rope.half > 0) {
+        const long long entries = (long long)a.S * a.rope.half;
+        const long long tb = (entries + 255) / 256;
+        rope_table_kernel<<<(unsigned)(tb < 4096 ? tb : 4096), 256, 0, stream>>>(a);
+    }
     const int threads = 256;
     const long long blocks = (rows + (threads / 32) - 1) / (threads / 32);
-    if (dtype == kDtypeBf16)
+    const bool vec = dtype == kDtypeBf16 && a.rope.rotary_dim % 16 == 0 && a.Dqk % 8 == 0 && a.Dv % 8 == 0 &&
+                     (a.rope.half / 8) + (a.Dqk - a.rope.rotary_dim) / 8 + a.Dv / 8 <= 32 * 64;
+    if (vec)
+        kprep_bf16_vec_kernel<<<(unsigned)blocks, threads, 0, stream>>>(a);
+    else if (dtype == kDtypeBf16)
         kprep_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, stream>>>(a);
     else
         kprep_kernel<float><<<(unsigned)blocks, threads, 0, stream>>>(a);

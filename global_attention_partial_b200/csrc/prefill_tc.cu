@@ -297,21 +297,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             // Whole tile visible to every row of the CTA?
             const bool full = (k0 + kBlockN - 1 <= p0) &&
                               (!p.is_swa || k0 >= p0 + p.P - 1 - p.window + 1);
-            float mx = -INFINITY;
-            if (full) {
+            float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (!full) {
+                // branch-free mask: column c is visible iff lo <= c <= hi
+                const int lo = lo_rel - k0;
+                const unsigned span = (unsigned)(hi_rel - lo_rel);
 #pragma unroll
                 for (int c = 0; c < kBlockN; ++c)
-                    mx = fmaxf(mx, x[c]);
-            } else {
-                const int hi = hi_rel - k0;
-                const int lo = lo_rel - k0;
-#pragma unroll
-                for (int c = 0; c < kBlockN; ++c) {
-                    if (c > hi || c < lo)
-                        x[c] = -INFINITY;
-                    mx = fmaxf(mx, x[c]);
-                }
+                    x[c] = ((unsigned)(c - lo) <= span) ? x[c] : -INFINITY;
             }
+#pragma unroll
+            for (int c = 0; c < kBlockN; ++c)
+                mxv[c & 3] = fmaxf(mxv[c & 3], x[c]);
+            const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3]));
             if (mx > m_ref + kRescaleThreshold || (m_ref == -INFINITY && mx > -INFINITY)) {
                 // New reference max: rescale the running sum, and O once an
                 // earlier P*V has landed in it.
@@ -337,20 +335,20 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 m_ref = mx;
             }
             const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-            float rs = 0.f;
+            float rsv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c0 = 0; c0 < kBlockN; c0 += 64) {
                 uint32_t r[32];
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
-                    const float e0 = exp2f(x[c0 + 2 * c] - m_use);
-                    const float e1 = exp2f(x[c0 + 2 * c + 1] - m_use);
-                    rs += e0 + e1;
+                    const float e0 = fast_exp2(x[c0 + 2 * c] - m_use);
+                    const float e1 = fast_exp2(x[c0 + 2 * c + 1] - m_use);
+                    rsv[c & 3] += e0 + e1;
                     r[c] = pack_bf16x2(e0, e1);
                 }
                 tmem_st32(s_addr + c0 / 2, r);
             }
-            l_sum += rs;
+            l_sum += (rsv[0] + rsv[1]) + (rsv[2] + rsv[3]);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars->p_full[sb]);
@@ -399,12 +397,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     }
 }
 
+} // namespace
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn encode_fn()
+static EncodeTiledFn encode_fn()
 {
     static EncodeTiledFn fn = nullptr;
     if (fn == nullptr) {
@@ -421,7 +421,7 @@ EncodeTiledFn encode_fn()
 // 4-D bf16 tensor map over [d3][d2][d1][d0] (d0 innermost) with a row pitch
 // of `pitch1` elements between consecutive d1 indices, d1*pitch1 between d2
 // indices, and d2_alloc*d1*pitch1 between d3 indices.
-bool make_map(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+bool make_bf16_map_4d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
               uint64_t d2_alloc, uint64_t d3, uint32_t b0, uint32_t b1, uint32_t b2)
 {
     EncodeTiledFn fn = encode_fn();
@@ -437,7 +437,6 @@ bool make_map(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint
     return r == CUDA_SUCCESS;
 }
 
-} // namespace
 
 bool prefill_tc_supported(const LayerArgs &L)
 {
@@ -462,9 +461,9 @@ cudaError_t launch_prefill_tc(const LayerArgs &L, const PrefillArgs &a, cudaStre
             }
     }
     const int P = kBlockM / gp;
-    if (!make_map(&p.tm_q, a.q, kDqk, L.Hq, a.S, a.S, a.B, 64, gp, P) ||
-        !make_map(&p.tm_k, a.krot, kDqk, L.Hkv, a.S, a.krot_rows, a.B, 64, 1, kBlockN) ||
-        !make_map(&p.tm_v, a.v, kDv, L.Hkv, a.S, a.S, a.B, 64, 1, kBlockN))
+    if (!make_bf16_map_4d(&p.tm_q, a.q, kDqk, L.Hq, a.S, a.S, a.B, 64, gp, P) ||
+        !make_bf16_map_4d(&p.tm_k, a.krot, kDqk, L.Hkv, a.S, a.krot_rows, a.B, 64, 1, kBlockN) ||
+        !make_bf16_map_4d(&p.tm_v, a.v, kDv, L.Hkv, a.S, a.S, a.B, 64, 1, kBlockN))
         return cudaErrorInvalidValue;
     p.out = reinterpret_cast<__nv_bfloat16 *>(a.out);
     p.positions = a.positions;

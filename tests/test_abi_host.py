@@ -114,7 +114,9 @@ def test_prefill_rejects_bad_shapes_and_buffers(lib):
         assert prefill_status(l, seq=0) == mimo.OK
         # well-formed arguments reach the launch step (the hook fails it)
         assert prefill_status(l) == mimo.ERR_CUDA
-        assert prefill_status(g, cache="both", cap=16, ws_bytes=0) == mimo.ERR_CUDA
+        # a global cache takes the rotated keys; the workspace then holds only the RoPE table
+        assert prefill_status(g, cache="both", cap=16, ws_bytes=0) == mimo.ERR_WORKSPACE
+        assert prefill_status(g, cache="both", cap=16, ws_bytes=16 * 32 * 8) == mimo.ERR_CUDA
     finally:
         mimo.mimo_attn_debug_fail_launches(False)
 
@@ -144,9 +146,9 @@ def test_decode_argument_checks(lib):
 
 def test_workspace_sizes(lib):
     l = layer()
-    # rotated keys of every token: B * S * Hkv * Dqk elements, rounded to 256 bytes
-    assert mimo.mimo_attn_prefill_workspace_size(l, mimo.BF16, 1, 4096) == 4096 * 8 * 192 * 2
-    assert mimo.mimo_attn_prefill_workspace_size(l, mimo.FP32, 1, 3) == 256 * math.ceil(3 * 8 * 192 * 4 / 256)
+    # RoPE table [S, r/2] (cos, sin) then rotated keys [B, S, Hkv, Dqk], each rounded to 256 bytes
+    assert mimo.mimo_attn_prefill_workspace_size(l, mimo.BF16, 1, 4096) == 4096 * 32 * 8 + 4096 * 8 * 192 * 2
+    assert mimo.mimo_attn_prefill_workspace_size(l, mimo.FP32, 1, 3) == 3 * 32 * 8 + 256 * math.ceil(3 * 8 * 192 * 4 / 256)
     # one split per sequence on the ring: no partials needed
     assert mimo.mimo_attn_decode_workspace_size(l, mimo.BF16, 64, 128) == 0
     g = layer(layer_type=mimo.GLOBAL, num_kv_heads=4)

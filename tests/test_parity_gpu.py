@@ -91,6 +91,15 @@ def test_bf16_other_dims_cuda_core_path():
     _assert(c, BF, "bf16 64/48")
 
 
+@pytest.mark.parametrize("B,S", [(3, 1000), (5, 777), (1, 2500)])
+def test_swa_prefill_ring_runs_every_output(B, S):
+    """Sliding layers with several KV-group runs per CTA and ring wrap-around
+    (contiguous tile ranges cross (batch, KV head) boundaries)."""
+    spec = synthetic.mimo_layer(1)
+    c, _, _ = check_prefill(spec, B, S, BF, seed=B * 1000 + S, heads=range(0, 64, 3))
+    _assert(c, BF, f"SWA B{B} S{S}")
+
+
 def test_swa_prefill_full_size_every_output():
     """Single SWA layer, B1 S4096 Hq64 Hkv8 qk192 v128 r64 W128: every output."""
     spec = synthetic.SWA_PREFILL.layers[0]
