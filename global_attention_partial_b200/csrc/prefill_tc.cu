@@ -35,15 +35,24 @@ namespace mimo {
 namespace {
 
 constexpr int kBlockM = 128;
-constexpr int kBlockN = 128;
-constexpr int kKStages = 2;
 constexpr int kDqk = 192;
 constexpr int kDv = 128;
 constexpr int kThreads = 192;
 constexpr int kQBytes = kBlockM * kDqk * 2;       // 49152
-constexpr int kKStageBytes = kBlockN * kDqk * 2;  // 49152
-constexpr int kVStageBytes = kBlockN * kDv * 2;   // 32768
 constexpr int kTmemCols = 512;
+
+// Key tile of BN keys, ST-deep K and V rings. Smaller tiles with more stages
+// keep more bytes in flight per SM for the same shared memory.
+template <int BN, int ST> struct TileCfg {
+    static constexpr int kKStageBytes = BN * kDqk * 2;
+    static constexpr int kVStageBytes = BN * kDv * 2;
+    static constexpr int kSmemBytes = 1024 + kQBytes + ST * (kKStageBytes + kVStageBytes) + 256;
+    static_assert(BN % 16 == 0 && BN <= 128, "key tile");
+    static_assert((BN * 128) % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
+    static_assert(kSmemBytes <= 232448, "shared memory");
+};
+constexpr int kBN = 128;     // keys per tile
+constexpr int kStages = 2;   // K/V ring depth
 constexpr int kColS0 = 0;
 constexpr int kColS1 = 128;
 constexpr int kColO = 256;
@@ -64,10 +73,10 @@ struct TcParams {
     RopeArgs rope;
 };
 
-struct SmemBars {
+template <int ST> struct SmemBars {
     uint64_t q_full, q_ready;
-    uint64_t k_full[kKStages], k_empty[kKStages];
-    uint64_t v_full[kKStages], v_empty[kKStages];
+    uint64_t k_full[ST], k_empty[ST];
+    uint64_t v_full[ST], v_empty[ST];
     uint64_t s_full[2], p_full[2];
     uint64_t o_done;
     uint64_t drain;
@@ -75,7 +84,6 @@ struct SmemBars {
     int abort;
 };
 
-constexpr int kSmemBytes = 1024 + kQBytes + kKStages * (kKStageBytes + kVStageBytes) + 256;
 
 // Byte offset of element e of row `row` in a 128B-swizzled operand whose
 // 64-column blocks are `block_bytes` apart.
@@ -86,15 +94,21 @@ __device__ __forceinline__ uint32_t swz_offset(int row, int e, int block_bytes)
     return (uint32_t)(blk * block_bytes + row * 128 + ((chunk ^ (row & 7)) << 4) + ((e & 7) << 1));
 }
 
+template <int BN, int ST>
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ TcParams p)
 {
+    using Cfg = TileCfg<BN, ST>;
+    constexpr int kBlockN = BN;
+    constexpr int kKStages = ST;
+    constexpr int kKStageBytes = Cfg::kKStageBytes;
+    constexpr int kVStageBytes = Cfg::kVStageBytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
     uint8_t *sQ = smem;
     uint8_t *sK = sQ + kQBytes;
     uint8_t *sV = sK + kKStages * kKStageBytes;
-    SmemBars *bars = reinterpret_cast<SmemBars *>(sV + kKStages * kVStageBytes);
+    SmemBars<ST> *bars = reinterpret_cast<SmemBars<ST> *>(sV + kKStages * kVStageBytes);
     volatile int *abort_flag = &bars->abort;
 
     const int warp = threadIdx.x >> 5;
@@ -284,14 +298,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             tc_fence_after();
             const uint32_t s_addr = lane_base + (sb ? kColS1 : kColS0);
             float x[kBlockN];
+            {
+                uint32_t r[kBlockN / 16][16];
 #pragma unroll
-            for (int c0 = 0; c0 < kBlockN; c0 += 32) {
-                uint32_t r[32];
-                tmem_ld32(s_addr + c0, r);
-                tmem_wait_ld(r);
+                for (int c = 0; c < kBlockN / 16; ++c)
+                    tmem_ld16(s_addr + 16 * c, r[c]);
+                tmem_wait_ld_only();
 #pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    x[c0 + c] = __uint_as_float(r[c]) * p.scale_log2;
+                for (int c = 0; c < kBlockN / 16; ++c) {
+                    tmem_tie(r[c]);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        x[16 * c + e] = __uint_as_float(r[c][e]) * p.scale_log2;
+                }
             }
             const int k0 = k_lo + j * kBlockN;
             // Whole tile visible to every row of the CTA?
@@ -337,16 +356,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
             float rsv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c0 = 0; c0 < kBlockN; c0 += 64) {
-                uint32_t r[32];
+            for (int c0 = 0; c0 < kBlockN; c0 += 16) {
+                uint32_t r[8];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
+                for (int c = 0; c < 8; ++c) {
                     const float e0 = fast_exp2(x[c0 + 2 * c] - m_use);
                     const float e1 = fast_exp2(x[c0 + 2 * c + 1] - m_use);
                     rsv[c & 3] += e0 + e1;
                     r[c] = pack_bf16x2(e0, e1);
                 }
-                tmem_st32(s_addr + c0 / 2, r);
+                tmem_st8(s_addr + c0 / 2, r);
             }
             l_sum += (rsv[0] + rsv[1]) + (rsv[2] + rsv[3]);
             tmem_wait_st();
@@ -462,8 +481,8 @@ cudaError_t launch_prefill_tc(const LayerArgs &L, const PrefillArgs &a, cudaStre
     }
     const int P = kBlockM / gp;
     if (!make_bf16_map_4d(&p.tm_q, a.q, kDqk, L.Hq, a.S, a.S, a.B, 64, gp, P) ||
-        !make_bf16_map_4d(&p.tm_k, a.krot, kDqk, L.Hkv, a.S, a.krot_rows, a.B, 64, 1, kBlockN) ||
-        !make_bf16_map_4d(&p.tm_v, a.v, kDv, L.Hkv, a.S, a.S, a.B, 64, 1, kBlockN))
+        !make_bf16_map_4d(&p.tm_k, a.krot, kDqk, L.Hkv, a.S, a.krot_rows, a.B, 64, 1, kBN) ||
+        !make_bf16_map_4d(&p.tm_v, a.v, kDv, L.Hkv, a.S, a.S, a.B, 64, 1, kBN))
         return cudaErrorInvalidValue;
     p.out = reinterpret_cast<__nv_bfloat16 *>(a.out);
     p.positions = a.positions;
@@ -484,14 +503,15 @@ cudaError_t launch_prefill_tc(const LayerArgs &L, const PrefillArgs &a, cudaStre
 
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<kBN, kStages>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             TileCfg<kBN, kStages>::kSmemBytes);
         if (e != cudaSuccess)
             return e;
         attr_set = true;
     }
     dim3 grid(p.num_p_tiles, L.Hkv * p.num_g_tiles, a.B);
-    prefill_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p);
+    prefill_tc_kernel<kBN, kStages><<<grid, kThreads, TileCfg<kBN, kStages>::kSmemBytes, stream>>>(p);
     return cudaGetLastError();
 }
 
