@@ -213,6 +213,8 @@ mimo_attn_status mimo_attn_prefill(const mimo_attn_layer *layer, int dtype, int 
     cudaError_t e;
     if (use_swa_kernel)
         e = mimo::launch_prefill_swa(L, pa, pa.rope_table, num_sms(), s);
+    else if (dtype == MIMO_ATTN_BF16 && mimo::prefill_ga_supported(L))
+        e = mimo::launch_prefill_ga(L, pa, s);
     else if (dtype == MIMO_ATTN_BF16 && mimo::prefill_tc_supported(L))
         e = mimo::launch_prefill_tc(L, pa, s);
     else

@@ -6,7 +6,7 @@
 //   whose key range holds the new token's slot also rotates the new key,
 //   writes key and value into the cache slot (L-1 for a global cache,
 //   (L-1) mod window for a sliding-window ring) and uses its own copy.
-//   K/V tiles of 64 keys stream through a two-stage cp.async pipeline with
+//   K/V tiles of 64 keys stream through a multi-stage cp.async pipeline with
 //   16-byte coalesced loads; each warp takes 16 keys of a tile and runs
 //   S = Q K^T and O += P V on mma.sync m16n8k16 (query heads on M, keys on
 //   N), with the row max / sum reduced by warp shuffles. Warps are merged
@@ -26,13 +26,18 @@ constexpr int kDqk = 192;
 constexpr int kDv = 128;
 constexpr int kThreads = 128;
 constexpr int kTileKeys = 64;
-constexpr int kStages = 2;
 constexpr int kKStride = kDqk + 8;  // elements; 400-byte rows keep ldmatrix conflict-free
 constexpr int kVStride = kDv + 8;   // 272-byte rows
 constexpr int kQStride = kDqk + 8;
 constexpr int kChunkKeys = 1024;    // keys per split on global layers
 constexpr int kStageElems = kTileKeys * (kKStride + kVStride);
-constexpr int kSmemBytes = (16 * kQStride + kStages * kStageElems + kDqk + kDv) * 2;
+// Ring depth x CTAs per SM: the bytes in flight per SM, (stages - 1) x 43 KB x
+// CTAs, must cover the HBM latency at full bandwidth.
+template <int ST> struct DecodeCfg {
+    static constexpr int kSmemBytes = (16 * kQStride + ST * kStageElems + kDqk + kDv) * 2;
+    static constexpr int kCtasPerSm = ST <= 2 ? 2 : 1;
+};
+constexpr int kDecodeStages = 2;
 
 struct DecodeSmem {
     float wm[4][16];
@@ -50,7 +55,8 @@ __device__ __forceinline__ bool kv_len_ok(int layer_type, int Lb, int cap)
     return Lb >= 1 && (layer_type == 1 || Lb <= cap);
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+template <int kStages>
+__global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
     decode_mma_kernel(const __grid_constant__ LayerArgs L, const __grid_constant__ DecodeArgs a)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -583,14 +589,15 @@ cudaError_t launch_decode(const LayerArgs &L, const DecodeArgs &a, int dtype, cu
     if (decode_mma_supported(L, dtype)) {
         static bool attr_set = false;
         if (!attr_set) {
-            cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<kDecodeStages>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 DecodeCfg<kDecodeStages>::kSmemBytes);
             if (e != cudaSuccess)
                 return e;
             attr_set = true;
         }
         dim3 grid(a.max_splits, L.Hkv, a.B);
-        decode_mma_kernel<<<grid, kThreads, kSmemBytes, stream>>>(L, a);
+        decode_mma_kernel<kDecodeStages><<<grid, kThreads, DecodeCfg<kDecodeStages>::kSmemBytes, stream>>>(L, a);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess || a.max_splits <= 1)
             return e;

@@ -60,6 +60,11 @@ cudaError_t launch_prefill_simt(const LayerArgs &L, const PrefillArgs &a, int dt
 bool prefill_tc_supported(const LayerArgs &L);
 cudaError_t launch_prefill_tc(const LayerArgs &L, const PrefillArgs &a, cudaStream_t stream);
 
+// Global-layer prefill with two query heads of a KV group per CTA (needs an
+// even number of query heads per KV head).
+bool prefill_ga_supported(const LayerArgs &L);
+cudaError_t launch_prefill_ga(const LayerArgs &L, const PrefillArgs &a, cudaStream_t stream);
+
 // Sliding-window prefill whose tiles need a single key span (persistent,
 // one CTA per SM); rope_table is the kprep table.
 bool prefill_swa_supported(const LayerArgs &L);

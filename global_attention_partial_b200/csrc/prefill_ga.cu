@@ -1,0 +1,451 @@
+// Prefill attention of a global (causal) MiMo-V2-Flash layer on the sm_100a
+// tensor cores: two query tiles per CTA share every K/V tile.
+//
+// A CTA owns query tiles A and B: the same 128 positions of two query heads
+// of one KV group, so both tiles see the same causal key range and mask, and
+// each K/V tile crosses L2 once for 256 query rows.
+//
+// Shared memory: Q_A and Q_B (2 x 48 KB, loaded once, rotated in place) and a
+// ring of 8 entries of 16 KB. Each key tile j (128 keys) occupies 5
+// consecutive entries: its K in 3 entries (64 dims each) and its V in 2
+// entries (64 value dims each). Entries are released in load order, each after
+// the last MMA that reads it, so the next tiles stream in while this one is
+// used. Every entry is a 128-byte-swizzled block of 128 rows (the TMA
+// SWIZZLE_128B layout): K-major for QK^T, MN-major for PV.
+//
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
+// P (bf16) is written over the S columns it replaces.
+//
+// MMA order (one thread): QK_A(0), QK_B(0), then for j >= 1:
+//   PV_A(j-1), QK_A(j), PV_B(j-1), QK_B(j)
+// and finally PV_A(n-1), PV_B(n-1). While softmax A works on S_A(j), the
+// tensor cores run PV_B(j-1) and QK_B(j), and the other way round. Because
+// the tensor core completes one thread's MMAs in order, S_A(j) being ready
+// also means PV_A(j-1) has landed in O_A, so a softmax thread may rescale its
+// O row without a further wait.
+//
+// Warp roles (384 threads = 3 warpgroups; setmaxnreg moves registers from the
+// control warpgroup to the two softmax warpgroups):
+//   warps 0-3   tile A: RoPE of its Q rows, softmax (thread r owns row r),
+//               conditional O rescale, epilogue.
+//   warps 4-7   tile B: the same.
+//   warp 8      TMA producer.
+//   warp 9      MMA issuer (and TMEM owner).
+//   warps 10-11 idle.
+#include "kernels.cuh"
+
+#include <math.h>
+
+namespace mimo {
+namespace {
+
+constexpr int kBlockM = 128;
+constexpr int kBlockN = 128;
+constexpr int kDqk = 192;
+constexpr int kDv = 128;
+constexpr int kThreads = 384;
+constexpr int kQBytes = kBlockM * kDqk * 2;   // 49152 per tile
+constexpr int kEntryBytes = kBlockN * 128;    // 16384: 128 rows x 64 columns
+constexpr int kRing = 8;
+constexpr int kEntriesPerTile = 5;            // K: 3, V: 2
+constexpr int kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;     // log2 units
+
+// Register split: the block launches with kThreads x kLaunchRegs (ptxas must
+// report exactly kLaunchRegs); the warpgroup shares add up to that pool.
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsControl = 88;
+static_assert(128 * (2 * kRegsSoftmax + kRegsControl) == kThreads * kLaunchRegs,
+              "warpgroup register shares must add up to the launch pool");
+
+__device__ __forceinline__ uint32_t col_s(int t) { return t ? 128u : 0u; }
+__device__ __forceinline__ uint32_t col_o(int t) { return t ? 384u : 256u; }
+
+struct GaParams {
+    CUtensorMap tm_q;  // [B, S, Hq, Dqk]     box {64, 1, 128, 1}
+    CUtensorMap tm_k;  // [B, rows, Hkv, Dqk] box {64, 1, 128, 1}
+    CUtensorMap tm_v;  // [B, S, Hkv, Dv]     box {64, 1, 128, 1}
+    __nv_bfloat16 *out;
+    const float2 *rope_table;  // [S][half]
+    const float *sinks;        // nullptr on global layers
+    unsigned *err;
+    int S, Hq, G, num_p_tiles, num_pairs;
+    int rope_half;
+    float scale_log2;
+    float v_scale;
+};
+
+struct Bars {
+    uint64_t q_full, q_ready[2];
+    uint64_t ring_full[kRing], ring_empty[kRing];
+    uint64_t s_full[2], p_full[2], pv_done[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+constexpr int kSmemBytes = 1024 + 2 * kQBytes + kRing * kEntryBytes + (int)sizeof(Bars) + 64;
+static_assert(kSmemBytes <= 232448, "shared memory");
+
+__global__ void __launch_bounds__(kThreads, 1) prefill_ga_kernel(const __grid_constant__ GaParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    uint8_t *sQ = smem;                  // Q_A, Q_B
+    uint8_t *sRing = sQ + 2 * kQBytes;   // kRing entries
+    Bars *bars = reinterpret_cast<Bars *>(sRing + kRing * kEntryBytes);
+    volatile int *abort_flag = &bars->abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // Heaviest causal tiles first.
+    const int pt = p.num_p_tiles - 1 - (int)blockIdx.x;
+    const int pair = (int)blockIdx.y;   // kv head * (G/2) + pair within the group
+    const int b = (int)blockIdx.z;
+    const int kvh = pair / (p.G / 2);
+    const int hA = kvh * p.G + 2 * (pair % (p.G / 2));
+    const int p0 = pt * kBlockM;
+    const int q_last = min(p0 + kBlockM, p.S) - 1;
+    const int n_tiles = q_last / kBlockN + 1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->q_full, 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&bars->q_ready[t], 128);
+            mbar_init(&bars->s_full[t], 1);
+            mbar_init(&bars->p_full[t], 128);
+            mbar_init(&bars->pv_done[t], 1);
+        }
+        for (int i = 0; i < kRing; ++i) {
+            mbar_init(&bars->ring_full[i], 1);
+            mbar_init(&bars->ring_empty[i], 1);
+        }
+        mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 9) {
+        tmem_alloc(&bars->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp >= 8) {
+        setmaxnreg_dec<kRegsControl>();
+        if (warp == 8 && lane == 0) {
+            // -------------------------------------------------- TMA producer
+            tma_prefetch_desc(&p.tm_q);
+            tma_prefetch_desc(&p.tm_k);
+            tma_prefetch_desc(&p.tm_v);
+            mbar_arrive_expect_tx(&bars->q_full, 2 * kQBytes);
+            for (int t = 0; t < 2; ++t)
+                for (int a = 0; a < 3; ++a)
+                    tma_load_4d(sQ + t * kQBytes + a * kEntryBytes, &p.tm_q, &bars->q_full, a * 64, hA + t, p0, b);
+            const int n_entries = n_tiles * kEntriesPerTile;
+            int e = 0;
+            for (; e < n_entries; ++e) {
+                const int slot = e % kRing;
+                if (!mbar_wait(&bars->ring_empty[slot], ((uint32_t)(e / kRing) & 1u) ^ 1u, abort_flag, p.err))
+                    break;
+                const int j = e / kEntriesPerTile;
+                const int part = e - j * kEntriesPerTile;
+                mbar_arrive_expect_tx(&bars->ring_full[slot], kEntryBytes);
+                if (part < 3)
+                    tma_load_4d(sRing + slot * kEntryBytes, &p.tm_k, &bars->ring_full[slot], part * 64, kvh,
+                                j * kBlockN, b);
+                else
+                    tma_load_4d(sRing + slot * kEntryBytes, &p.tm_v, &bars->ring_full[slot], (part - 3) * 64,
+                                kvh, j * kBlockN, b);
+            }
+            if (*abort_flag) {
+                mbar_drain(&bars->q_full, 0);
+                for (int x = max(0, e - kRing); x < e; ++x)
+                    mbar_drain(&bars->ring_full[x % kRing], (uint32_t)(x / kRing) & 1u);
+            }
+        } else if (warp == 9 && lane == 0) {
+            // ---------------------------------------------------- MMA issuer
+            const uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, false, false);
+            const uint32_t idesc_pv64 = idesc_bf16_f32(kBlockM, 64, false, true);
+            const uint32_t idesc_pv128 = idesc_bf16_f32(kBlockM, 128, false, true);
+            const uint32_t q_addr = smem_u32(sQ);
+            const uint32_t ring_addr = smem_u32(sRing);
+            bool ok = true;
+            auto wait_entry = [&](int e) -> bool {
+                return mbar_wait(&bars->ring_full[e % kRing], (uint32_t)(e / kRing) & 1u, abort_flag, p.err);
+            };
+            auto issue_qk = [&](int t, int j) -> bool {
+                if (j == 0 && !mbar_wait(&bars->q_ready[t], 0, abort_flag, p.err))
+                    return false;
+                const uint32_t d = tmem + col_s(t);
+                for (int atom = 0; atom < 3; ++atom) {
+                    const int e = j * kEntriesPerTile + atom;
+                    if (t == 0 && !wait_entry(e))
+                        return false;
+                    tc_fence_after();
+                    const uint32_t slot_addr = ring_addr + (e % kRing) * kEntryBytes;
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const uint32_t off = (uint32_t)k4 * 32u;
+                        umma_ss(d, sdesc_sw128(q_addr + t * kQBytes + atom * kEntryBytes + off, 16, 1024),
+                                sdesc_sw128(slot_addr + off, 16, 1024), idesc_qk, (atom | k4) ? 1u : 0u);
+                    }
+                    if (t == 1)
+                        umma_commit(&bars->ring_empty[e % kRing]);  // last reader of this K entry
+                }
+                umma_commit(&bars->s_full[t]);
+                return true;
+            };
+            auto issue_pv = [&](int t, int j) -> bool {
+                if (!mbar_wait(&bars->p_full[t], (uint32_t)j & 1u, abort_flag, p.err))
+                    return false;
+                const int e0 = j * kEntriesPerTile + 3;  // V: value dims 0-63, then 64-127
+                if (t == 0 && !(wait_entry(e0) && wait_entry(e0 + 1)))
+                    return false;
+                tc_fence_after();
+                const int s0 = e0 % kRing;
+                if (s0 + 1 < kRing) {
+                    // both halves in adjacent entries: one N = 128 MMA per 16 keys
+                    const uint32_t v_addr = ring_addr + s0 * kEntryBytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBlockN / 16; ++kk)
+                        umma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
+                                sdesc_sw128(v_addr + kk * 2048, kEntryBytes, 1024), idesc_pv128,
+                                (j > 0 || kk > 0) ? 1u : 0u);
+                } else {
+                    // the pair wraps around the ring: one N = 64 MMA per half
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t v_addr = ring_addr + ((e0 + h) % kRing) * kEntryBytes;
+#pragma unroll
+                        for (int kk = 0; kk < kBlockN / 16; ++kk)
+                            umma_ts(tmem + col_o(t) + 64 * h, tmem + col_s(t) + kk * 8,
+                                    sdesc_sw128(v_addr + kk * 2048, kEntryBytes, 1024), idesc_pv64,
+                                    (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                }
+                if (t == 1) {  // last reader of both V entries
+                    umma_commit(&bars->ring_empty[e0 % kRing]);
+                    umma_commit(&bars->ring_empty[(e0 + 1) % kRing]);
+                }
+                umma_commit(&bars->pv_done[t]);
+                return true;
+            };
+            ok = issue_qk(0, 0) && issue_qk(1, 0);
+            for (int j = 1; ok && j < n_tiles; ++j)
+                ok = issue_pv(0, j - 1) && issue_qk(0, j) && issue_pv(1, j - 1) && issue_qk(1, j);
+            if (ok)
+                ok = issue_pv(0, n_tiles - 1) && issue_pv(1, n_tiles - 1);
+            if (!ok) {
+                umma_commit(&bars->drain);
+                mbar_drain(&bars->drain, 0);
+            }
+        }
+    } else {
+        // ------------------------------------------ softmax of tile t (A or B)
+        setmaxnreg_inc<kRegsSoftmax>();
+        const int t = warp >> 2;
+        const int row = threadIdx.x & 127;
+        const int i = p0 + row;              // sequence index of this row
+        const int h = hA + t;
+        const bool row_valid = i < p.S;
+        const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        bool ok = mbar_wait(&bars->q_full, 0, abort_flag, p.err);
+
+        // Partial RoPE of this row of Q_t, in place in swizzled shared memory.
+        const int half = p.rope_half;
+        if (ok && row_valid && half > 0) {
+            uint8_t *qt = sQ + t * kQBytes;
+            const float2 *cs = p.rope_table + (size_t)i * half;
+            for (int j = 0; j < half; ++j) {
+                const int ea = j, eb = j + half;
+                __nv_bfloat16 *pa = reinterpret_cast<__nv_bfloat16 *>(
+                    qt + (ea >> 6) * kEntryBytes + row * 128 + ((((ea & 63) >> 3) ^ (row & 7)) << 4) + ((ea & 7) << 1));
+                __nv_bfloat16 *pb = reinterpret_cast<__nv_bfloat16 *>(
+                    qt + (eb >> 6) * kEntryBytes + row * 128 + ((((eb & 63) >> 3) ^ (row & 7)) << 4) + ((eb & 7) << 1));
+                const float xa = __bfloat162float(*pa);
+                const float xb = __bfloat162float(*pb);
+                const float2 c = __ldg(cs + j);
+                *pa = __float2bfloat16_rn(xa * c.x - xb * c.y);
+                *pb = __float2bfloat16_rn(xb * c.x + xa * c.y);
+            }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bars->q_ready[t]);
+
+        float m_ref = -INFINITY;  // reference max (base-2 units) of P and O
+        float l_sum = 0.f;
+        const uint32_t s_addr = lane_base + col_s(t);
+        const uint32_t o_addr = lane_base + col_o(t);
+        for (int j = 0; ok && j < n_tiles; ++j) {
+            if (!mbar_wait(&bars->s_full[t], (uint32_t)j & 1u, abort_flag, p.err)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float x[kBlockN];
+            {
+                uint32_t r[kBlockN / 16][16];
+#pragma unroll
+                for (int c = 0; c < kBlockN / 16; ++c)
+                    tmem_ld16(s_addr + 16 * c, r[c]);
+                tmem_wait_ld_only();
+#pragma unroll
+                for (int c = 0; c < kBlockN / 16; ++c) {
+                    tmem_tie(r[c]);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        x[16 * c + e] = __uint_as_float(r[c][e]);  // raw scores; scale folded below
+                }
+            }
+            const int k0 = j * kBlockN;
+            if (k0 + kBlockN - 1 > p0) {
+                // diagonal tile: key c visible iff k0 + c <= i (branch-free)
+                const int hi = i - k0;
+#pragma unroll
+                for (int c = 0; c < kBlockN; ++c)
+                    x[c] = (c <= hi) ? x[c] : -INFINITY;
+            }
+            float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < kBlockN; ++c)
+                mxv[c & 3] = fmaxf(mxv[c & 3], x[c]);
+            const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])) * p.scale_log2;
+            if (mx > m_ref + kRescaleThreshold || (m_ref == -INFINITY && mx > -INFINITY)) {
+                // New reference max; O already holds P*V of tiles < j (in-order MMAs).
+                const float corr = (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - mx);
+                if (j > 0 && m_ref != -INFINITY) {
+#pragma unroll
+                    for (int c0 = 0; c0 < kDv; c0 += 32) {
+                        uint32_t r[32];
+                        tmem_ld32(o_addr + c0, r);
+                        tmem_wait_ld(r);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            r[c] = __float_as_uint(__uint_as_float(r[c]) * corr);
+                        tmem_st32(o_addr + c0, r);
+                    }
+                }
+                l_sum *= corr;
+                m_ref = mx;
+            }
+            const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+            const float sc = p.scale_log2;
+            float rsv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int c0 = 0; c0 < kBlockN; c0 += 16) {
+                uint32_t r[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const float e0 = fast_exp2(fmaf(x[c0 + 2 * c], sc, -m_use));
+                    const float e1 = fast_exp2(fmaf(x[c0 + 2 * c + 1], sc, -m_use));
+                    rsv[c & 3] += e0 + e1;
+                    r[c] = pack_bf16x2(e0, e1);
+                }
+                tmem_st8(s_addr + c0 / 2, r);
+            }
+            l_sum += (rsv[0] + rsv[1]) + (rsv[2] + rsv[3]);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->p_full[t]);
+        }
+
+        // ----------------------------------------------------------- epilogue
+        if (ok && mbar_wait(&bars->pv_done[t], (uint32_t)(n_tiles - 1) & 1u, abort_flag, p.err)) {
+            tc_fence_after();
+            float o_scale;
+            if (p.sinks != nullptr) {
+                const float s2 = __ldg(p.sinks + h) * kLog2e;
+                const float m_fin = fmaxf(m_ref, s2);
+                const float a = exp2f(m_ref - m_fin);
+                o_scale = a * p.v_scale / (l_sum * a + exp2f(s2 - m_fin));
+            } else {
+                o_scale = p.v_scale / l_sum;
+            }
+            uint32_t o[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                tmem_ld32(o_addr + 32 * c, o[c]);
+            tmem_wait_ld_only();
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                tmem_tie(o[c]);
+            if (row_valid) {
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (((size_t)b * p.S + i) * p.Hq + h) * kDv);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(o[c][c8 * 8 + 0]) * o_scale, __uint_as_float(o[c][c8 * 8 + 1]) * o_scale);
+                        w.y = pack_bf16x2(__uint_as_float(o[c][c8 * 8 + 2]) * o_scale, __uint_as_float(o[c][c8 * 8 + 3]) * o_scale);
+                        w.z = pack_bf16x2(__uint_as_float(o[c][c8 * 8 + 4]) * o_scale, __uint_as_float(o[c][c8 * 8 + 5]) * o_scale);
+                        w.w = pack_bf16x2(__uint_as_float(o[c][c8 * 8 + 6]) * o_scale, __uint_as_float(o[c][c8 * 8 + 7]) * o_scale);
+                        dst[c * 4 + c8] = w;
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+} // namespace
+
+bool prefill_ga_supported(const LayerArgs &L)
+{
+    return L.layer_type == 0 && L.Dqk == kDqk && L.Dv == kDv && L.G % 2 == 0 && L.rope.rotary_dim <= kDqk;
+}
+
+cudaError_t launch_prefill_ga(const LayerArgs &L, const PrefillArgs &a, cudaStream_t stream)
+{
+    GaParams p;
+    memset(&p, 0, sizeof(p));
+    if (!make_bf16_map_4d(&p.tm_q, a.q, kDqk, L.Hq, a.S, a.S, a.B, 64, 1, kBlockM) ||
+        !make_bf16_map_4d(&p.tm_k, a.krot, kDqk, L.Hkv, a.S, a.krot_rows, a.B, 64, 1, kBlockN) ||
+        !make_bf16_map_4d(&p.tm_v, a.v, kDv, L.Hkv, a.S, a.S, a.B, 64, 1, kBlockN))
+        return cudaErrorInvalidValue;
+    p.out = reinterpret_cast<__nv_bfloat16 *>(a.out);
+    p.rope_table = a.rope_table;
+    p.sinks = L.sinks;
+    p.err = a.err;
+    p.S = a.S;
+    p.Hq = L.Hq;
+    p.G = L.G;
+    p.num_p_tiles = (a.S + kBlockM - 1) / kBlockM;
+    p.num_pairs = L.Hkv * (L.G / 2);
+    p.rope_half = L.rope.half;
+    p.scale_log2 = L.scale_log2;
+    p.v_scale = L.v_scale;
+
+    static bool attr_set = false;
+    if (!attr_set) {
+        // The setmaxnreg split needs a launch with exactly kLaunchRegs registers.
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, prefill_ga_kernel);
+        if (e != cudaSuccess)
+            return e;
+        if (fa.numRegs != kLaunchRegs)
+            return cudaErrorInvalidConfiguration;
+        e = cudaFuncSetAttribute(prefill_ga_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess)
+            return e;
+        attr_set = true;
+    }
+    dim3 grid(p.num_p_tiles, p.num_pairs, a.B);
+    prefill_ga_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p);
+    return cudaGetLastError();
+}
+
+} // namespace mimo
