@@ -29,7 +29,7 @@ constexpr int kTileKeys = 64;
 constexpr int kKStride = kDqk + 8;  // elements; 400-byte rows keep ldmatrix conflict-free
 constexpr int kVStride = kDv + 8;   // 272-byte rows
 constexpr int kQStride = kDqk + 8;
-constexpr int kChunkKeys = 1024;    // keys per split on global layers
+constexpr int kChunkKeys = 2048;    // keys per split on global layers
 constexpr int kStageElems = kTileKeys * (kKStride + kVStride);
 // Ring depth x CTAs per SM: the bytes in flight per SM, (stages - 1) x 43 KB x
 // CTAs, must cover the HBM latency at full bandwidth.
@@ -90,6 +90,41 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
     const int G = L.G;
     const int half = L.rope.half;
 
+    const size_t kv_row = (size_t)L.Hkv;  // rows of the cache are [slot][Hkv][D]
+    const __nv_bfloat16 *kc = reinterpret_cast<const __nv_bfloat16 *>(a.k_cache) +
+                              ((size_t)b * a.cap * kv_row + kvh) * kDqk;
+    const __nv_bfloat16 *vc = reinterpret_cast<const __nv_bfloat16 *>(a.v_cache) +
+                              ((size_t)b * a.cap * kv_row + kvh) * kDv;
+
+    // The first K/V tiles go out before anything else, so their latency
+    // overlaps the query preparation below.
+    const int n_tiles = (key_end - key_begin + kTileKeys - 1) / kTileKeys;
+    auto issue = [&](int t) {
+        __nv_bfloat16 *st = sStage + (t % kStages) * kStageElems;
+        const int base_key = key_begin + t * kTileKeys;
+        for (int c = tid; c < kTileKeys * 40; c += kThreads) {
+            const int r = c / 40;
+            const int ch = c - r * 40;
+            const int key = base_key + r;
+            const bool valid = key < key_end && key != slot_new;
+            const int ks = valid ? key : key_begin;
+            if (ch < 24) {
+                cp_async16(st + r * kKStride + ch * 8, kc + (size_t)ks * kv_row * kDqk + ch * 8,
+                           valid ? 16u : 0u);
+            } else {
+                const int cv = ch - 24;
+                cp_async16(st + kTileKeys * kKStride + r * kVStride + cv * 8,
+                           vc + (size_t)ks * kv_row * kDv + cv * 8, valid ? 16u : 0u);
+            }
+        }
+    };
+#pragma unroll
+    for (int s = 0; s < kStages - 1; ++s) {
+        if (s < n_tiles)
+            issue(s);
+        cp_async_commit();
+    }
+
     // cos/sin of the new token's position for every rotary pair, once per CTA
     __shared__ float2 s_cs[kMaxHalfRotary];
     for (int j = tid; j < half; j += kThreads) {
@@ -99,16 +134,62 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
     }
     __syncthreads();
 
-    const size_t kv_row = (size_t)L.Hkv;  // rows of the cache are [slot][Hkv][D]
-    const __nv_bfloat16 *kc = reinterpret_cast<const __nv_bfloat16 *>(a.k_cache) +
-                              ((size_t)b * a.cap * kv_row + kvh) * kDqk;
-    const __nv_bfloat16 *vc = reinterpret_cast<const __nv_bfloat16 *>(a.v_cache) +
-                              ((size_t)b * a.cap * kv_row + kvh) * kDv;
-
-    // Query heads of this KV group, rotated at position L-1 (rows >= G are 0).
-    {
-        const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(a.q) +
-                                  ((size_t)b * L.Hq + (size_t)kvh * G) * kDqk;
+    const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(a.q) +
+                              ((size_t)b * L.Hq + (size_t)kvh * G) * kDqk;
+    if (L.rope.rotary_dim % 16 == 0) {
+        // Query heads of this KV group, rotated at position L-1 (rows >= G are
+        // 0), in 16-byte units: a rotary unit is a chunk pair (c, c + r/16), a
+        // copy unit one pass-through chunk. All loads are issued before use.
+        const int npair = half / 8;
+        const int per_row = npair + (kDqk - L.rope.rotary_dim) / 8;
+        uint4 va[3], vb[3];
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            const int u = tid + k * kThreads;
+            const int r = u / per_row;
+            const int w = u - r * per_row;
+            va[k] = make_uint4(0, 0, 0, 0);
+            vb[k] = make_uint4(0, 0, 0, 0);
+            if (r < G && r < 16) {
+                const uint4 *qr = reinterpret_cast<const uint4 *>(qg + (size_t)r * kDqk);
+                if (w < npair) {
+                    va[k] = __ldg(qr + w);
+                    vb[k] = __ldg(qr + w + npair);
+                } else {
+                    va[k] = __ldg(qr + npair + w);
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            const int u = tid + k * kThreads;
+            const int r = u / per_row;
+            const int w = u - r * per_row;
+            if (r >= 16)
+                continue;
+            uint4 *dst = reinterpret_cast<uint4 *>(sQ + r * kQStride);
+            if (w < npair) {
+                uint4 ya, yb;
+                const uint32_t *pa = reinterpret_cast<const uint32_t *>(&va[k]);
+                const uint32_t *pb = reinterpret_cast<const uint32_t *>(&vb[k]);
+                uint32_t *qa = reinterpret_cast<uint32_t *>(&ya);
+                uint32_t *qb = reinterpret_cast<uint32_t *>(&yb);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 c0 = s_cs[w * 8 + 2 * e];
+                    const float2 c1 = s_cs[w * 8 + 2 * e + 1];
+                    const float2 xa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pa[e]));
+                    const float2 xb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pb[e]));
+                    qa[e] = pack_bf16x2(xa.x * c0.x - xb.x * c0.y, xa.y * c1.x - xb.y * c1.y);
+                    qb[e] = pack_bf16x2(xb.x * c0.x + xa.x * c0.y, xb.y * c1.x + xa.y * c1.y);
+                }
+                dst[w] = ya;
+                dst[w + npair] = yb;
+            } else {
+                dst[npair + w] = va[k];
+            }
+        }
+    } else {
         for (int idx = tid; idx < 16 * kDqk; idx += kThreads) {
             const int r = idx / kDqk;
             const int e = idx - r * kDqk;
@@ -172,33 +253,6 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
             ldmatrix_x4(base + ks * 32, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
     }
 
-    const int n_tiles = (key_end - key_begin + kTileKeys - 1) / kTileKeys;
-    auto issue = [&](int t) {
-        __nv_bfloat16 *st = sStage + (t % kStages) * kStageElems;
-        const int base_key = key_begin + t * kTileKeys;
-        for (int c = tid; c < kTileKeys * 40; c += kThreads) {
-            const int r = c / 40;
-            const int ch = c - r * 40;
-            const int key = base_key + r;
-            const bool valid = key < key_end && key != slot_new;
-            const int ks = valid ? key : key_begin;
-            if (ch < 24) {
-                cp_async16(st + r * kKStride + ch * 8, kc + (size_t)ks * kv_row * kDqk + ch * 8,
-                           valid ? 16u : 0u);
-            } else {
-                const int cv = ch - 24;
-                cp_async16(st + kTileKeys * kKStride + r * kVStride + cv * 8,
-                           vc + (size_t)ks * kv_row * kDv + cv * 8, valid ? 16u : 0u);
-            }
-        }
-    };
-#pragma unroll
-    for (int s = 0; s < kStages - 1; ++s) {
-        if (s < n_tiles)
-            issue(s);
-        cp_async_commit();
-    }
-
     const int g = lane >> 2;  // row (head) g and g + 8
     const int tq = lane & 3;
     float m0 = -INFINITY, m1 = -INFINITY;  // running max of rows g, g+8 (base 2)
@@ -226,7 +280,6 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
         if (t + kStages - 1 < n_tiles)
             issue(t + kStages - 1);
         cp_async_commit();
-
         const int kb = warp * 16;  // this warp's 16 keys within the tile
         if (base_key + kb >= key_end)
             continue;

@@ -13,22 +13,26 @@
 // and freed after the PV of the last tile that uses it. Q tiles stream through
 // two buffers.
 //
-// Warp roles (384 threads = 3 warpgroups, one CTA per SM; setmaxnreg moves
-// registers from the control warpgroup to the softmax and epilogue ones):
-//   warps 0-3   softmax: thread r owns row r; loads its 144 S values from
-//               TMEM at once, masks the window, takes the row max and sum,
-//               writes P (bf16) over the S columns and hands (max, sum) to
-//               the epilogue.
-//   warps 4-7   partial RoPE of the next Q tile, in place in swizzled shared
-//               memory (cos/sin from the table kprep wrote), then the
-//               epilogue of the current tile: loads O from TMEM, frees it,
-//               folds the sink, normalises, applies the V scale, stores.
-//   warp 8      TMA producer: Q tiles and K/V ring blocks.
-//   warp 9      MMA issuer: QK^T of tile n+1 and PV of tile n, in whichever
-//               order their inputs become ready.
-//   warps 10-11 idle (the control warpgroup gives up its registers).
+// Two worker warpgroups take alternate tiles (tile n goes to warpgroup n % 2),
+// so one softmax overlaps the other tile's MMAs and epilogue. A worker
+// rotates its Q tile (partial RoPE, in place in swizzled shared memory, cos /
+// sin from the table kprep wrote), runs the softmax (thread r owns row r: the
+// row's 144 S values from TMEM, window mask, max, P as bf16 over the S
+// columns), then the epilogue (O from TMEM, sink fold, normalise, V scale,
+// store). Both workers run the same code, which keeps the instruction cache
+// warm.
 //
-// TMEM (512 columns): S0 [0,144), S1 [160,304), O [320,448).
+// Warp roles (384 threads = 3 warpgroups; setmaxnreg moves registers from the
+// control warpgroup to the workers):
+//   warps 0-3   worker for even tiles    warps 4-7   worker for odd tiles
+//   warp 8      TMA producer: Q tiles and K/V ring blocks
+//   warp 9      MMA issuer: QK^T and PV of the tiles in flight, in whichever
+//               order their inputs become ready
+//   warps 10-11 idle
+//
+// TMEM (512 columns), per worker t: S_t = [256t, 256t + 144) and
+// O_t = [256t + 72, 256t + 200). O overlaps the upper S columns, which are
+// dead once the softmax has read them; P (bf16) takes the first 72 columns.
 // Shared memory: Q 2 x 48 KB; K ring 12 x 16 keys x 384 B; V ring 12 x 16
 // keys x 256 B (128B-swizzled 64-column blocks, 1024-byte aligned).
 #include "kernels.cuh"
@@ -47,12 +51,11 @@ constexpr int kDv = 128;
 constexpr int kThreads = 384;
 // Register split across the three warpgroups. The block launches with
 // kThreads x kLaunchRegs registers (ptxas must report exactly kLaunchRegs);
-// the shares below add up to that pool: 128 * (216 + 208 + 80) = 384 * 168.
+// the shares below add up to that pool: 128 * (208 + 208 + 88) = 384 * 168.
 constexpr int kLaunchRegs = 168;
-constexpr int kRegsSoftmax = 216;
-constexpr int kRegsEpilogue = 208;
-constexpr int kRegsControl = 80;
-static_assert(128 * (kRegsSoftmax + kRegsEpilogue + kRegsControl) == kThreads * kLaunchRegs,
+constexpr int kRegsWorker = 208;
+constexpr int kRegsControl = 88;
+static_assert(128 * (2 * kRegsWorker + kRegsControl) == kThreads * kLaunchRegs,
               "warpgroup register shares must add up to the launch pool");
 constexpr int kQBytes = kBlockM * kDqk * 2;             // 49152
 constexpr int kKAtom = kRing * kKeyBlock * 128;         // 24576: one 64-column block of the K ring
@@ -61,9 +64,9 @@ constexpr int kKBytes = 3 * kKAtom;
 constexpr int kVBytes = 2 * kVAtom;
 constexpr int kEntryBytes = kKeyBlock * (kDqk + kDv) * 2;  // 10240
 constexpr int kTmemCols = 512;
-constexpr int kColO = 320;
 
-__device__ __forceinline__ uint32_t col_s(int buf) { return buf ? 160u : 0u; }
+__device__ __forceinline__ uint32_t col_s(int t) { return t ? 256u : 0u; }
+__device__ __forceinline__ uint32_t col_o(int t) { return col_s(t) + 72u; }
 
 struct SwaParams {
     CUtensorMap tm_q;  // [B, S, Hq, Dqk]    box {64, gp, P, 1}
@@ -83,12 +86,10 @@ struct SwaParams {
 struct Bars {
     uint64_t q_full[2], q_ready[2], q_empty[2];
     uint64_t kv_full[kRing], kv_empty[kRing];
-    uint64_t s_full[2], p_full[2], stats_full[2];
-    uint64_t o_full, o_empty;
+    uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
-    float2 stats[2][kBlockM];  // (row max in base-2 units, row sum) per tile parity
 };
 
 constexpr int kSmemBytes = 1024 + 2 * kQBytes + kKBytes + kVBytes + (int)sizeof(Bars) + 64;
@@ -168,14 +169,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
             mbar_init(&bars->q_empty[i], 1);
             mbar_init(&bars->s_full[i], 1);
             mbar_init(&bars->p_full[i], 128);
-            mbar_init(&bars->stats_full[i], 128);
+            mbar_init(&bars->o_full[i], 1);
+            mbar_init(&bars->o_free[i], 128);
         }
         for (int i = 0; i < kRing; ++i) {
             mbar_init(&bars->kv_full[i], 1);
             mbar_init(&bars->kv_empty[i], 1);
         }
-        mbar_init(&bars->o_full, 1);
-        mbar_init(&bars->o_empty, 128);
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
         fence_barrier_init();
@@ -275,7 +275,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
             bool ok = true;
             while (ok && next_pv < n_local) {
                 bool progressed = false;
-                if (next_qk < n_local && next_qk <= next_pv + 1) {
+                // QK_n needs its worker's S/O columns back (epilogue of tile n-2
+                // done, which also implies PV_{n-2} landed), its rotated Q and its keys.
+                if (next_qk < n_local && mbar_test_wait(&bars->o_free[next_qk & 1], ((uint32_t)(next_qk >> 1) & 1u) ^ 1u)) {
                     const int n = next_qk;
                     const int qb = n & 1;
                     // Span of tile n in ring entries.
@@ -342,18 +344,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 if (next_pv < next_qk) {
                     const int n = next_pv;
                     const int sb = n & 1;
-                    if (mbar_test_wait(&bars->p_full[sb], (uint32_t)(n >> 1) & 1u) &&
-                        mbar_test_wait(&bars->o_empty, ((uint32_t)n & 1u) ^ 1u)) {
+                    if (mbar_test_wait(&bars->p_full[sb], (uint32_t)(n >> 1) & 1u)) {
                         tc_fence_after();
                         const int e0 = sb ? first1 : first0;
                         const int nb = sb ? nb1 : nb0;
                         for (int j = 0; j < nb; ++j) {
                             const int slot = (e0 + j) % kRing;
-                            umma_ts(tmem + kColO, tmem + col_s(sb) + j * 8,
+                            umma_ts(tmem + col_o(sb), tmem + col_s(sb) + j * 8,
                                     sdesc_sw128(v_base + slot * (kKeyBlock * 128), kVAtom, 1024), idesc_pv,
                                     j > 0 ? 1u : 0u);
                         }
-                        umma_commit(&bars->o_full);
+                        umma_commit(&bars->o_full[sb]);
                         // Release the ring entries no later tile uses: all of them
                         // unless tile n+1 (already walked by the QK side when it is
                         // in flight, else computed here) continues the same run.
@@ -399,94 +400,41 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 mbar_drain(&bars->drain, 0);
             }
         }
-    } else if (warp < 4) {
-        // ----------------------------------------------------------- softmax
-        setmaxnreg_inc<kRegsSoftmax>();
-        const int row = threadIdx.x;
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-        for (int n = 0; n < n_local; ++n) {
-            const int sb = n & 1;
-            const Tile c = tile_at(p, t_begin + n);
-            const int i = c.p0 + row / p.gp;
-            const int k0 = c.first_block * kKeyBlock;
-            const int hi = i - k0;                 // last visible column
-            const int lo = i - p.window + 1 - k0;  // first visible column
-            // column c is visible iff (unsigned)(c - lo) <= span (lo <= hi always)
-            const unsigned span = (unsigned)(hi - lo);
-            if (!mbar_wait(&bars->s_full[sb], (uint32_t)(n >> 1) & 1u, abort_flag, p.err))
-                break;
-            tc_fence_after();
-            const uint32_t s_addr = lane_base + col_s(sb);
-            // Two passes over S in 16-column chunks, as compact rolled loops
-            // (small code keeps the instruction cache warm for all roles).
-            float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll 1
-            for (int c0 = 0; c0 < kMaxSpanBlocks * kKeyBlock; c0 += 16) {
-                uint32_t r[16];
-                tmem_ld16(s_addr + c0, r);
-                tmem_wait_ld(r);
-#pragma unroll
-                for (int j = 0; j < 16; j += 2) {
-                    const unsigned d = (unsigned)(c0 + j - lo);
-                    mx0 = fmaxf(mx0, d <= span ? __uint_as_float(r[j]) : -INFINITY);
-                    mx1 = fmaxf(mx1, d + 1u <= span ? __uint_as_float(r[j + 1]) : -INFINITY);
-                }
-            }
-            const float mx = fmaxf(mx0, mx1);
-            const float m2 = mx * p.scale_log2;   // base-2 units
-            const float mu = (mx == -INFINITY) ? 0.f : m2;
-            const float sc = p.scale_log2;
-            float rs0 = 0.f, rs1 = 0.f;
-            // P = exp2(s * scale - max) as bf16 pairs; masked columns give 0.
-            // Chunk c (16 keys) becomes 8 packed columns at c/2: it only
-            // overwrites S columns this thread has already read.
-#pragma unroll 1
-            for (int c0 = 0; c0 < kMaxSpanBlocks * kKeyBlock; c0 += 16) {
-                uint32_t r[16];
-                uint32_t pk[8];
-                tmem_ld16(s_addr + c0, r);
-                tmem_wait_ld(r);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const unsigned d = (unsigned)(c0 + 2 * j - lo);
-                    const float x0 = d <= span ? fmaf(__uint_as_float(r[2 * j]), sc, -mu) : -INFINITY;
-                    const float x1 = d + 1u <= span ? fmaf(__uint_as_float(r[2 * j + 1]), sc, -mu) : -INFINITY;
-                    const float e0 = fast_exp2(x0);
-                    const float e1 = fast_exp2(x1);
-                    rs0 += e0;
-                    rs1 += e1;
-                    pk[j] = pack_bf16x2(e0, e1);
-                }
-                tmem_st8(s_addr + c0 / 2, pk);
-            }
-            const float rs = rs0 + rs1;
-            bars->stats[sb][row] = make_float2(m2, rs);
-            mbar_arrive(&bars->stats_full[sb]);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&bars->p_full[sb]);
-        }
     } else if (warp < 8) {
-        // ------------------------------------------- Q rotation and epilogue
-        setmaxnreg_inc<kRegsEpilogue>();
-        const int row = threadIdx.x - 128;
+        // ------------------------------------------------------------ workers
+        setmaxnreg_inc<kRegsWorker>();
+        const int t = warp >> 2;             // this worker takes tiles n with n % 2 == t
+        const int row = threadIdx.x & 127;
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const uint32_t s_addr = lane_base + col_s(t);
+        const uint32_t o_addr = lane_base + col_o(t);
         const int half = p.rope_half;
-        auto rotate_q = [&](int n) -> bool {
-            const int qb = n & 1;
-            if (!mbar_wait(&bars->q_full[qb], (uint32_t)(n >> 1) & 1u, abort_flag, p.err))
-                return false;
+        const float sc = p.scale_log2;
+        bool ok = true;
+        for (int n = t; ok && n < n_local; n += 2) {
+            const uint32_t ph = (uint32_t)(n >> 1) & 1u;
             const Tile c = tile_at(p, t_begin + n);
             const int i = c.p0 + row / p.gp;
-            if (i < p.S && half > 0) {
-                uint8_t *q_row = sQ + qb * kQBytes + row * 128;
-                const float2 *cs = p.rope_table + (size_t)i * half;
-                if (half == 32) {
-                    // cos/sin of the 32 pairs (16 x 16-byte loads issued together)
-                    float4 t[16];
+            const int h = c.h0 + row % p.gp;
+            // ---- partial RoPE of this row of Q_n (buffer t)
+            // cos/sin of the row's 32 pairs are fetched before waiting for Q,
+            // so their latency overlaps the Q load.
+            const bool fast_rope = half == 32 && i < p.S;
+            float4 tb[16];
+            if (fast_rope) {
+                const float4 *cs4 = reinterpret_cast<const float4 *>(p.rope_table + (size_t)i * half);
 #pragma unroll
-                    for (int w = 0; w < 16; ++w)
-                        t[w] = __ldg(reinterpret_cast<const float4 *>(cs) + w);
+                for (int w = 0; w < 16; ++w)
+                    tb[w] = __ldg(cs4 + w);
+            }
+            if (!mbar_wait(&bars->q_full[t], ph, abort_flag, p.err)) {
+                ok = false;
+                break;
+            }
+            if (i < p.S && half > 0) {
+                uint8_t *q_row = sQ + t * kQBytes + row * 128;
+                const float2 *cs = p.rope_table + (size_t)i * half;
+                if (fast_rope) {
                     // One 128-byte swizzled row: chunks 0-3 hold dims 0-31, 4-7 dims 32-63.
                     uint4 v[8];
 #pragma unroll
@@ -500,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                         for (int w = 0; w < 4; ++w) {
                             const float2 xa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&a[w]));
                             const float2 xb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&bb[w]));
-                            const float4 cc = t[ch * 4 + w];  // (cos, sin) of pairs 8ch+2w, 8ch+2w+1
+                            const float4 cc = tb[ch * 4 + w];  // (cos, sin) of pairs 8ch+2w, 8ch+2w+1
                             a[w] = pack_bf16x2(xa.x * cc.x - xb.x * cc.y, xa.y * cc.z - xb.y * cc.w);
                             bb[w] = pack_bf16x2(xb.x * cc.x + xa.x * cc.y, xb.y * cc.z + xa.y * cc.w);
                         }
@@ -512,10 +460,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                     for (int j = 0; j < half; ++j) {
                         const int ea = j, eb = j + half;
                         __nv_bfloat16 *pa = reinterpret_cast<__nv_bfloat16 *>(
-                            sQ + qb * kQBytes + (ea >> 6) * (kBlockM * 128) + row * 128 +
+                            sQ + t * kQBytes + (ea >> 6) * (kBlockM * 128) + row * 128 +
                             ((((ea & 63) >> 3) ^ (row & 7)) << 4) + ((ea & 7) << 1));
                         __nv_bfloat16 *pb = reinterpret_cast<__nv_bfloat16 *>(
-                            sQ + qb * kQBytes + (eb >> 6) * (kBlockM * 128) + row * 128 +
+                            sQ + t * kQBytes + (eb >> 6) * (kBlockM * 128) + row * 128 +
                             ((((eb & 63) >> 3) ^ (row & 7)) << 4) + ((eb & 7) << 1));
                         const float xa = __bfloat162float(*pa);
                         const float xb = __bfloat162float(*pb);
@@ -526,61 +474,98 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 }
             }
             fence_proxy_async_smem();
-            mbar_arrive(&bars->q_ready[qb]);
-            return true;
-        };
-        bool ok = n_local > 0 ? rotate_q(0) : true;
-        for (int n = 0; ok && n < n_local; ++n) {
-            if (n + 1 < n_local && !(ok = rotate_q(n + 1)))
-                break;
-            const int sb = n & 1;
-            const Tile c = tile_at(p, t_begin + n);
-            const int i = c.p0 + row / p.gp;
-            const int h = c.h0 + row % p.gp;
-            const float sink2 = p.sinks != nullptr ? __ldg(p.sinks + h) * kLog2e : 0.f;
-            if (!mbar_wait(&bars->stats_full[sb], (uint32_t)(n >> 1) & 1u, abort_flag, p.err) ||
-                !mbar_wait(&bars->o_full, (uint32_t)n & 1u, abort_flag, p.err)) {
+            mbar_arrive(&bars->q_ready[t]);
+
+            // ---- softmax over the tile's key span
+            const int k0 = c.first_block * kKeyBlock;
+            const int lo = i - p.window + 1 - k0;      // first visible column
+            const unsigned span = (unsigned)(p.window - 1);  // column c visible iff c - lo <= span
+            if (!mbar_wait(&bars->s_full[t], ph, abort_flag, p.err)) {
                 ok = false;
                 break;
             }
-            const float2 st = bars->stats[sb][row];
             tc_fence_after();
-            uint32_t o0[32], o1[32], o2[32], o3[32];
-            tmem_ld32(lane_base + kColO + 0, o0);
-            tmem_ld32(lane_base + kColO + 32, o1);
-            tmem_ld32(lane_base + kColO + 64, o2);
-            tmem_ld32(lane_base + kColO + 96, o3);
-            tmem_wait_ld_only();
-            tmem_tie(o0);
-            tmem_tie(o1);
-            tmem_tie(o2);
-            tmem_tie(o3);
+            float x[kMaxSpanBlocks * kKeyBlock];
+            {
+                uint32_t r[kMaxSpanBlocks][16];
+#pragma unroll
+                for (int q = 0; q < kMaxSpanBlocks; ++q)
+                    tmem_ld16(s_addr + 16 * q, r[q]);
+                tmem_wait_ld_only();
+#pragma unroll
+                for (int q = 0; q < kMaxSpanBlocks; ++q) {
+                    tmem_tie(r[q]);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        x[16 * q + e] = __uint_as_float(r[q][e]);
+                }
+            }
+            float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int col = 0; col < kMaxSpanBlocks * kKeyBlock; ++col) {
+                x[col] = ((unsigned)(col - lo) <= span) ? x[col] : -INFINITY;
+                mxv[col & 3] = fmaxf(mxv[col & 3], x[col]);
+            }
+            const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3]));
+            const float m2 = mx * sc;   // base-2 units
+            const float mu = (mx == -INFINITY) ? 0.f : m2;
+            float rsv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int q = 0; q < kMaxSpanBlocks; ++q) {
+                uint32_t pk[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float e0 = fast_exp2(fmaf(x[16 * q + 2 * e], sc, -mu));
+                    const float e1 = fast_exp2(fmaf(x[16 * q + 2 * e + 1], sc, -mu));
+                    rsv[e & 3] += e0 + e1;
+                    pk[e] = pack_bf16x2(e0, e1);
+                }
+                tmem_st8(s_addr + 8 * q, pk);
+            }
+            const float rs = (rsv[0] + rsv[1]) + (rsv[2] + rsv[3]);
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars->o_empty);
+            mbar_arrive(&bars->p_full[t]);
+
+            // ---- epilogue
             float o_scale;
             if (p.sinks != nullptr) {
-                const float mf = fmaxf(st.x, sink2);
-                const float a = exp2f(st.x - mf);
-                o_scale = a * p.v_scale / (st.y * a + exp2f(sink2 - mf));
+                const float s2 = __ldg(p.sinks + h) * kLog2e;
+                const float mf = fmaxf(m2, s2);
+                const float a = exp2f(m2 - mf);
+                o_scale = a * p.v_scale / (rs * a + exp2f(s2 - mf));
             } else {
-                o_scale = p.v_scale / st.y;
+                o_scale = p.v_scale / rs;
             }
+            if (!mbar_wait(&bars->o_full[t], ph, abort_flag, p.err)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t o[4][32];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                tmem_ld32(o_addr + 32 * q, o[q]);
+            tmem_wait_ld_only();
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                tmem_tie(o[q]);
+            tc_fence_before();
+            mbar_arrive(&bars->o_free[t]);
             if (i < p.S) {
                 uint4 *dst = reinterpret_cast<uint4 *>(p.out + (((size_t)c.b * p.S + i) * p.Hq + h) * kDv);
-#define MIMO_SWA_STORE(O, BASE)                                                                     \
-    _Pragma("unroll") for (int c8 = 0; c8 < 4; ++c8) {                                              \
-        uint4 w;                                                                                    \
-        w.x = pack_bf16x2(__uint_as_float(O[c8 * 8 + 0]) * o_scale, __uint_as_float(O[c8 * 8 + 1]) * o_scale); \
-        w.y = pack_bf16x2(__uint_as_float(O[c8 * 8 + 2]) * o_scale, __uint_as_float(O[c8 * 8 + 3]) * o_scale); \
-        w.z = pack_bf16x2(__uint_as_float(O[c8 * 8 + 4]) * o_scale, __uint_as_float(O[c8 * 8 + 5]) * o_scale); \
-        w.w = pack_bf16x2(__uint_as_float(O[c8 * 8 + 6]) * o_scale, __uint_as_float(O[c8 * 8 + 7]) * o_scale); \
-        dst[(BASE) / 8 + c8] = w;                                                                   \
-    }
-                MIMO_SWA_STORE(o0, 0)
-                MIMO_SWA_STORE(o1, 32)
-                MIMO_SWA_STORE(o2, 64)
-                MIMO_SWA_STORE(o3, 96)
-#undef MIMO_SWA_STORE
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(o[q][c8 * 8 + 0]) * o_scale, __uint_as_float(o[q][c8 * 8 + 1]) * o_scale);
+                        w.y = pack_bf16x2(__uint_as_float(o[q][c8 * 8 + 2]) * o_scale, __uint_as_float(o[q][c8 * 8 + 3]) * o_scale);
+                        w.z = pack_bf16x2(__uint_as_float(o[q][c8 * 8 + 4]) * o_scale, __uint_as_float(o[q][c8 * 8 + 5]) * o_scale);
+                        w.w = pack_bf16x2(__uint_as_float(o[q][c8 * 8 + 6]) * o_scale, __uint_as_float(o[q][c8 * 8 + 7]) * o_scale);
+                        dst[q * 4 + c8] = w;
+                    }
+                }
             }
         }
     }

@@ -160,7 +160,7 @@ MIMO_ATTN_API mimo_attn_status mimo_attn_decode(const mimo_attn_layer *layer, in
  *   - Limit: mimo_attn_decode_workspace_size(layer, dtype, batch,
  *     cache_capacity) must be at most 16 MiB (16777216 bytes), else the call
  *     returns MIMO_ATTN_ERR_WORKSPACE and launches nothing. (Example: 64
- *     query heads, cache 32768, up to 15 sequences per call.)
+ *     query heads, cache 32768, up to 31 sequences per call.)
  *   - The array is device memory held by every GPU that loads the library,
  *     until the process exits.
  *   - The first call on a device looks up the array's device address there

@@ -152,7 +152,7 @@ def test_workspace_sizes(lib):
     # one split per sequence on the ring: no partials needed
     assert mimo.mimo_attn_decode_workspace_size(l, mimo.BF16, 64, 128) == 0
     g = layer(layer_type=mimo.GLOBAL, num_kv_heads=4)
-    splits = 32768 // 1024
+    splits = 32768 // 2048
     assert mimo.mimo_attn_decode_workspace_size(g, mimo.BF16, 64, 32768) == 64 * 64 * splits * 130 * 4
     assert mimo.mimo_attn_prefill_workspace_size(layer(num_kv_heads=7), mimo.BF16, 1, 8) == 0
 

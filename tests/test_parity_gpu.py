@@ -208,8 +208,9 @@ def _check_decode(spec, out, inputs, caches, batches, lens, dtype=BF):
 @pytest.mark.parametrize("layer_type", [0, 1])
 def test_decode_small_every_output(layer_type):
     spec = synthetic.mimo_layer(layer_type)
-    lens = [1, 2, 63, 64, 65, 127, 128, 129, 1023, 1024, 1025, 2000]
-    cap = 2048
+    # lengths around the 64-key tiles, the 128-slot ring and the 2048-key splits
+    lens = [1, 2, 63, 64, 65, 127, 128, 129, 1023, 2047, 2048, 2049, 4097, 5000]
+    cap = 5000
     out, inputs, caches = _run_decode(spec, len(lens), cap, lens)
     _check_decode(spec, out, inputs, caches, range(len(lens)), lens)
 
