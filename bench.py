@@ -365,12 +365,13 @@ def oracle_sample(seconds: float, seed: int = 1, kind: str = "stack"):
 
 
 # ------------------------------------------------------------------ traffic
-def committed_traffic(kernel_tag: str):
-    """Per-launch DRAM bytes of `kernel_tag` from the committed ncu summary,
-    valid only while the kernel source still matches the hash recorded there."""
+def committed_traffic(kernel_tag: str, source: str):
+    """Per-launch DRAM bytes from the committed ncu summary profiles/<kernel_tag>.md,
+    valid only while the kernel's source file (csrc/<source>) still matches the
+    hash recorded there."""
     import hashlib
     path = os.path.join(ROOT, "profiles", f"{kernel_tag}.md")
-    src = os.path.join(ROOT, "global_attention_partial_b200", "csrc", "prefill_tc.cu")
+    src = os.path.join(ROOT, "global_attention_partial_b200", "csrc", source)
     if not os.path.exists(path) or not os.path.exists(src):
         return None
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
@@ -543,14 +544,15 @@ def main():
             ach = prefill_flops(spec, w.pw.batch, w.pw.seq) / (per * 1e-3) / 1e12
             roofline = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
                         "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"],
-                        "traffic": committed_traffic("prefill_tc_global"),
-                        "kernel": "prefill_tc_kernel (global layer, B4 S32768 causal)",
+                        "traffic": committed_traffic("prefill_ga_global", "prefill_ga.cu"),
+                        "kernel": "prefill_ga_kernel (global layer, B4 S32768 causal)",
                         "peak_kind": f"bf16 dense, sustained, {peaks['source']}"}
         else:
             ach = prefill_bytes(spec, w.pw.batch, w.pw.seq) / (per * 1e-3) / 1e9
             roofline = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                        "frac": ach / peaks["hbm_gbs"], "traffic": committed_traffic("prefill_tc_swa"),
-                        "kernel": "prefill_tc_kernel (sliding layer)", "peak_kind": f"HBM copy, {peaks['source']}"}
+                        "frac": ach / peaks["hbm_gbs"],
+                        "traffic": committed_traffic("prefill_swa_sliding", "prefill_swa.cu"),
+                        "kernel": "prefill_swa_kernel (sliding layer)", "peak_kind": f"HBM copy, {peaks['source']}"}
     if w.do_decode:
         per = statistics.mean(kinds["decode_stack"])
         byt = w.decode_bytes()

@@ -78,7 +78,8 @@ struct GaParams {
 
 struct Bars {
     uint64_t q_full, q_ready[2];
-    uint64_t ring_full[kRing], ring_empty[kRing];
+    uint64_t k_full[2], v_full[2];    // per key tile (j & 1): all of its K / V entries landed
+    uint64_t k_free[2], v_free[2];    // per key tile (j & 1): its K / V entries may be overwritten
     uint64_t s_full[2], p_full[2], pv_done[2];
     uint64_t drain;
     uint32_t tmem_base;
@@ -119,9 +120,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_ga_kernel(const __grid_co
             mbar_init(&bars->p_full[t], 128);
             mbar_init(&bars->pv_done[t], 1);
         }
-        for (int i = 0; i < kRing; ++i) {
-            mbar_init(&bars->ring_full[i], 1);
-            mbar_init(&bars->ring_empty[i], 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&bars->k_full[x], 1);
+            mbar_init(&bars->v_full[x], 1);
+            mbar_init(&bars->k_free[x], 1);
+            mbar_init(&bars->v_free[x], 1);
         }
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
@@ -148,99 +151,150 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_ga_kernel(const __grid_co
             for (int t = 0; t < 2; ++t)
                 for (int a = 0; a < 3; ++a)
                     tma_load_4d(sQ + t * kQBytes + a * kEntryBytes, &p.tm_q, &bars->q_full, a * 64, hA + t, p0, b);
-            const int n_entries = n_tiles * kEntriesPerTile;
-            int e = 0;
-            for (; e < n_entries; ++e) {
-                const int slot = e % kRing;
-                if (!mbar_wait(&bars->ring_empty[slot], ((uint32_t)(e / kRing) & 1u) ^ 1u, abort_flag, p.err))
+            // Entry e of the ring (e = 5j + part) may be refilled once entry
+            // e - kRing is free; entries are released per key tile (K and V
+            // separately), so the wait is on the barrier of the tile that
+            // owned it. A tile's K (or V) is issued only once all of its
+            // entries are free, so an abort never leaves a tile half issued.
+            auto wait_free = [&](int e) -> bool {
+                if (e < kRing)
+                    return true;
+                const int jo = (e - kRing) / kEntriesPerTile;
+                const int part = (e - kRing) - jo * kEntriesPerTile;
+                uint64_t *bar = part < 3 ? &bars->k_free[jo & 1] : &bars->v_free[jo & 1];
+                return mbar_wait(bar, (uint32_t)(jo >> 1) & 1u, abort_flag, p.err);
+            };
+            int k_armed[2] = {-1, -1}, v_armed[2] = {-1, -1};
+            for (int j = 0; j < n_tiles; ++j) {
+                const int e = j * kEntriesPerTile;
+                if (!(wait_free(e) && wait_free(e + 1) && wait_free(e + 2)))
                     break;
-                const int j = e / kEntriesPerTile;
-                const int part = e - j * kEntriesPerTile;
-                mbar_arrive_expect_tx(&bars->ring_full[slot], kEntryBytes);
-                if (part < 3)
-                    tma_load_4d(sRing + slot * kEntryBytes, &p.tm_k, &bars->ring_full[slot], part * 64, kvh,
-                                j * kBlockN, b);
-                else
-                    tma_load_4d(sRing + slot * kEntryBytes, &p.tm_v, &bars->ring_full[slot], (part - 3) * 64,
-                                kvh, j * kBlockN, b);
+                mbar_arrive_expect_tx(&bars->k_full[j & 1], 3 * kEntryBytes);
+                k_armed[j & 1] = j;
+                for (int part = 0; part < 3; ++part)
+                    tma_load_4d(sRing + ((e + part) % kRing) * kEntryBytes, &p.tm_k, &bars->k_full[j & 1],
+                                part * 64, kvh, j * kBlockN, b);
+                if (!(wait_free(e + 3) && wait_free(e + 4)))
+                    break;
+                mbar_arrive_expect_tx(&bars->v_full[j & 1], 2 * kEntryBytes);
+                v_armed[j & 1] = j;
+                for (int part = 0; part < 2; ++part)
+                    tma_load_4d(sRing + ((e + 3 + part) % kRing) * kEntryBytes, &p.tm_v, &bars->v_full[j & 1],
+                                part * 64, kvh, j * kBlockN, b);
             }
             if (*abort_flag) {
                 mbar_drain(&bars->q_full, 0);
-                for (int x = max(0, e - kRing); x < e; ++x)
-                    mbar_drain(&bars->ring_full[x % kRing], (uint32_t)(x / kRing) & 1u);
+                for (int x = 0; x < 2; ++x) {
+                    if (k_armed[x] >= 0)
+                        mbar_drain(&bars->k_full[x], (uint32_t)(k_armed[x] >> 1) & 1u);
+                    if (v_armed[x] >= 0)
+                        mbar_drain(&bars->v_full[x], (uint32_t)(v_armed[x] >> 1) & 1u);
+                }
             }
         } else if (warp == 9 && lane == 0) {
             // ---------------------------------------------------- MMA issuer
+            // Straight-line issue: one wait per dependency, no branch between
+            // the MMAs of a group. On sm_100a a single issuing thread loses
+            // tens of cycles per branch or per freshly built descriptor, which
+            // is the whole budget of a 128x128x16 MMA (64 cycles), so the
+            // descriptors are built once and stepped by adding byte offsets
+            // >> 4 to the start-address field (addresses stay below 2^18).
             const uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, false, false);
             const uint32_t idesc_pv64 = idesc_bf16_f32(kBlockM, 64, false, true);
             const uint32_t idesc_pv128 = idesc_bf16_f32(kBlockM, 128, false, true);
-            const uint32_t q_addr = smem_u32(sQ);
-            const uint32_t ring_addr = smem_u32(sRing);
+            const uint32_t q_lo = sdesc_lo(smem_u32(sQ), 16);
+            const uint32_t k_lo = sdesc_lo(smem_u32(sRing), 16);
+            const uint32_t v_lo = sdesc_lo(smem_u32(sRing), kEntryBytes);
+            constexpr uint32_t kStep = kEntryBytes >> 4;
             bool ok = true;
-            auto wait_entry = [&](int e) -> bool {
-                return mbar_wait(&bars->ring_full[e % kRing], (uint32_t)(e / kRing) & 1u, abort_flag, p.err);
+            auto wait = [&](uint64_t *bar, uint32_t parity) {
+                if (!mbar_try_wait(bar, parity) && !mbar_wait(bar, parity, abort_flag, p.err))
+                    ok = false;
             };
-            auto issue_qk = [&](int t, int j) -> bool {
-                if (j == 0 && !mbar_wait(&bars->q_ready[t], 0, abort_flag, p.err))
-                    return false;
+            // S_t = Q_t K_j^T: 3 entries x 4 k-steps of 16.
+            auto qk = [&](int t, int j) {
+                const int e = j * kEntriesPerTile;
+                const uint32_t qa = q_lo + (uint32_t)t * (kQBytes >> 4);
+                const uint32_t kb0 = k_lo + (uint32_t)(e % kRing) * kStep;
+                const uint32_t kb1 = k_lo + (uint32_t)((e + 1) % kRing) * kStep;
+                const uint32_t kb2 = k_lo + (uint32_t)((e + 2) % kRing) * kStep;
                 const uint32_t d = tmem + col_s(t);
-                for (int atom = 0; atom < 3; ++atom) {
-                    const int e = j * kEntriesPerTile + atom;
-                    if (t == 0 && !wait_entry(e))
-                        return false;
-                    tc_fence_after();
-                    const uint32_t slot_addr = ring_addr + (e % kRing) * kEntryBytes;
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        const uint32_t off = (uint32_t)k4 * 32u;
-                        umma_ss(d, sdesc_sw128(q_addr + t * kQBytes + atom * kEntryBytes + off, 16, 1024),
-                                sdesc_sw128(slot_addr + off, 16, 1024), idesc_qk, (atom | k4) ? 1u : 0u);
-                    }
-                    if (t == 1)
-                        umma_commit(&bars->ring_empty[e % kRing]);  // last reader of this K entry
-                }
-                umma_commit(&bars->s_full[t]);
-                return true;
+                for (int k4 = 0; k4 < 4; ++k4)
+                    umma_ss_lo(d, qa + 2 * k4, kb0 + 2 * k4, idesc_qk, k4 ? 1u : 0u);
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4)
+                    umma_ss_lo(d, qa + kStep + 2 * k4, kb1 + 2 * k4, idesc_qk, 1u);
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4)
+                    umma_ss_lo(d, qa + 2 * kStep + 2 * k4, kb2 + 2 * k4, idesc_qk, 1u);
             };
-            auto issue_pv = [&](int t, int j) -> bool {
-                if (!mbar_wait(&bars->p_full[t], (uint32_t)j & 1u, abort_flag, p.err))
-                    return false;
-                const int e0 = j * kEntriesPerTile + 3;  // V: value dims 0-63, then 64-127
-                if (t == 0 && !(wait_entry(e0) && wait_entry(e0 + 1)))
-                    return false;
-                tc_fence_after();
-                const int s0 = e0 % kRing;
+            // O_t (+)= P_t V_j: P from the S_t columns of TMEM, V from its two entries.
+            auto pv = [&](int t, int j) {
+                const int s0 = (j * kEntriesPerTile + 3) % kRing;
+                const uint32_t o = tmem + col_o(t), a = tmem + col_s(t);
+                const uint32_t acc0 = j > 0 ? 1u : 0u;
                 if (s0 + 1 < kRing) {
                     // both halves in adjacent entries: one N = 128 MMA per 16 keys
-                    const uint32_t v_addr = ring_addr + s0 * kEntryBytes;
+                    const uint32_t vb = v_lo + (uint32_t)s0 * kStep;
+                    umma_ts_lo(o, a, vb, idesc_pv128, acc0);
 #pragma unroll
-                    for (int kk = 0; kk < kBlockN / 16; ++kk)
-                        umma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
-                                sdesc_sw128(v_addr + kk * 2048, kEntryBytes, 1024), idesc_pv128,
-                                (j > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 1; kk < kBlockN / 16; ++kk)
+                        umma_ts_lo(o, a + kk * 8, vb + kk * (2048 >> 4), idesc_pv128, 1u);
                 } else {
                     // the pair wraps around the ring: one N = 64 MMA per half
-                    for (int h = 0; h < 2; ++h) {
-                        const uint32_t v_addr = ring_addr + ((e0 + h) % kRing) * kEntryBytes;
+                    const uint32_t vb0 = v_lo + (uint32_t)s0 * kStep, vb1 = v_lo;
+                    umma_ts_lo(o, a, vb0, idesc_pv64, acc0);
 #pragma unroll
-                        for (int kk = 0; kk < kBlockN / 16; ++kk)
-                            umma_ts(tmem + col_o(t) + 64 * h, tmem + col_s(t) + kk * 8,
-                                    sdesc_sw128(v_addr + kk * 2048, kEntryBytes, 1024), idesc_pv64,
-                                    (j > 0 || kk > 0) ? 1u : 0u);
-                    }
+                    for (int kk = 1; kk < kBlockN / 16; ++kk)
+                        umma_ts_lo(o, a + kk * 8, vb0 + kk * (2048 >> 4), idesc_pv64, 1u);
+                    umma_ts_lo(o + 64, a, vb1, idesc_pv64, acc0);
+#pragma unroll
+                    for (int kk = 1; kk < kBlockN / 16; ++kk)
+                        umma_ts_lo(o + 64, a + kk * 8, vb1 + kk * (2048 >> 4), idesc_pv64, 1u);
                 }
-                if (t == 1) {  // last reader of both V entries
-                    umma_commit(&bars->ring_empty[e0 % kRing]);
-                    umma_commit(&bars->ring_empty[(e0 + 1) % kRing]);
-                }
-                umma_commit(&bars->pv_done[t]);
-                return true;
             };
-            ok = issue_qk(0, 0) && issue_qk(1, 0);
-            for (int j = 1; ok && j < n_tiles; ++j)
-                ok = issue_pv(0, j - 1) && issue_qk(0, j) && issue_pv(1, j - 1) && issue_qk(1, j);
-            if (ok)
-                ok = issue_pv(0, n_tiles - 1) && issue_pv(1, n_tiles - 1);
+            wait(&bars->q_ready[0], 0);
+            wait(&bars->q_ready[1], 0);
+            wait(&bars->k_full[0], 0);
+            tc_fence_after();
+            qk(0, 0);
+            umma_commit(&bars->s_full[0]);
+            qk(1, 0);
+            umma_commit(&bars->k_free[0]);
+            umma_commit(&bars->s_full[1]);
+            for (int j = 1; ok && j < n_tiles; ++j) {
+                const int i = j - 1;
+                // tile A: PV_A(j-1), QK_A(j)
+                wait(&bars->p_full[0], (uint32_t)i & 1u);
+                wait(&bars->v_full[i & 1], (uint32_t)(i >> 1) & 1u);
+                tc_fence_after();
+                pv(0, i);
+                wait(&bars->k_full[j & 1], (uint32_t)(j >> 1) & 1u);
+                qk(0, j);
+                umma_commit(&bars->s_full[0]);
+                // tile B: PV_B(j-1), QK_B(j); it is the last reader of both tiles
+                wait(&bars->p_full[1], (uint32_t)i & 1u);
+                tc_fence_after();
+                pv(1, i);
+                umma_commit(&bars->v_free[i & 1]);
+                qk(1, j);
+                umma_commit(&bars->k_free[j & 1]);
+                umma_commit(&bars->s_full[1]);
+            }
+            if (ok) {
+                const int i = n_tiles - 1;
+                wait(&bars->p_full[0], (uint32_t)i & 1u);
+                wait(&bars->v_full[i & 1], (uint32_t)(i >> 1) & 1u);
+                tc_fence_after();
+                pv(0, i);
+                umma_commit(&bars->pv_done[0]);
+                wait(&bars->p_full[1], (uint32_t)i & 1u);
+                tc_fence_after();
+                pv(1, i);
+                umma_commit(&bars->v_free[i & 1]);
+                umma_commit(&bars->pv_done[1]);
+            }
             if (!ok) {
                 umma_commit(&bars->drain);
                 mbar_drain(&bars->drain, 0);
@@ -356,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_ga_kernel(const __grid_co
         }
 
         // ----------------------------------------------------------- epilogue
-        if (ok && mbar_wait(&bars->pv_done[t], (uint32_t)(n_tiles - 1) & 1u, abort_flag, p.err)) {
+        if (ok && mbar_wait(&bars->pv_done[t], 0, abort_flag, p.err)) {
             tc_fence_after();
             float o_scale;
             if (p.sinks != nullptr) {
