@@ -75,6 +75,31 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// 32-byte global store (sm_100 256-bit access). A thread that writes a whole
+// output row with these keeps every store a full pair of 32-byte sectors;
+// 16-byte stores of rows 256 bytes apart (one row per lane) halve the memory
+// throughput of a kernel that also streams its inputs.
+__device__ __forceinline__ void st_global_v8(void *p, const uint32_t (&v)[8])
+{
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]), "r"(v[1]),
+                 "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+
+// 32 bytes of an output row: one 256-bit store when the row is 32-byte
+// aligned (v8), else two 16-byte stores (the library only requires 16-byte
+// aligned outputs).
+__device__ __forceinline__ void st_global_32B(void *p, const uint32_t (&v)[8], bool v8)
+{
+    if (v8) {
+        st_global_v8(p, v);
+    } else {
+        uint4 *q = reinterpret_cast<uint4 *>(p);
+        q[0] = make_uint4(v[0], v[1], v[2], v[3]);
+        q[1] = make_uint4(v[4], v[5], v[6], v[7]);
+    }
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -427,6 +452,13 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src,
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
                  "l"(gmem_src), "r"(src_bytes)
                  : "memory");
+}
+
+// Arrives on `bar` (without raising its pending count) once every cp.async
+// this thread issued so far has landed.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void cp_async_commit()

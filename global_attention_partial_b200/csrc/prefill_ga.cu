@@ -67,6 +67,7 @@ struct GaParams {
     CUtensorMap tm_k;  // [B, rows, Hkv, Dqk] box {64, 1, 128, 1}
     CUtensorMap tm_v;  // [B, S, Hkv, Dv]     box {64, 1, 128, 1}
     __nv_bfloat16 *out;
+    int out_v8;                // out is 32-byte aligned: 256-bit stores
     const float2 *rope_table;  // [S][half]
     const float *sinks;        // nullptr on global layers
     unsigned *err;
@@ -430,17 +431,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_ga_kernel(const __grid_co
             for (int c = 0; c < 4; ++c)
                 tmem_tie(o[c]);
             if (row_valid) {
-                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (((size_t)b * p.S + i) * p.Hq + h) * kDv);
+                uint8_t *dst = reinterpret_cast<uint8_t *>(p.out + (((size_t)b * p.S + i) * p.Hq + h) * kDv);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
 #pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(o[c][c8 * 8 + 0]) * o_scale, __uint_as_float(o[c][c8 * 8 + 1]) * o_scale);
-                        w.y = pack_bf16x2(__uint_as_float(o[c][c8 * 8 + 2]) * o_scale, __uint_as_float(o[c][c8 * 8 + 3]) * o_scale);
-                        w.z = pack_bf16x2(__uint_as_float(o[c][c8 * 8 + 4]) * o_scale, __uint_as_float(o[c][c8 * 8 + 5]) * o_scale);
-                        w.w = pack_bf16x2(__uint_as_float(o[c][c8 * 8 + 6]) * o_scale, __uint_as_float(o[c][c8 * 8 + 7]) * o_scale);
-                        dst[c * 4 + c8] = w;
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t w[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            w[e] = pack_bf16x2(__uint_as_float(o[c][hh * 16 + 2 * e]) * o_scale,
+                                               __uint_as_float(o[c][hh * 16 + 2 * e + 1]) * o_scale);
+                        st_global_32B(dst + (c * 2 + hh) * 32, w, p.out_v8 != 0);
                     }
                 }
             }
@@ -471,6 +472,7 @@ cudaError_t launch_prefill_ga(const LayerArgs &L, const PrefillArgs &a, cudaStre
         !make_bf16_map_4d(&p.tm_v, a.v, kDv, L.Hkv, a.S, a.S, a.B, 64, 1, kBlockN))
         return cudaErrorInvalidValue;
     p.out = reinterpret_cast<__nv_bfloat16 *>(a.out);
+    p.out_v8 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
     p.rope_table = a.rope_table;
     p.sinks = L.sinks;
     p.err = a.err;

@@ -26,9 +26,9 @@
 // control warpgroup to the workers):
 //   warps 0-3   worker for even tiles    warps 4-7   worker for odd tiles
 //   warp 8      TMA producer: Q tiles and K/V ring blocks
-//   warp 9      MMA issuer: QK^T and PV of the tiles in flight, in whichever
-//               order their inputs become ready
-//   warps 10-11 idle
+//   warp 9      MMA issuer of worker 0 (QK^T and PV of the even tiles)
+//   warp 10     MMA issuer of worker 1 (the odd tiles)
+//   warp 11     idle
 //
 // TMEM (512 columns), per worker t: S_t = [256t, 256t + 144) and
 // O_t = [256t + 72, 256t + 200). O overlaps the upper S columns, which are
@@ -73,6 +73,7 @@ struct SwaParams {
     CUtensorMap tm_k;  // [B, S, Hkv, Dqk]   box {64, 1, 16, 1}
     CUtensorMap tm_v;  // [B, S, Hkv, Dv]    box {64, 1, 16, 1}
     __nv_bfloat16 *out;
+    int out_v8;                // out is 32-byte aligned: 256-bit stores
     const float2 *rope_table;  // [S][half] (cos, sin) of each token's position
     const float *sinks;
     unsigned *err;
@@ -87,12 +88,16 @@ struct Bars {
     uint64_t q_full[2], q_ready[2], q_empty[2];
     uint64_t kv_full[kRing], kv_empty[kRing];
     uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
-    uint64_t drain;
+    uint64_t tab_full[2];  // the worker's 128 threads copied its RoPE table slice
+    uint64_t drain[2];
     uint32_t tmem_base;
     int abort;
 };
 
-constexpr int kSmemBytes = 1024 + 2 * kQBytes + kKBytes + kVBytes + (int)sizeof(Bars) + 64;
+// RoPE table slice of one tile per worker: 16 positions x 32 (cos, sin) pairs.
+constexpr int kTabBytes = 16 * 32 * 8;
+constexpr int kSmemBytes = 1024 + 2 * kQBytes + kKBytes + kVBytes + 2 * kTabBytes + (int)sizeof(Bars) + 64;
+static_assert(kSmemBytes <= 232448, "shared memory");
 
 struct Tile {
     int b, kvh, h0, p0;
@@ -153,7 +158,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
     uint8_t *sQ = smem;                  // 2 buffers
     uint8_t *sK = sQ + 2 * kQBytes;      // 3 atoms of the ring
     uint8_t *sV = sK + kKBytes;          // 2 atoms of the ring
-    Bars *bars = reinterpret_cast<Bars *>(sV + kVBytes);
+    uint8_t *sTab = sV + kVBytes;        // 2 RoPE table slices
+    Bars *bars = reinterpret_cast<Bars *>(sTab + 2 * kTabBytes);
     volatile int *abort_flag = &bars->abort;
 
     const int warp = threadIdx.x >> 5;
@@ -171,12 +177,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
             mbar_init(&bars->p_full[i], 128);
             mbar_init(&bars->o_full[i], 1);
             mbar_init(&bars->o_free[i], 128);
+            mbar_init(&bars->tab_full[i], 128);
         }
         for (int i = 0; i < kRing; ++i) {
             mbar_init(&bars->kv_full[i], 1);
-            mbar_init(&bars->kv_empty[i], 1);
+            mbar_init(&bars->kv_empty[i], 2);  // one commit from each issuer
         }
-        mbar_init(&bars->drain, 1);
+        mbar_init(&bars->drain[0], 1);
+        mbar_init(&bars->drain[1], 1);
         bars->abort = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -251,153 +259,98 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                     mbar_drain(&bars->kv_full[e % kRing], (uint32_t)(e / kRing) & 1u);
             }
         }
-    } else if (warp == 9) {
-        // ------------------------------------------------------- MMA issuer
-        if (lane == 0 && n_local > 0) {
+    } else if (warp == 9 || warp == 10) {
+        // ------------------------------------------------------ MMA issuers
+        // Issuer t (warp 9 + t) serves worker t: the tiles n with n % 2 == t,
+        // in order, each with blocking waits, so it reacts as soon as an input
+        // is ready. Both walk every tile with the producer's ring cursor to
+        // number the entries. An entry is free (its kv_empty barrier counts
+        // two arrivals) once each issuer has committed it: issuer t commits the
+        // entries below the span of its next tile after the PV of its current
+        // one, and every remaining entry after its last tile.
+        const int t = warp - 9;
+        if (lane == 0 && t < n_local) {
             const uint32_t idesc_pv = idesc_bf16_f32(kBlockM, kDv, false, true);
-            const uint32_t q_base = smem_u32(sQ);
-            const uint32_t k_base = smem_u32(sK);
-            const uint32_t v_base = smem_u32(sV);
-            // Ring ranges of the tiles in flight (registers only, by parity).
-            int first0 = 0, nb0 = 0, first1 = 0, nb1 = 0;
-            // Tile walk without divisions: run and first block of tile next_qk.
-            const Tile t0 = tile_at(p, t_begin);
-            int qk_pt = t0.p0 / p.P;  // position tile of next_qk within its run
-            int qk_run = t0.run;
-            int qk_base = -t0.first_block;  // entry of block 0 of qk_run
-            int qk_last_block = -1;
-            int pushed = 0;                 // entries the producer pushes for tiles < next_qk
-            int known_full = 0;             // entries [0, known_full) have landed
-            int freed = 0;
-            int next_qk = 0, next_pv = 0;
-            long long t_last = cycles_now();
-            uint32_t idle = 0;
+            const uint32_t q_lo = sdesc_lo(smem_u32(sQ + t * kQBytes), 16);
+            const uint32_t k_lo = sdesc_lo(smem_u32(sK), 16);
+            const uint32_t v_lo = sdesc_lo(smem_u32(sV), kVAtom);
+            constexpr uint32_t kQAtomStep = (kBlockM * 128) >> 4;
+            constexpr uint32_t kKAtomStep = kKAtom >> 4;
+            constexpr uint32_t kSlotStep = (kKeyBlock * 128) >> 4;
+            const uint32_t s_col = tmem + col_s(t), o_col = tmem + col_o(t);
             bool ok = true;
-            while (ok && next_pv < n_local) {
-                bool progressed = false;
-                // QK_n needs its worker's S/O columns back (epilogue of tile n-2
-                // done, which also implies PV_{n-2} landed), its rotated Q and its keys.
-                if (next_qk < n_local && mbar_test_wait(&bars->o_free[next_qk & 1], ((uint32_t)(next_qk >> 1) & 1u) ^ 1u)) {
-                    const int n = next_qk;
-                    const int qb = n & 1;
-                    // Span of tile n in ring entries.
-                    const int p0 = qk_pt * p.P;
-                    const int k_lo = p0 - p.window + 1;
-                    const int fb = k_lo > 0 ? k_lo / kKeyBlock : 0;
-                    const int lb = (p0 + p.P - 1) / kKeyBlock;
-                    int base = qk_base;
-                    int push = pushed;
-                    if (qk_last_block < 0) {  // first tile of a run in this CTA
-                        base = pushed - fb;
-                        push += lb - fb + 1;
-                    } else {
-                        push += lb - qk_last_block;
-                    }
-                    const int e0 = base + fb;
-                    const int nb = lb - fb + 1;
-                    while (known_full < push &&
-                           mbar_test_wait(&bars->kv_full[known_full % kRing], (uint32_t)(known_full / kRing) & 1u))
-                        ++known_full;
-                    if (known_full >= e0 + nb && mbar_test_wait(&bars->q_ready[qb], (uint32_t)(n >> 1) & 1u)) {
-                        tc_fence_after();
-                        const uint32_t q_addr = q_base + qb * kQBytes;
-                        const int s0 = e0 % kRing;
-                        const int run1 = min(nb, kRing - s0);
-                        for (int part = 0; part < 2; ++part) {
-                            const int blocks = part == 0 ? run1 : nb - run1;
-                            if (blocks <= 0)
-                                continue;
-                            const int slot = part == 0 ? s0 : 0;
-                            const uint32_t d = tmem + col_s(qb) + (part == 0 ? 0u : (uint32_t)(run1 * kKeyBlock));
-                            const uint32_t idesc = idesc_bf16_f32(kBlockM, blocks * kKeyBlock, false, false);
+            auto wait = [&](uint64_t *bar, uint32_t parity) {
+                if (!mbar_try_wait(bar, parity) && !mbar_wait(bar, parity, abort_flag, p.err))
+                    ok = false;
+            };
+            RingCursor cur;
+            int walked = -1;  // tiles [0, walked] have been walked
+            int e0 = 0, nb = 0;
+            auto walk_to = [&](int n) {
+                while (walked < n) {
+                    ++walked;
+                    const Tile c = tile_at(p, t_begin + walked);
+                    cur.advance(c);
+                    e0 = cur.entry(c.first_block);
+                    nb = c.last_block - c.first_block + 1;
+                }
+            };
+            // S_t = Q_t K^T over the entries [e0, e0 + nb): one group of 12
+            // MMAs (N = 16 keys per entry), two when the span wraps the ring.
+            auto qk_part = [&](uint32_t d, int slot, int blocks) {
+                const uint32_t idesc = idesc_bf16_f32(kBlockM, blocks * kKeyBlock, false, false);
+                const uint32_t kb = k_lo + (uint32_t)slot * kSlotStep;
 #pragma unroll
-                            for (int kk = 0; kk < kDqk / 16; ++kk) {
-                                const int atom = kk >> 2;
-                                const uint32_t off = (uint32_t)(kk & 3) * 32u;
-                                umma_ss(d, sdesc_sw128(q_addr + atom * (kBlockM * 128) + off, 16, 1024),
-                                        sdesc_sw128(k_base + atom * kKAtom + slot * (kKeyBlock * 128) + off, 16, 1024),
-                                        idesc, kk > 0 ? 1u : 0u);
-                            }
-                        }
-                        umma_commit(&bars->s_full[qb]);
-                        umma_commit(&bars->q_empty[qb]);
-                        if (qb) {
-                            first1 = e0;
-                            nb1 = nb;
-                        } else {
-                            first0 = e0;
-                            nb0 = nb;
-                        }
-                        // advance the walk to the next tile
-                        pushed = push;
-                        qk_base = base;
-                        qk_last_block = lb;
-                        if (++qk_pt == p.num_p_tiles) {
-                            qk_pt = 0;
-                            ++qk_run;
-                            qk_last_block = -1;
-                        }
-                        ++next_qk;
-                        progressed = true;
-                    }
+                for (int atom = 0; atom < 3; ++atom)
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4)
+                        umma_ss_lo(d, q_lo + atom * kQAtomStep + 2 * k4, kb + atom * kKAtomStep + 2 * k4, idesc,
+                                   (atom | k4) ? 1u : 0u);
+            };
+            int known_full = 0;  // entries [0, known_full) have landed
+            int freed = 0;       // entries [0, freed) committed by this issuer
+            walk_to(t);
+            for (int n = t; ok && n < n_local; n += 2) {
+                const uint32_t ph = (uint32_t)(n >> 1) & 1u;
+                wait(&bars->o_free[t], ph ^ 1u);  // epilogue of tile n - 2 has read O
+                wait(&bars->q_ready[t], ph);
+                // Only this tile's entries: those below e0 may already be
+                // released (and refilled) on behalf of the other worker.
+                for (known_full = max(known_full, e0); known_full < e0 + nb; ++known_full)
+                    wait(&bars->kv_full[known_full % kRing], (uint32_t)(known_full / kRing) & 1u);
+                tc_fence_after();
+                const int s0 = e0 % kRing;
+                const int run1 = min(nb, kRing - s0);
+                qk_part(s_col, s0, run1);
+                if (nb > run1)
+                    qk_part(s_col + (uint32_t)(run1 * kKeyBlock), 0, nb - run1);
+                umma_commit(&bars->s_full[t]);
+                umma_commit(&bars->q_empty[t]);
+                // O_t = P_t V over the same entries, one N = 128 MMA per entry.
+                wait(&bars->p_full[t], ph);
+                tc_fence_after();
+                int slot = s0;
+                for (int j = 0; j < nb; ++j) {
+                    umma_ts_lo(o_col, s_col + (uint32_t)(j * 8), v_lo + (uint32_t)slot * kSlotStep, idesc_pv,
+                               j > 0 ? 1u : 0u);
+                    slot = slot + 1 == kRing ? 0 : slot + 1;
                 }
-                if (next_pv < next_qk) {
-                    const int n = next_pv;
-                    const int sb = n & 1;
-                    if (mbar_test_wait(&bars->p_full[sb], (uint32_t)(n >> 1) & 1u)) {
-                        tc_fence_after();
-                        const int e0 = sb ? first1 : first0;
-                        const int nb = sb ? nb1 : nb0;
-                        for (int j = 0; j < nb; ++j) {
-                            const int slot = (e0 + j) % kRing;
-                            umma_ts(tmem + col_o(sb), tmem + col_s(sb) + j * 8,
-                                    sdesc_sw128(v_base + slot * (kKeyBlock * 128), kVAtom, 1024), idesc_pv,
-                                    j > 0 ? 1u : 0u);
-                        }
-                        umma_commit(&bars->o_full[sb]);
-                        // Release the ring entries no later tile uses: all of them
-                        // unless tile n+1 (already walked by the QK side when it is
-                        // in flight, else computed here) continues the same run.
-                        int keep_from = e0 + nb;
-                        if (n + 1 < n_local) {
-                            int nfirst;
-                            if (n + 1 < next_qk) {
-                                nfirst = sb ? first0 : first1;
-                            } else {
-                                // tile n+1 not walked yet: same run iff its walk state continues
-                                const int p0 = qk_pt * p.P;
-                                const int k_lo = p0 - p.window + 1;
-                                const int fb = k_lo > 0 ? k_lo / kKeyBlock : 0;
-                                nfirst = qk_last_block < 0 ? e0 + nb : qk_base + fb;
-                            }
-                            keep_from = min(keep_from, nfirst);
-                        }
-                        for (; freed < keep_from; ++freed)
-                            umma_commit(&bars->kv_empty[freed % kRing]);
-                        ++next_pv;
-                        progressed = true;
-                    }
-                }
-                if (progressed) {
-                    idle = 0;
+                umma_commit(&bars->o_full[t]);
+                // Release what no later tile of this worker reads.
+                int keep_from;
+                if (n + 2 < n_local) {
+                    walk_to(n + 2);
+                    keep_from = e0;
                 } else {
-                    // Nothing ready: yield the issue slots to the softmax warp
-                    // sharing this SM sub-partition, and bound the wait.
-                    __nanosleep(32);
-                    if (idle++ == 0)
-                        t_last = cycles_now();
-                    if (*abort_flag) {
-                        ok = false;
-                    } else if ((idle & 63u) == 0 && cycles_now() - t_last > kWaitLimitCycles) {
-                        *abort_flag = 1;
-                        atomicOr(p.err, kErrTimeout);
-                        ok = false;
-                    }
+                    walk_to(n_local - 1);
+                    keep_from = cur.next_entry;
                 }
+                for (; freed < keep_from; ++freed)
+                    umma_commit(&bars->kv_empty[freed % kRing]);
             }
             if (!ok) {
-                umma_commit(&bars->drain);
-                mbar_drain(&bars->drain, 0);
+                umma_commit(&bars->drain[t]);
+                mbar_drain(&bars->drain[t], 0);
             }
         }
     } else if (warp < 8) {
@@ -417,24 +370,30 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
             const int i = c.p0 + row / p.gp;
             const int h = c.h0 + row % p.gp;
             // ---- partial RoPE of this row of Q_n (buffer t)
-            // cos/sin of the row's 32 pairs are fetched before waiting for Q,
-            // so their latency overlaps the Q load.
-            const bool fast_rope = half == 32 && i < p.S;
-            float4 tb[16];
+            // With 16 positions per tile and 32 pairs (the MiMo layer), the
+            // tile's 4 KB slice of the RoPE table is copied into shared memory
+            // before waiting for Q, so its latency overlaps the Q load without
+            // holding registers across the wait.
+            const bool fast_rope = half == 32 && p.P == 16;
+            const float4 *tab_row = reinterpret_cast<const float4 *>(sTab + t * kTabBytes) + (row >> 3) * 16;
             if (fast_rope) {
-                const float4 *cs4 = reinterpret_cast<const float4 *>(p.rope_table + (size_t)i * half);
-#pragma unroll
-                for (int w = 0; w < 16; ++w)
-                    tb[w] = __ldg(cs4 + w);
+                const int pos = c.p0 + (row >> 3);
+                const bool in = pos < p.S;
+                const float2 *src = p.rope_table + (size_t)(in ? pos : 0) * 32 + (row & 7) * 4;
+                uint8_t *dst = sTab + t * kTabBytes + (row >> 3) * 256 + (row & 7) * 32;
+                cp_async16(dst, src, in ? 16u : 0u);
+                cp_async16(dst + 16, src + 2, in ? 16u : 0u);
+                cp_async_mbar_arrive(&bars->tab_full[t]);  // arrives once this thread's copies landed
             }
-            if (!mbar_wait(&bars->q_full[t], ph, abort_flag, p.err)) {
+            if (!mbar_wait(&bars->q_full[t], ph, abort_flag, p.err) ||
+                (fast_rope && !mbar_wait(&bars->tab_full[t], ph, abort_flag, p.err))) {
                 ok = false;
                 break;
             }
             if (i < p.S && half > 0) {
                 uint8_t *q_row = sQ + t * kQBytes + row * 128;
                 const float2 *cs = p.rope_table + (size_t)i * half;
-                if (fast_rope) {
+                if (fast_rope && i < p.S) {
                     // One 128-byte swizzled row: chunks 0-3 hold dims 0-31, 4-7 dims 32-63.
                     uint4 v[8];
 #pragma unroll
@@ -448,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                         for (int w = 0; w < 4; ++w) {
                             const float2 xa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&a[w]));
                             const float2 xb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&bb[w]));
-                            const float4 cc = tb[ch * 4 + w];  // (cos, sin) of pairs 8ch+2w, 8ch+2w+1
+                            const float4 cc = tab_row[ch * 4 + w];  // (cos, sin) of pairs 8ch+2w, 8ch+2w+1
                             a[w] = pack_bf16x2(xa.x * cc.x - xb.x * cc.y, xa.y * cc.z - xb.y * cc.w);
                             bb[w] = pack_bf16x2(xb.x * cc.x + xa.x * cc.y, xb.y * cc.z + xa.y * cc.w);
                         }
@@ -553,21 +512,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
             tc_fence_before();
             mbar_arrive(&bars->o_free[t]);
             if (i < p.S) {
-                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (((size_t)c.b * p.S + i) * p.Hq + h) * kDv);
+                uint8_t *dst = reinterpret_cast<uint8_t *>(p.out + (((size_t)c.b * p.S + i) * p.Hq + h) * kDv);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
 #pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(o[q][c8 * 8 + 0]) * o_scale, __uint_as_float(o[q][c8 * 8 + 1]) * o_scale);
-                        w.y = pack_bf16x2(__uint_as_float(o[q][c8 * 8 + 2]) * o_scale, __uint_as_float(o[q][c8 * 8 + 3]) * o_scale);
-                        w.z = pack_bf16x2(__uint_as_float(o[q][c8 * 8 + 4]) * o_scale, __uint_as_float(o[q][c8 * 8 + 5]) * o_scale);
-                        w.w = pack_bf16x2(__uint_as_float(o[q][c8 * 8 + 6]) * o_scale, __uint_as_float(o[q][c8 * 8 + 7]) * o_scale);
-                        dst[q * 4 + c8] = w;
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t w[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            w[e] = pack_bf16x2(__uint_as_float(o[q][hh * 16 + 2 * e]) * o_scale,
+                                               __uint_as_float(o[q][hh * 16 + 2 * e + 1]) * o_scale);
+                        st_global_32B(dst + (q * 2 + hh) * 32, w, p.out_v8 != 0);
                     }
                 }
             }
         }
+        cp_async_wait<0>();  // no table copy may land after an abort ended the loop
     }
 
     tc_fence_before();
@@ -617,6 +577,7 @@ cudaError_t launch_prefill_swa(const LayerArgs &L, const PrefillArgs &a, const f
         !make_bf16_map_4d(&p.tm_v, a.v, kDv, L.Hkv, a.S, a.S, a.B, 64, 1, kKeyBlock))
         return cudaErrorInvalidValue;
     p.out = reinterpret_cast<__nv_bfloat16 *>(a.out);
+    p.out_v8 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
     p.rope_table = rope_table;
     p.sinks = L.sinks;
     p.err = a.err;

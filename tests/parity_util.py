@@ -72,13 +72,20 @@ def oracle_prefill(spec, q, k, v, sinks, rows_by_b_h, positions=None, window=Non
 
 
 def check_prefill(spec, B, S, dtype, *, seed=0, layer_idx=0, rows="all", heads=None, batches=None,
-                  positions=None, window=None, rotary=None, n_random_rows=24):
-    """Runs the library prefill and compares it with the oracle. Returns Cmp."""
+                  positions=None, window=None, rotary=None, n_random_rows=24, out_offset_elems=0):
+    """Runs the library prefill and compares it with the oracle. Returns Cmp.
+    out_offset_elems > 0 places the output that many elements past a 256-byte
+    aligned allocation (8 bf16 = 16 bytes: 16- but not 32-byte aligned)."""
     q, k, v, sinks = synthetic.prefill_inputs(spec, B, S, seed=seed, layer=layer_idx, dtype=dtype, device="cuda")
     if spec.layer_type == 0:
         sinks = None
     lay = lib_layer(spec, sinks, window, rotary)
-    out = mimo.prefill(lay, q, k, v, positions=positions)
+    out = None
+    if out_offset_elems:
+        n = B * S * spec.num_q_heads * spec.v_dim
+        base = torch.empty(n + out_offset_elems, dtype=dtype, device="cuda")
+        out = base[out_offset_elems:].view(B, S, spec.num_q_heads, spec.v_dim)
+    out = mimo.prefill(lay, q, k, v, positions=positions, out=out)
     torch.cuda.synchronize()
     heads = range(spec.num_q_heads) if heads is None else heads
     batches = range(B) if batches is None else batches

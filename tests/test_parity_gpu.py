@@ -52,6 +52,16 @@ def test_tc_prefill_small_and_ragged_full(layer_type, S):
     _assert(c, BF, f"type {layer_type} S {S}")
 
 
+@pytest.mark.parametrize("layer_type", [0, 1])
+def test_tc_prefill_output_16_byte_aligned(layer_type):
+    """An output that is 16- but not 32-byte aligned takes the 16-byte store
+    path of the epilogue (32-byte aligned outputs use 256-bit stores)."""
+    spec = synthetic.mimo_layer(layer_type)
+    c, out, _ = check_prefill(spec, 2, 300, BF, seed=3, out_offset_elems=8)
+    assert out.data_ptr() % 32 == 16
+    _assert(c, BF, f"type {layer_type} 16-byte aligned output")
+
+
 @pytest.mark.parametrize("window", [1, 2, 17, 129, 500])
 def test_tc_prefill_windows(window):
     spec = synthetic.mimo_layer(1)
