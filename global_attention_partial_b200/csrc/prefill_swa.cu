@@ -25,10 +25,11 @@
 // Warp roles (384 threads = 3 warpgroups; setmaxnreg moves registers from the
 // control warpgroup to the workers):
 //   warps 0-3   worker for even tiles    warps 4-7   worker for odd tiles
-//   warp 8      TMA producer: Q tiles and K/V ring blocks
+//   warp 8      TMA producer of the Q tiles
 //   warp 9      MMA issuer of worker 0 (QK^T and PV of the even tiles)
 //   warp 10     MMA issuer of worker 1 (the odd tiles)
-//   warp 11     idle
+//   warp 11     TMA producer of the K/V ring blocks
+
 //
 // TMEM (512 columns), per worker t: S_t = [256t, 256t + 144) and
 // O_t = [256t + 72, 256t + 200). O overlaps the upper S columns, which are
@@ -202,35 +203,48 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
         setmaxnreg_dec<kRegsControl>();
     }
     if (warp == 8) {
-        // ------------------------------------------------------ TMA producer
+        // ------------------------------------------------- TMA producer: Q
+        // Q tiles through their two buffers, each refilled once the QK^T of
+        // the tile two before has read it.
         if (lane == 0 && n_local > 0) {
             tma_prefetch_desc(&p.tm_q);
-            tma_prefetch_desc(&p.tm_k);
-            tma_prefetch_desc(&p.tm_v);
             int last_q[2] = {-1, -1};
-            int loaded = 0;  // ring entries issued
-            RingCursor cur;
-            bool ok = true;
-            auto load_q = [&](int n) -> bool {
+            for (int n = 0; n < n_local; ++n) {
                 const int qb = n & 1;
                 if (!mbar_wait(&bars->q_empty[qb], ((uint32_t)(n >> 1) & 1u) ^ 1u, abort_flag, p.err))
-                    return false;
+                    break;
                 const Tile c = tile_at(p, t_begin + n);
                 mbar_arrive_expect_tx(&bars->q_full[qb], kQBytes);
                 for (int a = 0; a < 3; ++a)
                     tma_load_4d(sQ + qb * kQBytes + a * (kBlockM * 128), &p.tm_q, &bars->q_full[qb], a * 64,
                                 c.h0, c.p0, c.b);
                 last_q[qb] = n;
-                return true;
-            };
-            auto load_blocks = [&](int n) -> bool {
+            }
+            if (*abort_flag)
+                for (int qb = 0; qb < 2; ++qb)
+                    if (last_q[qb] >= 0)
+                        mbar_drain(&bars->q_full[qb], (uint32_t)(last_q[qb] >> 1) & 1u);
+        }
+    } else if (warp == 11) {
+        // ---------------------------------------------- TMA producer: K/V ring
+        // Independent of the Q stream, so key blocks run ahead of the tiles
+        // as far as the ring's free entries allow.
+        if (lane == 0 && n_local > 0) {
+            tma_prefetch_desc(&p.tm_k);
+            tma_prefetch_desc(&p.tm_v);
+            int loaded = 0;  // ring entries issued
+            RingCursor cur;
+            bool ok = true;
+            for (int n = 0; ok && n < n_local; ++n) {
                 const Tile c = tile_at(p, t_begin + n);
                 const int first_new = cur.advance(c);
                 for (int blk = first_new; blk <= c.last_block; ++blk) {
                     const int e = loaded;
                     const int slot = e % kRing;
-                    if (!mbar_wait(&bars->kv_empty[slot], ((uint32_t)(e / kRing) & 1u) ^ 1u, abort_flag, p.err))
-                        return false;
+                    if (!mbar_wait(&bars->kv_empty[slot], ((uint32_t)(e / kRing) & 1u) ^ 1u, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
                     mbar_arrive_expect_tx(&bars->kv_full[slot], kEntryBytes);
                     const int key0 = blk * kKeyBlock;
                     for (int a = 0; a < 3; ++a)
@@ -241,23 +255,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                                     a * 64, c.kvh, key0, c.b);
                     ++loaded;
                 }
-                return true;
-            };
-            ok = load_q(0) && load_blocks(0);
-            if (ok && n_local > 1)
-                ok = load_q(1);
-            for (int n = 1; ok && n < n_local; ++n) {
-                ok = load_blocks(n);
-                if (ok && n + 1 < n_local)
-                    ok = load_q(n + 1);
             }
-            if (*abort_flag) {
-                for (int qb = 0; qb < 2; ++qb)
-                    if (last_q[qb] >= 0)
-                        mbar_drain(&bars->q_full[qb], (uint32_t)(last_q[qb] >> 1) & 1u);
+            if (*abort_flag)
                 for (int e = max(0, loaded - kRing); e < loaded; ++e)
                     mbar_drain(&bars->kv_full[e % kRing], (uint32_t)(e / kRing) & 1u);
-            }
         }
     } else if (warp == 9 || warp == 10) {
         // ------------------------------------------------------ MMA issuers
