@@ -220,7 +220,7 @@ class StackWorkload:
         return sum(decode_bytes(L["spec"], self.lens) for L in self.decode_layers)
 
     def launches_per_step(self):
-        n = 2 * len(self.prefill_layers)  # K-prep + attention
+        n = 3 * len(self.prefill_layers)  # RoPE table + K-prep + attention
         for L in self.decode_layers:
             n += 2 if L["need"] > 0 else 1  # split kernel (+ combine)
         return n
@@ -238,6 +238,34 @@ class StackWorkload:
                                 L["vc"], L["cap"], L["out"], L["ws"], L["ws"].numel(), stream)
         if st != m.OK:
             raise m.MimoAttnError(st, "mimo_attn_decode")
+
+    def capture_decode(self):
+        """Captures the decode stack (every layer's kernels) in one CUDA graph,
+        as a serving loop replays it each step; the first, uncaptured pass sets
+        the kernels' launch attributes."""
+        if not self.decode_layers:
+            return
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for L in self.decode_layers:
+                self.run_decode_layer(L, side)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            cs = torch.cuda.current_stream()
+            for L in self.decode_layers:
+                self.run_decode_layer(L, cs)
+        torch.cuda.synchronize()
+        self.decode_graph = g
+
+    def run_decode_stack(self, stream):
+        if getattr(self, "decode_graph", None) is not None:
+            self.decode_graph.replay()
+        else:
+            for L in self.decode_layers:
+                self.run_decode_layer(L, stream)
 
     def step(self, stream, events=None):
         """One pass of the hot path. events: optional dict of lists collecting
@@ -257,8 +285,7 @@ class StackWorkload:
             if events is not None:
                 e0 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-            for L in self.decode_layers:
-                self.run_decode_layer(L, stream)
+            self.run_decode_stack(stream)
             if events is not None:
                 e1 = torch.cuda.Event(enable_timing=True)
                 e1.record(stream)
@@ -453,6 +480,9 @@ def workload_config(args, reference=False):
            "kv_len_range": list(synthetic.HYBRID_DECODE.kv_len_range), "layers": "0,1,1,1,1,1,0,1",
            "parallelism": f"replicas x{args.gpus} (weak, no collective on the data path)",
            "l2": "no flush: each step streams ~60 GB of inputs, far above the 126 MB L2"}
+    if args.workload in ("stack", "decode"):
+        cfg["decode_launch"] = ("direct C-ABI calls, one per layer" if args.no_graph else
+                                "the 8 layers' C-ABI calls captured once in a CUDA graph, replayed each step")
     if args.workload != "stack":
         cfg["l2"] = "inputs larger than L2" if args.workload != "swa" else "L2 flushed between steps (256 MB write)"
     return cfg
@@ -467,6 +497,7 @@ def main():
     ap.add_argument("--workload", choices=["stack", "swa", "global", "decode"], default="stack")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch the decode layers one call at a time")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     if args.impl == "reference":
@@ -479,6 +510,8 @@ def main():
     mimo.load()
     peaks = measured_peaks()
     w = StackWorkload(args.workload)
+    if not args.no_graph:
+        w.capture_decode()
     stream = torch.cuda.current_stream()
     flush = None
     if args.workload == "swa":

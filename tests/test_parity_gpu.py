@@ -234,6 +234,45 @@ def test_decode_fp32_cuda_core_path(layer_type):
     _check_decode(spec, out, inputs, caches, range(len(lens)), lens, dtype=torch.float32)
 
 
+@pytest.mark.parametrize("layer_type", [0, 1])
+def test_decode_cuda_graph_replay(layer_type):
+    """After its first call the decode entry point makes no synchronising or
+    allocating CUDA call, so a serving loop can capture it in a CUDA graph: a
+    replay writes the same output as a direct call, and that output passes
+    parity."""
+    spec = synthetic.mimo_layer(layer_type)
+    lens = [1, 65, 129, 2049, 5000]
+    B, cap = len(lens), 5000
+    kv_lens = torch.tensor(lens, dtype=torch.int32)
+    q, kn, vn, kc, vc, sinks = synthetic.decode_inputs(spec, B, cap, kv_lens, seed=7, layer=0, dtype=BF,
+                                                       device="cuda")
+    sinks = sinks if layer_type == 1 else None
+    kc0, vc0 = kc.clone(), vc.clone()
+    lay = lib_layer(spec, sinks)
+    lens_dev = kv_lens.cuda()
+    out = torch.empty((B, spec.num_q_heads, spec.v_dim), dtype=BF, device="cuda")
+    need = mimo.mimo_attn_decode_workspace_size(lay, mimo.BF16, B, kc.shape[1])
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device="cuda")
+
+    slots = kc.shape[1]  # the ring of a sliding layer has `window` slots
+
+    def call(stream):
+        st = mimo.mimo_attn_decode(lay, mimo.BF16, B, q, kn, vn, lens_dev, kc, vc, slots, out, ws, ws.numel(), stream)
+        assert st == mimo.OK
+
+    call(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    direct = out.clone()
+    out.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call(torch.cuda.current_stream())
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, direct)
+    _check_decode(spec, out, (q, kn, vn, kc0, vc0, sinks), (kc, vc), range(B), lens)
+
+
 def test_decode_full_size_sampled_batches():
     """Hybrid decode workload (B64, L ~ U[1024, 32768], cache 32768): one
     global and one SWA layer; every head of 6 sampled sequences."""
