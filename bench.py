@@ -591,7 +591,21 @@ def main():
         byt = w.decode_bytes()
         parts["decode"] = {"ms_per_stack": per, "gbs": byt / (per * 1e-3) / 1e9,
                            "frac_of_hbm_peak": byt / (per * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                           "bytes_per_stack": byt}
+                           "bytes_per_stack": byt,
+                           "launch": "direct calls" if getattr(w, "decode_graph", None) is None else "CUDA graph"}
+        if getattr(w, "decode_graph", None) is not None:
+            # the same stack as 8 back-to-back direct calls, outside the timed region
+            d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 5
+            d0.record(stream)
+            for _ in range(reps):
+                for L in w.decode_layers:
+                    w.run_decode_layer(L, stream)
+            d1.record(stream)
+            torch.cuda.synchronize()
+            per_d = d0.elapsed_time(d1) / reps
+            parts["decode"]["ms_per_stack_direct_calls"] = per_d
+            parts["decode"]["gbs_direct_calls"] = byt / (per_d * 1e-3) / 1e9
         if roofline is None:
             ach = byt / (per * 1e-3) / 1e9
             roofline = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",

@@ -42,8 +42,11 @@ constexpr int kDecodeStages = 2;
 struct DecodeSmem {
     float wm[4][16];
     float wl[4][16];
-    float o[16][kDv];
 };
+// Row stride (floats) of the per-warp O slices of the final merge, which
+// reuse the stage buffers: 4 x 16 rows x 136 floats = 34 KB.
+constexpr int kMergeStride = kDv + 8;
+static_assert(4 * 16 * kMergeStride * 4 <= kStageElems * 2 * 2, "merge slices fit in the stage buffers");
 
 __device__ __forceinline__ int visible_count(int layer_type, int Lb, int window)
 {
@@ -72,6 +75,45 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
     const int split = blockIdx.x;
     const int kvh = blockIdx.y;
     const int b = blockIdx.z;
+    const int G = L.G;
+    const int half = L.rope.half;
+
+    // The query rows of this KV group and the new token's k/v do not depend
+    // on kv_lens: their loads go out first, beside the kv_lens load, instead
+    // of one dependent round trip after another.
+    const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(a.q) +
+                              ((size_t)b * L.Hq + (size_t)kvh * G) * kDqk;
+    const bool vec_rope = L.rope.rotary_dim % 16 == 0;
+    // Rotary unit: a 16-byte chunk pair (c, c + r/16); copy unit: one
+    // pass-through chunk.
+    const int npair = half / 8;
+    const int per_row = npair + (kDqk - L.rope.rotary_dim) / 8;
+    uint4 va[3], vb[3];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        const int u = tid + k * kThreads;
+        const int r = u / per_row;
+        const int w = u - r * per_row;
+        va[k] = make_uint4(0, 0, 0, 0);
+        vb[k] = make_uint4(0, 0, 0, 0);
+        if (vec_rope && r < G && r < 16) {
+            const uint4 *qr = reinterpret_cast<const uint4 *>(qg + (size_t)r * kDqk);
+            if (w < npair) {
+                va[k] = __ldg(qr + w);
+                vb[k] = __ldg(qr + w + npair);
+            } else {
+                va[k] = __ldg(qr + npair + w);
+            }
+        }
+    }
+    const __nv_bfloat16 *kn = reinterpret_cast<const __nv_bfloat16 *>(a.k_new) + ((size_t)b * L.Hkv + kvh) * kDqk;
+    const __nv_bfloat16 *vn = reinterpret_cast<const __nv_bfloat16 *>(a.v_new) + ((size_t)b * L.Hkv + kvh) * kDv;
+    uint4 nv = make_uint4(0, 0, 0, 0);  // chunk tid of k_new (tid < 24) or v_new (24 <= tid < 40)
+    if (tid < 24)
+        nv = __ldg(reinterpret_cast<const uint4 *>(kn) + tid);
+    else if (tid < 40)
+        nv = __ldg(reinterpret_cast<const uint4 *>(vn) + (tid - 24));
+
     const int Lb = __ldg(a.kv_lens + b);
     if (!kv_len_ok(L.layer_type, Lb, a.cap)) {
         if (split == 0 && kvh == 0 && tid == 0)
@@ -87,8 +129,6 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
     const int slot_new = L.layer_type == 1 ? (Lb - 1) % L.window : Lb - 1;
     const bool owns_new = slot_new >= key_begin && slot_new < key_end;
     const double pos = (double)(Lb - 1);
-    const int G = L.G;
-    const int half = L.rope.half;
 
     const size_t kv_row = (size_t)L.Hkv;  // rows of the cache are [slot][Hkv][D]
     const __nv_bfloat16 *kc = reinterpret_cast<const __nv_bfloat16 *>(a.k_cache) +
@@ -96,8 +136,7 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
     const __nv_bfloat16 *vc = reinterpret_cast<const __nv_bfloat16 *>(a.v_cache) +
                               ((size_t)b * a.cap * kv_row + kvh) * kDv;
 
-    // The first K/V tiles go out before anything else, so their latency
-    // overlaps the query preparation below.
+    // The first K/V tiles go out before the query preparation below.
     const int n_tiles = (key_end - key_begin + kTileKeys - 1) / kTileKeys;
     auto issue = [&](int t) {
         __nv_bfloat16 *st = sStage + (t % kStages) * kStageElems;
@@ -125,41 +164,22 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
         cp_async_commit();
     }
 
-    // cos/sin of the new token's position for every rotary pair, once per CTA
+    // cos/sin of the new token's position for every rotary pair, once per CTA;
+    // the raw new k/v chunks go to shared memory.
     __shared__ float2 s_cs[kMaxHalfRotary];
     for (int j = tid; j < half; j += kThreads) {
         float c, s;
         rope_cos_sin(pos, L.rope.inv_freq[j], c, s);
         s_cs[j] = make_float2(c, s);
     }
+    if (tid < 24)
+        reinterpret_cast<uint4 *>(sKnew)[tid] = nv;
+    else if (tid < 40)
+        reinterpret_cast<uint4 *>(sVnew)[tid - 24] = nv;
     __syncthreads();
 
-    const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(a.q) +
-                              ((size_t)b * L.Hq + (size_t)kvh * G) * kDqk;
-    if (L.rope.rotary_dim % 16 == 0) {
-        // Query heads of this KV group, rotated at position L-1 (rows >= G are
-        // 0), in 16-byte units: a rotary unit is a chunk pair (c, c + r/16), a
-        // copy unit one pass-through chunk. All loads are issued before use.
-        const int npair = half / 8;
-        const int per_row = npair + (kDqk - L.rope.rotary_dim) / 8;
-        uint4 va[3], vb[3];
-#pragma unroll
-        for (int k = 0; k < 3; ++k) {
-            const int u = tid + k * kThreads;
-            const int r = u / per_row;
-            const int w = u - r * per_row;
-            va[k] = make_uint4(0, 0, 0, 0);
-            vb[k] = make_uint4(0, 0, 0, 0);
-            if (r < G && r < 16) {
-                const uint4 *qr = reinterpret_cast<const uint4 *>(qg + (size_t)r * kDqk);
-                if (w < npair) {
-                    va[k] = __ldg(qr + w);
-                    vb[k] = __ldg(qr + w + npair);
-                } else {
-                    va[k] = __ldg(qr + npair + w);
-                }
-            }
-        }
+    if (vec_rope) {
+        // Query heads of this KV group rotated at position L-1 (rows >= G are 0).
 #pragma unroll
         for (int k = 0; k < 3; ++k) {
             const int u = tid + k * kThreads;
@@ -209,36 +229,42 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
             sQ[r * kQStride + e] = __float2bfloat16_rn(y);
         }
     }
-    // New token: rotate k, write k and v into the cache slot, keep a copy.
+    // New token (CTA-uniform branch): rotate k from its raw copy, then write k
+    // and v into the cache slot and keep the rotated copy for the tile.
     if (owns_new) {
-        const __nv_bfloat16 *kn = reinterpret_cast<const __nv_bfloat16 *>(a.k_new) +
-                                  ((size_t)b * L.Hkv + kvh) * kDqk;
-        const __nv_bfloat16 *vn = reinterpret_cast<const __nv_bfloat16 *>(a.v_new) +
-                                  ((size_t)b * L.Hkv + kvh) * kDv;
         __nv_bfloat16 *kdst = reinterpret_cast<__nv_bfloat16 *>(a.k_cache) +
                               (((size_t)b * a.cap + slot_new) * kv_row + kvh) * kDqk;
         __nv_bfloat16 *vdst = reinterpret_cast<__nv_bfloat16 *>(a.v_cache) +
                               (((size_t)b * a.cap + slot_new) * kv_row + kvh) * kDv;
-        for (int e = tid; e < kDqk; e += kThreads) {
-            float y;
-            if (e < L.rope.rotary_dim) {
-                const int j = e < half ? e : e - half;
-                const float2 cs = s_cs[j];
-                const float xa = __bfloat162float(kn[j]);
-                const float xb = __bfloat162float(kn[j + half]);
-                y = e < half ? xa * cs.x - xb * cs.y : xb * cs.x + xa * cs.y;
-            } else {
-                y = __bfloat162float(kn[e]);
+        __nv_bfloat16 yk[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int e = tid + k * kThreads;
+            float y = 0.f;
+            if (e < kDqk) {
+                if (e < L.rope.rotary_dim) {
+                    const int j = e < half ? e : e - half;
+                    const float2 cs = s_cs[j];
+                    const float xa = __bfloat162float(sKnew[j]);
+                    const float xb = __bfloat162float(sKnew[j + half]);
+                    y = e < half ? xa * cs.x - xb * cs.y : xb * cs.x + xa * cs.y;
+                } else {
+                    y = __bfloat162float(sKnew[e]);
+                }
             }
-            const __nv_bfloat16 yb = __float2bfloat16_rn(y);
-            sKnew[e] = yb;
-            kdst[e] = yb;
+            yk[k] = __float2bfloat16_rn(y);
         }
-        for (int e = tid; e < kDv; e += kThreads) {
-            const __nv_bfloat16 x = vn[e];
-            sVnew[e] = x;
-            vdst[e] = x;
+        __syncthreads();  // every raw element read before any is overwritten
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int e = tid + k * kThreads;
+            if (e < kDqk) {
+                sKnew[e] = yk[k];
+                kdst[e] = yk[k];
+            }
         }
+        if (tid < kDv)
+            vdst[tid] = sVnew[tid];
     }
     __syncthreads();
 
@@ -263,7 +289,14 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
         o[d][0] = o[d][1] = o[d][2] = o[d][3] = 0.f;
 
     for (int t = 0; t < n_tiles; ++t) {
-        cp_async_wait<kStages - 2>();
+        // Tile t + kStages - 1 goes out before the wait for tile t, so kStages
+        // tiles are in flight during it; the barrier first makes sure every
+        // warp is done with the buffer it refills (that of tile t - 1).
+        __syncthreads();
+        if (t + kStages - 1 < n_tiles)
+            issue(t + kStages - 1);
+        cp_async_commit();
+        cp_async_wait<kStages - 1>();
         __syncthreads();
         __nv_bfloat16 *st = sStage + (t % kStages) * kStageElems;
         const int base_key = key_begin + t * kTileKeys;
@@ -277,9 +310,6 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
                     *reinterpret_cast<const uint4 *>(sVnew + (tid - 24) * 8);
             __syncthreads();
         }
-        if (t + kStages - 1 < n_tiles)
-            issue(t + kStages - 1);
-        cp_async_commit();
         const int kb = warp * 16;  // this warp's 16 keys within the tile
         if (base_key + kb >= key_end)
             continue;
@@ -376,9 +406,7 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
         red.wl[warp][g] = l0;
         red.wl[warp][g + 8] = l1;
     }
-    for (int idx = tid; idx < 16 * kDv; idx += kThreads)
-        (&red.o[0][0])[idx] = 0.f;
-    __syncthreads();
+    __syncthreads();  // every warp is past its last tile: the stage buffers are free
     float M0 = -INFINITY, M1 = -INFINITY;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
@@ -387,19 +415,20 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
     }
     const float f0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M0);
     const float f1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M1);
-    for (int w = 0; w < 4; ++w) {
-        if (warp == w) {
+    // Each warp writes its rescaled partial O into its own slice (rows padded
+    // to kMergeStride floats: the 8 rows of a warp's access fall in different
+    // banks), then one pass sums the four slices.
+    float *slices = reinterpret_cast<float *>(sStage);
+    {
+        float *sl = slices + warp * 16 * kMergeStride;
 #pragma unroll
-            for (int d = 0; d < 16; ++d) {
-                const int col = d * 8 + 2 * tq;
-                red.o[g][col] += o[d][0] * f0;
-                red.o[g][col + 1] += o[d][1] * f0;
-                red.o[g + 8][col] += o[d][2] * f1;
-                red.o[g + 8][col + 1] += o[d][3] * f1;
-            }
+        for (int d = 0; d < 16; ++d) {
+            const int col = d * 8 + 2 * tq;
+            *reinterpret_cast<float2 *>(sl + g * kMergeStride + col) = make_float2(o[d][0] * f0, o[d][1] * f0);
+            *reinterpret_cast<float2 *>(sl + (g + 8) * kMergeStride + col) = make_float2(o[d][2] * f1, o[d][3] * f1);
         }
-        __syncthreads();
     }
+    __syncthreads();
 
     // Row r = query head kvh*G + r; thread -> (row, 16 columns).
     for (int idx = tid; idx < G * (kDv / 16); idx += kThreads) {
@@ -413,6 +442,24 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
 #pragma unroll
         for (int w = 0; w < 4; ++w)
             Ls += (red.wm[w][r] == -INFINITY) ? 0.f : red.wl[w][r] * exp2f(red.wm[w][r] - M);
+        // this row's 16 columns, summed over the four warps' slices
+        float v[16];
+#pragma unroll
+        for (int c = 0; c < 16; c += 4) {
+            float4 acc = *reinterpret_cast<const float4 *>(slices + r * kMergeStride + c0 + c);
+#pragma unroll
+            for (int w = 1; w < 4; ++w) {
+                const float4 x = *reinterpret_cast<const float4 *>(slices + (w * 16 + r) * kMergeStride + c0 + c);
+                acc.x += x.x;
+                acc.y += x.y;
+                acc.z += x.z;
+                acc.w += x.w;
+            }
+            v[c] = acc.x;
+            v[c + 1] = acc.y;
+            v[c + 2] = acc.z;
+            v[c + 3] = acc.w;
+        }
         const int h = kvh * G + r;
         if (nsplit == 1) {
             float scale;
@@ -426,21 +473,21 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
             }
             __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.out) + ((size_t)b * L.Hq + h) * kDv + c0;
             uint4 w0, w1;
-            w0.x = pack_bf16x2(red.o[r][c0 + 0] * scale, red.o[r][c0 + 1] * scale);
-            w0.y = pack_bf16x2(red.o[r][c0 + 2] * scale, red.o[r][c0 + 3] * scale);
-            w0.z = pack_bf16x2(red.o[r][c0 + 4] * scale, red.o[r][c0 + 5] * scale);
-            w0.w = pack_bf16x2(red.o[r][c0 + 6] * scale, red.o[r][c0 + 7] * scale);
-            w1.x = pack_bf16x2(red.o[r][c0 + 8] * scale, red.o[r][c0 + 9] * scale);
-            w1.y = pack_bf16x2(red.o[r][c0 + 10] * scale, red.o[r][c0 + 11] * scale);
-            w1.z = pack_bf16x2(red.o[r][c0 + 12] * scale, red.o[r][c0 + 13] * scale);
-            w1.w = pack_bf16x2(red.o[r][c0 + 14] * scale, red.o[r][c0 + 15] * scale);
+            w0.x = pack_bf16x2(v[0] * scale, v[1] * scale);
+            w0.y = pack_bf16x2(v[2] * scale, v[3] * scale);
+            w0.z = pack_bf16x2(v[4] * scale, v[5] * scale);
+            w0.w = pack_bf16x2(v[6] * scale, v[7] * scale);
+            w1.x = pack_bf16x2(v[8] * scale, v[9] * scale);
+            w1.y = pack_bf16x2(v[10] * scale, v[11] * scale);
+            w1.z = pack_bf16x2(v[12] * scale, v[13] * scale);
+            w1.w = pack_bf16x2(v[14] * scale, v[15] * scale);
             reinterpret_cast<uint4 *>(dst)[0] = w0;
             reinterpret_cast<uint4 *>(dst)[1] = w1;
         } else {
             float *part = a.partial + (((size_t)b * L.Hq + h) * a.max_splits + split) * (kDv + 2);
 #pragma unroll
             for (int c = 0; c < 16; ++c)
-                part[c0 + c] = red.o[r][c0 + c];
+                part[c0 + c] = v[c];
             if (c0 == 0) {
                 part[kDv] = M;
                 part[kDv + 1] = Ls;
