@@ -185,3 +185,63 @@ def prefill_layer(q, k, v, *, layer_type: int, num_kv_heads: int, rotary_dim: in
             out[b, rows, h, :] = prefill_rows(q_rot, rows, k_rot[kv], v[b, :, kv, :], layer_type,
                                               window, scale, sink, vs)
     return out
+
+
+def prefill_cached_layer(q, k, v, k_cache, v_cache, past_lens, *, layer_type: int, num_kv_heads: int,
+                         rotary_dim: int, theta: float, window: int, sinks, hidden_size: int,
+                         softmax_scale: Optional[float] = None, rows=None, heads=None, batches=None):
+    """Prefill of a chunk that continues a cache (the cache-aware prefill of the
+    rotating cache: lablup/mlxcel issue 842, "Implementation plan"). Token t
+    of batch b sits at position P_b + t, P_b = past_lens[b]. Its keys are the
+    cached ones (already rotated: a global cache holds position p in slot p, a
+    sliding ring holds the last `window` positions in slots p mod window) and
+    the chunk's own keys, rotated at their positions, up to itself, with the
+    layer's mask (causal; window on sliding layers).
+
+    q [B, S, Hq, Dqk], k [B, S, Hkv, Dqk], v [B, S, Hkv, Dv] (unrotated);
+    k_cache [B, cap, Hkv, Dqk], v_cache [B, cap, Hkv, Dv] (cap = window on a
+    sliding layer). Returns (out [B, S, Hq, Dv], k_cache', v_cache') with the
+    chunk's rotated keys and its values written into their slots, in token
+    order (on a ring a later token takes the slot of an earlier one).
+    """
+    q = np.asarray(q)
+    k = np.asarray(k)
+    v = np.asarray(v)
+    B, S, Hq, Dqk = q.shape
+    Dv = v.shape[3]
+    G = Hq // num_kv_heads
+    kc = np.array(k_cache, dtype=np.float64, copy=True, order="C")
+    vc = np.array(v_cache, dtype=np.float64, copy=True, order="C")
+    scale = default_softmax_scale(Dqk) if softmax_scale is None else softmax_scale
+    vs = v_scale(hidden_size, Hq, Dv)
+    rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
+    heads = range(Hq) if heads is None else heads
+    past = [int(x) for x in np.asarray(past_lens).reshape(-1)]
+    out = np.full((B, S, Hq, Dv), np.nan, dtype=np.float64)
+    for b in range(B):
+        P = past[b]
+        n = P + S
+        pos_new = P + np.arange(S, dtype=np.float64)
+        # keys and values over positions [0, P + S)
+        K = np.zeros((n, num_kv_heads, Dqk))
+        V = np.zeros((n, num_kv_heads, Dv))
+        for p in range(P):
+            if layer_type == GLOBAL:
+                K[p], V[p] = kc[b, p], vc[b, p]
+            elif p >= P - (window - 1):  # older positions are outside every query's window
+                K[p], V[p] = kc[b, p % window], vc[b, p % window]
+        for kv in range(num_kv_heads):
+            K[P:, kv] = rope(k[b, :, kv, :], rotary_dim, theta, pos_new)
+        V[P:] = _f64(v[b])
+        if batches is None or b in batches:
+            for h in heads:
+                kv = h // G
+                q_rot = rope(q[b, rows, h, :], rotary_dim, theta, pos_new[rows])
+                sink = None if sinks is None else float(np.asarray(sinks)[h])
+                out[b, rows, h, :] = prefill_rows(q_rot, P + rows, K[:, kv, :], V[:, kv, :], layer_type,
+                                                  window, scale, sink, vs)
+        for t in range(S):
+            p = P + t
+            slot = p if layer_type == GLOBAL else p % window
+            kc[b, slot], vc[b, slot] = K[p], V[p]
+    return out, kc, vc

@@ -319,3 +319,79 @@ def test_decode_rejects_bad_lengths():
         oracle.decode(rnd(1, D), rnd(D), rnd(Dv), rnd(4, D), rnd(4, Dv), 0, 4, 1e4, 0, 0, 1.0, None, 1.0)
     with pytest.raises(ValueError):  # ring capacity must equal the window
         oracle.decode(rnd(1, D), rnd(D), rnd(Dv), rnd(4, D), rnd(4, Dv), 3, 4, 1e4, 1, 5, 1.0, None, 1.0)
+
+
+# --------------------------------------------------- prefill continuing a cache
+
+def _chunk_layer(layer_type, W):
+    return dict(layer_type=layer_type, num_kv_heads=2, rotary_dim=16, theta=1e4 if layer_type else 1e6,
+                window=W, hidden_size=256)
+
+
+@pytest.mark.parametrize("layer_type,W", [(0, 0), (1, 4), (1, 16)])
+def test_cached_prefill_with_empty_cache_is_plain_prefill(layer_type, W):
+    """With no past tokens the chunk is a whole sequence: prefill_layer's
+    output, and the cache holds the rotated keys / values in their slots.
+    Catches a position offset applied twice or a wrong slot."""
+    B, S, Hq, D, Dv = 2, 11, 4, 48, 32
+    q, k, v = rnd(B, S, Hq, D), rnd(B, S, 2, D), rnd(B, S, 2, Dv)
+    sinks = rnd(Hq) if layer_type else None
+    kw = _chunk_layer(layer_type, W)
+    cap = S if layer_type == 0 else W
+    out, kc, vc = oracle.prefill_cached_layer(q, k, v, np.zeros((B, cap, 2, D)), np.zeros((B, cap, 2, Dv)),
+                                              [0, 0], sinks=sinks, **kw)
+    ref = oracle.prefill_layer(q, k, v, sinks=sinks, **kw)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-13)
+    for b in range(B):
+        for p in range(S):
+            if layer_type == 1 and p < S - W:
+                continue  # overwritten by a later token of the ring
+            slot = p if layer_type == 0 else p % W
+            for kv in range(2):
+                kr = oracle.rope(k[b, p, kv], 16, kw["theta"], [float(p)])
+                np.testing.assert_allclose(kc[b, slot, kv], kr, rtol=0, atol=1e-14)
+                assert np.array_equal(vc[b, slot, kv], v[b, p, kv])
+
+
+@pytest.mark.parametrize("layer_type,W,S1,S2", [(0, 0, 7, 9), (0, 0, 1, 1), (1, 4, 6, 7), (1, 8, 3, 20),
+                                                (1, 8, 20, 3), (1, 16, 5, 5)])
+def test_two_chunks_equal_one_shot(layer_type, W, S1, S2):
+    """Prefilling S1 tokens, then continuing with S2 from the resulting cache,
+    gives the one-shot prefill's last S2 rows, for sliding layers also when a
+    chunk is longer than the window (ring wrap). Ties the cached path to the
+    plain prefill, which is pinned to SDPA; catches an off-by-one in the
+    positions, the window or the ring slot."""
+    B, Hq, D, Dv = 2, 4, 48, 32
+    S = S1 + S2
+    q, k, v = rnd(B, S, Hq, D), rnd(B, S, 2, D), rnd(B, S, 2, Dv)
+    sinks = rnd(Hq) if layer_type else None
+    kw = _chunk_layer(layer_type, W)
+    cap = S if layer_type == 0 else W
+    kc0, vc0 = np.zeros((B, cap, 2, D)), np.zeros((B, cap, 2, Dv))
+    _, kc1, vc1 = oracle.prefill_cached_layer(q[:, :S1], k[:, :S1], v[:, :S1], kc0, vc0, [0, 0],
+                                              sinks=sinks, **kw)
+    out2, _, _ = oracle.prefill_cached_layer(q[:, S1:], k[:, S1:], v[:, S1:], kc1, vc1, [S1, S1],
+                                             sinks=sinks, **kw)
+    ref = oracle.prefill_layer(q, k, v, sinks=sinks, **kw)
+    np.testing.assert_allclose(out2, ref[:, S1:], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("layer_type,W,P", [(0, 0, 0), (0, 0, 13), (1, 8, 3), (1, 8, 21)])
+def test_one_token_chunk_equals_decode(layer_type, W, P):
+    """A one-token chunk is a decode step: same output, same cache afterwards
+    (oracle.decode counts the new token in L = P + 1)."""
+    Hq, D, Dv = 4, 48, 32
+    kw = _chunk_layer(layer_type, W)
+    cap = 32 if layer_type == 0 else W
+    kc, vc = rnd(1, cap, 2, D), rnd(1, cap, 2, Dv)
+    q, k, v = rnd(1, 1, Hq, D), rnd(1, 1, 2, D), rnd(1, 1, 2, Dv)
+    sinks = rnd(Hq) if layer_type else None
+    out, kc2, vc2 = oracle.prefill_cached_layer(q, k, v, kc, vc, [P], sinks=sinks, **kw)
+    for kv in range(2):
+        hs = slice(2 * kv, 2 * kv + 2)
+        o, kcd, vcd = oracle.decode(q[0, 0, hs], k[0, 0, kv], v[0, 0, kv], kc[0, :, kv], vc[0, :, kv], P + 1,
+                                    16, kw["theta"], layer_type, W, 1 / math.sqrt(D),
+                                    None if sinks is None else sinks[hs], oracle.v_scale(256, Hq, Dv))
+        np.testing.assert_allclose(out[0, 0, hs], o, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(kc2[0, :, kv], kcd, rtol=0, atol=1e-14)
+        np.testing.assert_allclose(vc2[0, :, kv], vcd, rtol=0, atol=0)
