@@ -32,6 +32,8 @@ EXPORTED = (
     "mimo_attn_rotary_dim",
     "mimo_attn_prefill_workspace_size",
     "mimo_attn_prefill",
+    "mimo_attn_prefill_cached_workspace_size",
+    "mimo_attn_prefill_cached",
     "mimo_attn_decode_workspace_size",
     "mimo_attn_decode",
     "mimo_attn_decode_static",
@@ -84,6 +86,10 @@ def load() -> ctypes.CDLL:
     lib.mimo_attn_prefill_workspace_size.restype = sz
     lib.mimo_attn_prefill.argtypes = [lp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]
     lib.mimo_attn_prefill.restype = i32
+    lib.mimo_attn_prefill_cached_workspace_size.argtypes = [lp, i32, i32, i32, i32]
+    lib.mimo_attn_prefill_cached_workspace_size.restype = sz
+    lib.mimo_attn_prefill_cached.argtypes = [lp, i32, i32, i32, vp, vp, vp, vp, i32, vp, vp, vp, i32, vp, sz, vp]
+    lib.mimo_attn_prefill_cached.restype = i32
     lib.mimo_attn_decode_workspace_size.argtypes = [lp, i32, i32, i32]
     lib.mimo_attn_decode_workspace_size.restype = sz
     lib.mimo_attn_decode.argtypes = [lp, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
@@ -180,6 +186,22 @@ def mimo_attn_prefill(layer: mimo_attn_layer, dtype: int, batch: int, seq: int, 
         _stream(stream)))
 
 
+def mimo_attn_prefill_cached_workspace_size(layer: mimo_attn_layer, dtype: int, batch: int, seq: int,
+                                            max_past_len: int) -> int:
+    return int(load().mimo_attn_prefill_cached_workspace_size(ctypes.byref(layer), dtype, batch, seq,
+                                                              int(max_past_len)))
+
+
+def mimo_attn_prefill_cached(layer: mimo_attn_layer, dtype: int, batch: int, seq: int, q, k, v, past_lens,
+                             max_past_len: int, out, k_cache, v_cache, cache_capacity: int, workspace=None,
+                             workspace_bytes: int = 0, stream=None) -> int:
+    """Same arguments as the C entry point; tensors in place of pointers."""
+    return int(load().mimo_attn_prefill_cached(
+        ctypes.byref(layer), dtype, batch, seq, _ptr(q), _ptr(k), _ptr(v), _ptr(past_lens), int(max_past_len),
+        _ptr(out), _ptr(k_cache), _ptr(v_cache), int(cache_capacity), _ptr(workspace), int(workspace_bytes),
+        _stream(stream)))
+
+
 def mimo_attn_decode(layer: mimo_attn_layer, dtype: int, batch: int, q, k_new, v_new, kv_lens, k_cache,
                      v_cache, cache_capacity: int, out, workspace=None, workspace_bytes: int = 0,
                      stream=None) -> int:
@@ -238,6 +260,28 @@ def prefill(layer: mimo_attn_layer, q: torch.Tensor, k: torch.Tensor, v: torch.T
     cap = 0 if k_cache is None else k_cache.shape[1]
     _check(mimo_attn_prefill(layer, dt, B, S, q, k, v, positions, out, k_cache, v_cache, cap, workspace,
                              0 if workspace is None else workspace.numel(), stream), "mimo_attn_prefill")
+    return out
+
+
+def prefill_cached(layer: mimo_attn_layer, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                   past_lens: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                   max_past_len: Optional[int] = None, out: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Runs mimo_attn_prefill_cached (a chunk after past_lens[b] cached tokens;
+    updates the caches in place). max_past_len defaults to max(past_lens), read
+    on the host (one synchronisation); pass it to avoid that."""
+    B, S = q.shape[0], q.shape[1]
+    dt = dtype_code(q.dtype)
+    if max_past_len is None:
+        max_past_len = int(past_lens.max().item()) if past_lens.numel() else 0
+    if out is None:
+        out = torch.empty((B, S, layer.num_q_heads, layer.v_dim), dtype=q.dtype, device=q.device)
+    need = mimo_attn_prefill_cached_workspace_size(layer, dt, B, S, max_past_len)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check(mimo_attn_prefill_cached(layer, dt, B, S, q, k, v, past_lens, max_past_len, out, k_cache, v_cache,
+                                    k_cache.shape[1], workspace, 0 if workspace is None else workspace.numel(),
+                                    stream), "mimo_attn_prefill_cached")
     return out
 
 

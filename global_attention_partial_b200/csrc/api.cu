@@ -107,6 +107,11 @@ mimo_attn_status resolve_layer(const mimo_attn_layer *layer, int dtype, mimo::La
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Continuing a cache on a sliding layer: window row of query 0. At least the
+// window - 1 older positions precede it; a multiple of 16 keeps the 16-key
+// blocks of the tensor-core kernel aligned with the queries' spans.
+int cached_key_off(const mimo::LayerArgs &L) { return (int)round_up((size_t)(L.window - 1), 16); }
+
 } // namespace
 
 extern "C" {
@@ -200,10 +205,13 @@ mimo_attn_status mimo_attn_prefill(const mimo_attn_layer *layer, int dtype, int 
         return MIMO_ATTN_ERR_CUDA;
 
     mimo::PrefillArgs pa;
+    memset(&pa, 0, sizeof(pa));
     pa.q = q;
     pa.krot = kp.dst_k;
     pa.krot_rows = kp.dst_rows;
+    pa.key_rows_valid = seq;
     pa.v = v;
+    pa.v_rows = seq;
     pa.positions = positions;
     pa.rope_table = kp.rope_table;
     pa.out = out;
@@ -217,6 +225,121 @@ mimo_attn_status mimo_attn_prefill(const mimo_attn_layer *layer, int dtype, int 
         e = mimo::launch_prefill_ga(L, pa, s);
     else if (dtype == MIMO_ATTN_BF16 && mimo::prefill_tc_supported(L))
         e = mimo::launch_prefill_tc(L, pa, s);
+    else
+        e = mimo::launch_prefill_simt(L, pa, dtype, s);
+    return e == cudaSuccess ? MIMO_ATTN_OK : MIMO_ATTN_ERR_CUDA;
+}
+
+size_t mimo_attn_prefill_cached_workspace_size(const mimo_attn_layer *layer, int dtype, int batch, int seq,
+                                               int max_past_len)
+{
+    mimo::LayerArgs L;
+    if (resolve_layer(layer, dtype, &L) != MIMO_ATTN_OK || batch < 0 || seq < 0 || max_past_len < 0)
+        return 0;
+    // the RoPE table of positions 0 .. max_past + seq - 1, then (SWA) the key
+    // and value windows [B, key_off + seq, Hkv, D]
+    size_t bytes = round_up(((size_t)max_past_len + seq) * L.rope.half * sizeof(float2), 256);
+    if (L.layer_type == MIMO_ATTN_SWA) {
+        const size_t rows = (size_t)batch * (cached_key_off(L) + seq) * L.Hkv;
+        bytes += round_up(rows * L.Dqk * elem_size(dtype), 256) + round_up(rows * L.Dv * elem_size(dtype), 256);
+    }
+    return bytes;
+}
+
+mimo_attn_status mimo_attn_prefill_cached(const mimo_attn_layer *layer, int dtype, int batch, int seq,
+                                          const void *q, const void *k, const void *v, const int32_t *past_lens,
+                                          int max_past_len, void *out, void *k_cache, void *v_cache,
+                                          int cache_capacity, void *workspace, size_t workspace_bytes,
+                                          void *stream)
+{
+    mimo::LayerArgs L;
+    mimo_attn_status st = resolve_layer(layer, dtype, &L);
+    if (st != MIMO_ATTN_OK)
+        return st;
+    if (batch < 0 || seq < 0 || max_past_len < 0)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (k_cache == nullptr || v_cache == nullptr)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (L.layer_type == MIMO_ATTN_SWA && cache_capacity != L.window)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (L.layer_type == MIMO_ATTN_GLOBAL && (long long)cache_capacity < (long long)max_past_len + seq)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (batch == 0 || seq == 0)
+        return MIMO_ATTN_OK;
+    if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || past_lens == nullptr)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (dtype == MIMO_ATTN_BF16 &&
+        !(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out) && aligned16(k_cache) &&
+          aligned16(v_cache) && aligned16(workspace)))
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    const size_t need = mimo_attn_prefill_cached_workspace_size(layer, dtype, batch, seq, max_past_len);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+        return MIMO_ATTN_ERR_WORKSPACE;
+    if (g_fail_launches)
+        return MIMO_ATTN_ERR_CUDA;
+    unsigned *err = device_error_ptr();
+    if (err == nullptr)
+        return MIMO_ATTN_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    const bool swa = L.layer_type == MIMO_ATTN_SWA;
+    const int key_off = swa ? cached_key_off(L) : 0;
+    const size_t table_bytes = round_up(((size_t)max_past_len + seq) * L.rope.half * sizeof(float2), 256);
+    float2 *table = L.rope.half > 0 ? reinterpret_cast<float2 *>(workspace) : nullptr;
+    char *win = static_cast<char *>(workspace) + table_bytes;
+    const size_t win_rows = (size_t)batch * (key_off + seq) * L.Hkv;
+    void *win_k = swa ? static_cast<void *>(win) : nullptr;
+    void *win_v = swa ? static_cast<void *>(win + round_up(win_rows * L.Dqk * elem_size(dtype), 256)) : nullptr;
+    if (mimo::launch_rope_table(L.rope, table, (long long)max_past_len + seq, s) != cudaSuccess)
+        return MIMO_ATTN_ERR_CUDA;
+
+    mimo::CachedPrepArgs cp;
+    memset(&cp, 0, sizeof(cp));
+    cp.k = k;
+    cp.v = v;
+    cp.past_lens = past_lens;
+    cp.max_past = max_past_len;
+    cp.k_cache = k_cache;
+    cp.v_cache = v_cache;
+    cp.cap = cache_capacity;
+    cp.kv_k = win_k;
+    cp.kv_v = win_v;
+    cp.key_off = key_off;
+    cp.layer_type = L.layer_type;
+    cp.B = batch;
+    cp.S = seq;
+    cp.Hkv = L.Hkv;
+    cp.Dqk = L.Dqk;
+    cp.Dv = L.Dv;
+    cp.window = L.window;
+    cp.rope_table = table;
+    cp.rope = L.rope;
+    cp.err = err;
+    if (mimo::launch_cached_prep(cp, dtype, s) != cudaSuccess)
+        return MIMO_ATTN_ERR_CUDA;
+
+    // Keys and values: the global cache itself, or the SWA windows.
+    mimo::PrefillArgs pa;
+    memset(&pa, 0, sizeof(pa));
+    pa.q = q;
+    pa.krot = swa ? win_k : k_cache;
+    pa.krot_rows = swa ? key_off + seq : cache_capacity;
+    pa.key_rows_valid = pa.krot_rows;
+    pa.v = swa ? win_v : v_cache;
+    pa.v_rows = pa.krot_rows;
+    pa.rope_table = table;
+    pa.past_lens = past_lens;
+    pa.max_past = max_past_len;
+    pa.swa_key_off = key_off;
+    pa.out = out;
+    pa.B = batch;
+    pa.S = seq;
+    pa.err = err;
+    cudaError_t e;
+    if (dtype == MIMO_ATTN_BF16 && swa && mimo::prefill_swa_supported(L))
+        e = mimo::launch_prefill_swa(L, pa, table, num_sms(), s);
+    else if (dtype == MIMO_ATTN_BF16 && !swa && mimo::prefill_ga_supported(L))
+        e = mimo::launch_prefill_ga(L, pa, s);
     else
         e = mimo::launch_prefill_simt(L, pa, dtype, s);
     return e == cudaSuccess ? MIMO_ATTN_OK : MIMO_ATTN_ERR_CUDA;

@@ -40,15 +40,53 @@ struct KprepArgs {
 };
 cudaError_t launch_kprep(const KprepArgs &a, int dtype, cudaStream_t stream);
 
+// cos / sin of positions 0..n-1 for every rotary pair: table [n][rotary_dim/2].
+cudaError_t launch_rope_table(const RopeArgs &rope, float2 *table, long long n, cudaStream_t stream);
+
+// Prefill continuing a cache: writes the chunk's rotated keys and values
+// where the attention kernels read them. Global layers: cache rows
+// past_lens[b] + t. Sliding layers: the key window kv_k / kv_v
+// [B, key_off + S, Hkv, D] (row u = position past_lens[b] - key_off + u: old
+// keys from the ring, the chunk's own rotated), then the ring takes the
+// chunk's last `window` tokens. Out-of-range past_lens set the device error
+// word; their rows are skipped.
+struct CachedPrepArgs {
+    const void *k;
+    const void *v;
+    const int *past_lens;
+    int max_past;
+    void *k_cache;
+    void *v_cache;
+    int cap;
+    void *kv_k;
+    void *kv_v;
+    int key_off;
+    int layer_type, B, S, Hkv, Dqk, Dv, window;
+    const float2 *rope_table;
+    RopeArgs rope;
+    unsigned *err;
+};
+cudaError_t launch_cached_prep(const CachedPrepArgs &a, int dtype, cudaStream_t stream);
+
 // Prefill attention on CUDA cores (any dims up to 256, fp32 or bf16).
 // krot: rotated keys [B, krot_rows, Hkv, Dqk].
+// Query token t of batch b attends the keys of index (t + key offset), the
+// key offset being past_lens[b] on global layers and swa_key_off on sliding
+// layers; without past_lens (plain prefill) both are 0 and queries and keys
+// share the sequence index. krot / v hold key_rows / v_rows rows per batch
+// (row stride krot_rows / v_rows), of which the first key_rows_valid are read.
 struct PrefillArgs {
     const void *q;
     const void *krot;
     long long krot_rows;
+    long long key_rows_valid;
     const void *v;
+    long long v_rows;
     const int *positions;
-    const float2 *rope_table;  // [S][rotary_dim/2] (cos, sin), built by launch_kprep
+    const float2 *rope_table;  // (cos, sin) per position: row (past_lens[b] + t) for token t
+    const int *past_lens;      // [B] tokens already in the cache, or nullptr
+    int max_past;              // >= every past_lens[b]: the table has max_past + S rows
+    int swa_key_off;           // sliding layers: key index of query 0 (a multiple of 16)
     void *out;
     int B, S;
     unsigned *err;

@@ -68,10 +68,13 @@ struct GaParams {
     CUtensorMap tm_v;  // [B, S, Hkv, Dv]     box {64, 1, 128, 1}
     __nv_bfloat16 *out;
     int out_v8;                // out is 32-byte aligned: 256-bit stores
-    const float2 *rope_table;  // [S][half]
+    const float2 *rope_table;  // row (past + i): (cos, sin) of the pairs at query i's position
     const float *sinks;        // nullptr on global layers
+    const int *past_lens;      // [B] cached tokens before the chunk, or nullptr
     unsigned *err;
     int S, Hq, G, num_p_tiles, num_pairs;
+    int key_rows;              // key rows readable per batch (cache capacity when continuing a cache)
+    int max_past;              // the RoPE table has max_past + S rows
     int rope_half;
     float scale_log2;
     float v_scale;
@@ -111,7 +114,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_ga_kernel(const __grid_co
     const int hA = kvh * p.G + 2 * (pair % (p.G / 2));
     const int p0 = pt * kBlockM;
     const int q_last = min(p0 + kBlockM, p.S) - 1;
-    const int n_tiles = q_last / kBlockN + 1;
+    // Query i is the token at key index past + i (past = 0 for a plain prefill).
+    const int past = p.past_lens != nullptr ? __ldg(p.past_lens + b) : 0;
+    if (past < 0 || past > p.max_past || past + p.S > p.key_rows) {  // the whole CTA leaves before any setup
+        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0)
+            atomicOr(p.err, kErrKvLen);
+        return;
+    }
+    const int n_tiles = (q_last + past) / kBlockN + 1;
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
@@ -316,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_ga_kernel(const __grid_co
         const int half = p.rope_half;
         if (ok && row_valid && half > 0) {
             uint8_t *qt = sQ + t * kQBytes;
-            const float2 *cs = p.rope_table + (size_t)i * half;
+            const float2 *cs = p.rope_table + (size_t)(past + i) * half;
             for (int j = 0; j < half; ++j) {
                 const int ea = j, eb = j + half;
                 __nv_bfloat16 *pa = reinterpret_cast<__nv_bfloat16 *>(
@@ -359,9 +369,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_ga_kernel(const __grid_co
                 }
             }
             const int k0 = j * kBlockN;
-            if (k0 + kBlockN - 1 > p0) {
-                // diagonal tile: key c visible iff k0 + c <= i (branch-free)
-                const int hi = i - k0;
+            if (k0 + kBlockN - 1 > p0 + past) {
+                // diagonal tile: key c visible iff k0 + c <= past + i (branch-free)
+                const int hi = past + i - k0;
 #pragma unroll
                 for (int c = 0; c < kBlockN; ++c)
                     x[c] = (c <= hi) ? x[c] : -INFINITY;
@@ -468,15 +478,18 @@ cudaError_t launch_prefill_ga(const LayerArgs &L, const PrefillArgs &a, cudaStre
     GaParams p;
     memset(&p, 0, sizeof(p));
     if (!make_bf16_map_4d(&p.tm_q, a.q, kDqk, L.Hq, a.S, a.S, a.B, 64, 1, kBlockM) ||
-        !make_bf16_map_4d(&p.tm_k, a.krot, kDqk, L.Hkv, a.S, a.krot_rows, a.B, 64, 1, kBlockN) ||
-        !make_bf16_map_4d(&p.tm_v, a.v, kDv, L.Hkv, a.S, a.S, a.B, 64, 1, kBlockN))
+        !make_bf16_map_4d(&p.tm_k, a.krot, kDqk, L.Hkv, a.key_rows_valid, a.krot_rows, a.B, 64, 1, kBlockN) ||
+        !make_bf16_map_4d(&p.tm_v, a.v, kDv, L.Hkv, a.key_rows_valid, a.v_rows, a.B, 64, 1, kBlockN))
         return cudaErrorInvalidValue;
     p.out = reinterpret_cast<__nv_bfloat16 *>(a.out);
     p.out_v8 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
     p.rope_table = a.rope_table;
     p.sinks = L.sinks;
+    p.past_lens = a.past_lens;
     p.err = a.err;
     p.S = a.S;
+    p.key_rows = (int)a.key_rows_valid;
+    p.max_past = a.past_lens != nullptr ? a.max_past : 0;
     p.Hq = L.Hq;
     p.G = L.G;
     p.num_p_tiles = (a.S + kBlockM - 1) / kBlockM;

@@ -169,8 +169,15 @@ __global__ void prefill_simt_kernel(const __grid_constant__ LayerArgs L, const _
     const int b = blockIdx.z;
     if (i >= a.S)
         return;
+    // Query i is the token at position past + i and key index past + i
+    // (global) or swa_key_off + i (sliding window); past = 0 for a plain prefill.
+    const int past = a.past_lens != nullptr ? min(max(__ldg(a.past_lens + b), 0), a.max_past) : 0;
+    const int key_off = a.past_lens == nullptr ? 0 : (L.layer_type == 1 ? a.swa_key_off : past);
+    const int ki = i + key_off;
+    if (ki >= a.key_rows_valid)  // out-of-range past_lens: reported by the cache prep
+        return;
     const int half = L.rope.half;
-    const float2 *cs = a.rope_table + (size_t)i * half;
+    const float2 *cs = a.rope_table + (size_t)(past + i) * half;
     const T *q = reinterpret_cast<const T *>(a.q) + (((size_t)b * a.S + i) * L.Hq + h) * L.Dqk;
     for (int e = lane; e < L.Dqk; e += 32) {
         float y;
@@ -187,13 +194,13 @@ __global__ void prefill_simt_kernel(const __grid_constant__ LayerArgs L, const _
     }
     __syncwarp();
     const int kvh = h / L.G;
-    const int lo = L.layer_type == 1 ? max(0, i - L.window + 1) : 0;
+    const int lo = L.layer_type == 1 ? max(max(0, key_off - past), ki - L.window + 1) : 0;
     float m = -INFINITY, l = 0.f;
     float acc[8];
 #pragma unroll
     for (int t = 0; t < 8; ++t)
         acc[t] = 0.f;
-    for (int j = lo; j <= i; ++j) {
+    for (int j = lo; j <= ki; ++j) {
         const T *kr = reinterpret_cast<const T *>(a.krot) + (((size_t)b * a.krot_rows + j) * L.Hkv + kvh) * L.Dqk;
         float part = 0.f;
         for (int e = lane; e < L.Dqk; e += 32)
@@ -206,7 +213,7 @@ __global__ void prefill_simt_kernel(const __grid_constant__ LayerArgs L, const _
         const float c = (m == -INFINITY) ? 0.f : exp2f(m - mn);
         const float pj = exp2f(x - mn);
         l = l * c + pj;
-        const T *vr = reinterpret_cast<const T *>(a.v) + (((size_t)b * a.S + j) * L.Hkv + kvh) * L.Dv;
+        const T *vr = reinterpret_cast<const T *>(a.v) + (((size_t)b * a.v_rows + j) * L.Hkv + kvh) * L.Dv;
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
             const int e = lane + 32 * t;
@@ -255,6 +262,20 @@ cudaError_t launch_kprep(const KprepArgs &a, int dtype, cudaStream_t stream)
         kprep_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, stream>>>(a);
     else
         kprep_kernel<float><<<(unsigned)blocks, threads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rope_table(const RopeArgs &rope, float2 *table, long long n, cudaStream_t stream)
+{
+    if (rope.half == 0 || n == 0)
+        return cudaSuccess;
+    KprepArgs a;
+    memset(&a, 0, sizeof(a));
+    a.S = (int)n;
+    a.rope_table = table;
+    a.rope = rope;
+    const long long tb = (n * rope.half + 255) / 256;
+    rope_table_kernel<<<(unsigned)(tb < 4096 ? tb : 4096), 256, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -75,10 +75,13 @@ struct SwaParams {
     CUtensorMap tm_v;  // [B, S, Hkv, Dv]    box {64, 1, 16, 1}
     __nv_bfloat16 *out;
     int out_v8;                // out is 32-byte aligned: 256-bit stores
-    const float2 *rope_table;  // [S][half] (cos, sin) of each token's position
+    const float2 *rope_table;  // row (past + i): (cos, sin) of the pairs at query i's position
     const float *sinks;
+    const int *past_lens;      // [B] cached tokens before the chunk, or nullptr
     unsigned *err;
     int S, Hq, Hkv, G, gp, P, window;
+    int key_off;               // key index of query 0 (a multiple of 16; 0 for a plain prefill)
+    int max_past;
     int num_p_tiles, num_g_tiles, num_tiles, tiles_per_cta;
     int rope_half;
     float scale_log2;
@@ -118,9 +121,9 @@ __device__ __forceinline__ Tile tile_at(const SwaParams &p, int t)
     c.b = bk / p.Hkv;
     c.h0 = c.kvh * p.G + gt * p.gp;
     c.p0 = pt * p.P;
-    const int k_lo = c.p0 - p.window + 1;
+    const int k_lo = c.p0 + p.key_off - p.window + 1;
     c.first_block = k_lo > 0 ? k_lo / kKeyBlock : 0;
-    c.last_block = (c.p0 + p.P - 1) / kKeyBlock;
+    c.last_block = (c.p0 + p.key_off + p.P - 1) / kKeyBlock;
     return c;
 }
 
@@ -267,8 +270,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
         // is ready. Both walk every tile with the producer's ring cursor to
         // number the entries. An entry is free (its kv_empty barrier counts
         // two arrivals) once each issuer has committed it: issuer t commits the
-        // entries below the span of its next tile after the PV of its current
-        // one, and every remaining entry after its last tile.
+        // entries below the span of a tile before waiting for it and below the
+        // span of its next tile after the PV of its current one, and every
+        // remaining entry after its last tile. As a tile spans at most 9 of
+        // the 12 entries, every entry the producer waits on is then committed
+        // by an issuer that is not waiting on that producer.
         const int t = warp - 9;
         if (lane == 0 && t < n_local) {
             const uint32_t idesc_pv = idesc_bf16_f32(kBlockM, kDv, false, true);
@@ -313,6 +319,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
             walk_to(t);
             for (int n = t; ok && n < n_local; n += 2) {
                 const uint32_t ph = (uint32_t)(n >> 1) & 1u;
+                // Entries below this tile's span are never read by this issuer
+                // again: commit them before waiting, so that the ring can refill
+                // while this tile's blocks are still missing (otherwise two
+                // tiles of 9 blocks from different runs, one per issuer, could
+                // wait on each other's 12-entry ring).
+                for (; freed < e0; ++freed)
+                    umma_commit(&bars->kv_empty[freed % kRing]);
                 wait(&bars->o_free[t], ph ^ 1u);  // epilogue of tile n - 2 has read O
                 wait(&bars->q_ready[t], ph);
                 // Only this tile's entries: those below e0 may already be
@@ -370,6 +383,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
             const Tile c = tile_at(p, t_begin + n);
             const int i = c.p0 + row / p.gp;
             const int h = c.h0 + row % p.gp;
+            // cached tokens before this chunk (0 for a plain prefill): query i
+            // has position past + i; key rows below key_off - past precede
+            // position 0 and are never visible
+            const int past = p.past_lens != nullptr ? min(max(__ldg(p.past_lens + c.b), 0), p.max_past) : 0;
             // ---- partial RoPE of this row of Q_n (buffer t)
             // With 16 positions per tile and 32 pairs (the MiMo layer), the
             // tile's 4 KB slice of the RoPE table is copied into shared memory
@@ -378,9 +395,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
             const bool fast_rope = half == 32 && p.P == 16;
             const float4 *tab_row = reinterpret_cast<const float4 *>(sTab + t * kTabBytes) + (row >> 3) * 16;
             if (fast_rope) {
-                const int pos = c.p0 + (row >> 3);
-                const bool in = pos < p.S;
-                const float2 *src = p.rope_table + (size_t)(in ? pos : 0) * 32 + (row & 7) * 4;
+                const int qi = c.p0 + (row >> 3);
+                const bool in = qi < p.S;
+                const float2 *src = p.rope_table + (size_t)(past + (in ? qi : 0)) * 32 + (row & 7) * 4;
                 uint8_t *dst = sTab + t * kTabBytes + (row >> 3) * 256 + (row & 7) * 32;
                 cp_async16(dst, src, in ? 16u : 0u);
                 cp_async16(dst + 16, src + 2, in ? 16u : 0u);
@@ -393,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
             }
             if (i < p.S && half > 0) {
                 uint8_t *q_row = sQ + t * kQBytes + row * 128;
-                const float2 *cs = p.rope_table + (size_t)i * half;
+                const float2 *cs = p.rope_table + (size_t)(past + i) * half;
                 if (fast_rope && i < p.S) {
                     // One 128-byte swizzled row: chunks 0-3 hold dims 0-31, 4-7 dims 32-63.
                     uint4 v[8];
@@ -438,8 +455,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
 
             // ---- softmax over the tile's key span
             const int k0 = c.first_block * kKeyBlock;
-            const int lo = i - p.window + 1 - k0;      // first visible column
-            const unsigned span = (unsigned)(p.window - 1);  // column c visible iff c - lo <= span
+            const int hi = i + p.key_off - k0;  // the row's own key column
+            const int lo = max(hi - p.window + 1, max(p.key_off - past, 0) - k0);  // first visible column
+            const unsigned span = (unsigned)(hi - lo);  // column c visible iff c - lo <= span
             if (!mbar_wait(&bars->s_full[t], ph, abort_flag, p.err)) {
                 ok = false;
                 break;
@@ -574,15 +592,18 @@ cudaError_t launch_prefill_swa(const LayerArgs &L, const PrefillArgs &a, const f
     const int gp = swa_heads_per_tile(L);
     const int P = kBlockM / gp;
     if (!make_bf16_map_4d(&p.tm_q, a.q, kDqk, L.Hq, a.S, a.S, a.B, 64, gp, P) ||
-        !make_bf16_map_4d(&p.tm_k, a.krot, kDqk, L.Hkv, a.S, a.krot_rows, a.B, 64, 1, kKeyBlock) ||
-        !make_bf16_map_4d(&p.tm_v, a.v, kDv, L.Hkv, a.S, a.S, a.B, 64, 1, kKeyBlock))
+        !make_bf16_map_4d(&p.tm_k, a.krot, kDqk, L.Hkv, a.key_rows_valid, a.krot_rows, a.B, 64, 1, kKeyBlock) ||
+        !make_bf16_map_4d(&p.tm_v, a.v, kDv, L.Hkv, a.key_rows_valid, a.v_rows, a.B, 64, 1, kKeyBlock))
         return cudaErrorInvalidValue;
     p.out = reinterpret_cast<__nv_bfloat16 *>(a.out);
     p.out_v8 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
     p.rope_table = rope_table;
     p.sinks = L.sinks;
+    p.past_lens = a.past_lens;
     p.err = a.err;
     p.S = a.S;
+    p.key_off = a.past_lens != nullptr ? a.swa_key_off : 0;
+    p.max_past = a.max_past;
     p.Hq = L.Hq;
     p.Hkv = L.Hkv;
     p.G = L.G;

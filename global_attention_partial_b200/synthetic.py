@@ -153,6 +153,21 @@ def decode_inputs(spec: LayerSpec, batch: int, capacity: int, kv_lens: torch.Ten
     return q, k_new, v_new, k_cache, v_cache, sinks
 
 
+def cached_prefill_inputs(spec: LayerSpec, batch: int, seq: int, capacity: int, *, seed: int, layer: int,
+                          dtype=torch.bfloat16, device="cpu"):
+    """(q, k, v, k_cache, v_cache, sinks) for a chunk of `seq` tokens that
+    continues a cache: the chunk as prefill_inputs draws it, and caches of
+    N(0,1) values taken as already-rotated keys (a ring of `window` slots on a
+    sliding layer)."""
+    q, k, v, sinks = prefill_inputs(spec, batch, seq, seed=seed, layer=layer, dtype=dtype, device=device)
+    cap = spec.window if spec.layer_type == 1 else capacity
+    k_cache = normal((batch, cap, spec.num_kv_heads, spec.qk_dim), seed=seed,
+                     tensor_id=tensor_id(layer, ROLE_KCACHE), dtype=dtype, device=device)
+    v_cache = normal((batch, cap, spec.num_kv_heads, spec.v_dim), seed=seed,
+                     tensor_id=tensor_id(layer, ROLE_VCACHE), dtype=dtype, device=device)
+    return q, k, v, k_cache, v_cache, sinks
+
+
 def decode_kv_lens(batch: int, lo: int, hi: int, *, seed: int) -> torch.Tensor:
     """KV lengths (counting the new token) uniform in [lo, hi], int32 on the CPU."""
     return uniform_int(batch, lo, hi, seed=seed, tensor_id=tensor_id(255, ROLE_LENS))

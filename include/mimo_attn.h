@@ -121,6 +121,46 @@ MIMO_ATTN_API mimo_attn_status mimo_attn_prefill(const mimo_attn_layer *layer, i
                                    void *k_cache, void *v_cache, int cache_capacity,
                                    void *workspace, size_t workspace_bytes, void *stream);
 
+/* Bytes of workspace mimo_attn_prefill_cached needs: the RoPE table of
+ * positions 0 .. max_past_len + seq - 1 and, on SWA, the per-sequence key and
+ * value windows [batch, round_up(window - 1, 16) + seq, Hkv, D]. 0 on a bad
+ * layer or negative sizes. */
+MIMO_ATTN_API size_t mimo_attn_prefill_cached_workspace_size(const mimo_attn_layer *layer, int dtype,
+                                                             int batch, int seq, int max_past_len);
+
+/* Prefill continuing a cache (chunked prefill): a chunk of seq new tokens per
+ * sequence after past_lens[b] tokens that are already in the caches. This is
+ * the cache-aware prefill of the rotating cache (lablup/mlxcel issue 842,
+ * "Implementation plan"; the attention itself as in mimo_attn_prefill).
+ *   q [batch, seq, Hq, Dqk], k [batch, seq, Hkv, Dqk], v [batch, seq, Hkv, Dv]:
+ *              the chunk, unrotated; token t of sequence b has position
+ *              past_lens[b] + t (RoPE and mask).
+ *   past_lens: device int32 [batch], 0 <= past_lens[b] <= max_past_len.
+ *   max_past_len: host bound of past_lens (sizes the RoPE table).
+ *   out [batch, seq, Hq, Dv]: token t attends every cached key and the
+ *              chunk's keys up to itself (GLOBAL: positions <= its own; SWA:
+ *              the last `window` positions including its own), sink on SWA.
+ *   k_cache, v_cache (required; hold rotated keys, as decode and prefill
+ *              leave them): GLOBAL linear [batch, cache_capacity, Hkv, D]
+ *              with cache_capacity >= max_past_len + seq, position p in slot
+ *              p; SWA ring [batch, window, Hkv, D], cache_capacity == window,
+ *              position p in slot p mod window. On return the chunk's rotated
+ *              keys and values are in their slots (on SWA the chunk's last
+ *              `window` tokens).
+ *   workspace: at least mimo_attn_prefill_cached_workspace_size() bytes,
+ *              256-byte aligned.
+ * Errors: as mimo_attn_prefill, plus MIMO_ATTN_ERR_INVALID_ARG for null
+ * past_lens or caches, max_past_len < 0 or a cache capacity that breaks the
+ * rules above. past_lens[b] outside [0, max_past_len] (or, on GLOBAL, beyond
+ * the capacity) is caught on the device: MIMO_ATTN_DEVERR_KV_LEN is set in the
+ * device error word and that sequence's cache rows are not written (its
+ * outputs are undefined). */
+MIMO_ATTN_API mimo_attn_status mimo_attn_prefill_cached(const mimo_attn_layer *layer, int dtype, int batch,
+                                                        int seq, const void *q, const void *k, const void *v,
+                                                        const int32_t *past_lens, int max_past_len, void *out,
+                                                        void *k_cache, void *v_cache, int cache_capacity,
+                                                        void *workspace, size_t workspace_bytes, void *stream);
+
 /* Bytes of workspace mimo_attn_decode needs (split-KV partial results) for
  * this layer, batch and cache capacity. */
 MIMO_ATTN_API size_t mimo_attn_decode_workspace_size(const mimo_attn_layer *layer, int dtype, int batch,

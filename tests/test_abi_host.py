@@ -173,3 +173,47 @@ def test_layer_selection_from_config(lib):
             assert (l.layer_type, l.num_kv_heads, l.rope_theta) == (mimo.GLOBAL, 4, 5e6)
             assert l.sinks is None
         assert l.rotary_dim == 64 and l.qk_dim == 192 and l.v_dim == 128
+
+
+def cached_status(l, batch=2, seq=16, max_past=100, cap=None, ws_bytes=1 << 30, past=True, caches=True):
+    if cap is None:
+        cap = l.window if l.layer_type == mimo.SWA else max_past + seq
+    return mimo.mimo_attn_prefill_cached(l, mimo.BF16, batch, seq, T(), T(), T(), T() if past else None, max_past,
+                                         T(), T() if caches else None, T() if caches else None, cap, T(),
+                                         ws_bytes, 0)
+
+
+def test_prefill_cached_argument_checks(lib):
+    mimo.mimo_attn_debug_fail_launches(True)
+    try:
+        swa = layer()
+        ga = layer(layer_type=mimo.GLOBAL, num_kv_heads=4)
+        assert cached_status(swa, caches=False) == mimo.ERR_INVALID_ARG      # caches are required
+        assert cached_status(swa, cap=64) == mimo.ERR_INVALID_ARG            # ring must equal the window
+        assert cached_status(ga, cap=100 + 16 - 1) == mimo.ERR_INVALID_ARG   # cap < max_past + seq
+        assert cached_status(ga, max_past=-1, cap=16) == mimo.ERR_INVALID_ARG
+        assert cached_status(ga, past=False) == mimo.ERR_INVALID_ARG
+        assert cached_status(ga, batch=0) == mimo.OK                         # empty problems are no-ops
+        assert cached_status(swa, seq=0) == mimo.OK
+        assert cached_status(ga, ws_bytes=10) == mimo.ERR_WORKSPACE
+        assert cached_status(ga) == mimo.ERR_CUDA                            # reaches the launch step
+        assert cached_status(swa) == mimo.ERR_CUDA
+    finally:
+        mimo.mimo_attn_debug_fail_launches(False)
+
+
+def test_prefill_cached_workspace_sizes(lib):
+    ga = layer(layer_type=mimo.GLOBAL, num_kv_heads=4)
+    # global: only the RoPE table of positions 0 .. max_past + seq - 1
+    assert mimo.mimo_attn_prefill_cached_workspace_size(ga, mimo.BF16, 4, 4096, 28672) == (28672 + 4096) * 32 * 8
+    # sliding: the table, then key and value windows of round_up(W - 1, 16) + seq rows
+    swa = layer()
+    rows = 2 * (128 + 100) * 8
+    want = 256 * math.ceil((50 + 100) * 32 * 8 / 256) + 256 * math.ceil(rows * 192 * 2 / 256) + \
+        256 * math.ceil(rows * 128 * 2 / 256)
+    assert mimo.mimo_attn_prefill_cached_workspace_size(swa, mimo.BF16, 2, 100, 50) == want
+    w17 = layer(window=17)  # key offset round_up(16, 16) = 16
+    rows = 1 * (16 + 10) * 8
+    assert mimo.mimo_attn_prefill_cached_workspace_size(w17, mimo.FP32, 1, 10, 0) == \
+        256 * math.ceil(10 * 32 * 8 / 256) + 256 * math.ceil(rows * 192 * 4 / 256) + 256 * math.ceil(rows * 128 * 4 / 256)
+    assert mimo.mimo_attn_prefill_cached_workspace_size(ga, mimo.BF16, 1, 8, -1) == 0
