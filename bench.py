@@ -71,6 +71,16 @@ def prefill_flops(spec, B: int, S: int) -> float:
     return float(B) * spec.num_q_heads * visible_pairs(spec, S) * 2 * (spec.qk_dim + spec.v_dim)
 
 
+def chunk_flops(spec, B: int, S: int, past: int) -> float:
+    """FLOPs of a chunk of S tokens after `past` cached ones: token t sees
+    past + t + 1 keys (global) or min(past + t + 1, W) (sliding)."""
+    if spec.layer_type == 0:
+        pairs = S * past + S * (S + 1) // 2
+    else:
+        pairs = sum(min(past + t + 1, spec.window) for t in range(S))
+    return float(B) * spec.num_q_heads * pairs * 2 * (spec.qk_dim + spec.v_dim)
+
+
 def prefill_bytes(spec, B: int, S: int) -> float:
     """Compulsory HBM bytes of one prefill layer: read Q, K, V, write O."""
     e = 2
@@ -158,6 +168,9 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# chunked prefill workload: the hybrid stack's last CHUNK_SEQ tokens after CHUNK_PAST cached ones
+CHUNK_PAST, CHUNK_SEQ = 28672, 4096
+
 # ------------------------------------------------------------------ workload
 class StackWorkload:
     """Device-resident inputs, outputs, caches and workspaces of the step."""
@@ -175,6 +188,7 @@ class StackWorkload:
             pw = synthetic.GLOBAL_PREFILL
         self.do_prefill = kind in ("stack", "swa", "global")
         self.do_decode = kind in ("stack", "decode")
+        self.do_chunked = kind == "chunked"
         self.pw, self.dw = pw, dw
         self.prefill_layers = []
         if self.do_prefill:
@@ -190,6 +204,23 @@ class StackWorkload:
                 ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
                 self.prefill_layers.append(dict(spec=spec, lay=lay, q=q, k=k, v=v, sinks=sinks, out=out, ws=ws,
                                                 need=need))
+        # chunked: the stack's last 4096 tokens as a chunk after 28672 cached ones
+        self.chunk_layers = []
+        self.chunk_past, self.chunk_seq = CHUNK_PAST, CHUNK_SEQ
+        if self.do_chunked:
+            B, S, P = pw.batch, CHUNK_SEQ, CHUNK_PAST
+            self.past_dev = torch.full((B,), P, dtype=torch.int32, device=dev)
+            for li, spec in enumerate(pw.layers):
+                q, k, v, kc, vc, sinks = synthetic.cached_prefill_inputs(spec, B, S, P + S, seed=seed, layer=li,
+                                                                         device=dev)
+                sinks = sinks if spec.layer_type == 1 else None
+                lay = mimo.make_layer(spec.layer_type, spec.num_q_heads, spec.num_kv_heads, spec.qk_dim,
+                                      spec.v_dim, spec.rotary_dim, spec.window, spec.theta,
+                                      spec.hidden_size, sinks)
+                out = torch.empty((B, S, spec.num_q_heads, spec.v_dim), dtype=torch.bfloat16, device=dev)
+                need = mimo.mimo_attn_prefill_cached_workspace_size(lay, mimo.BF16, B, S, P)
+                ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+                self.chunk_layers.append(dict(spec=spec, lay=lay, q=q, k=k, v=v, kc=kc, vc=vc, out=out, ws=ws))
         self.decode_layers = []
         if self.do_decode:
             B = dw.batch
@@ -216,11 +247,24 @@ class StackWorkload:
     def decode_flops(self):
         return sum(decode_flops(L["spec"], self.lens) for L in self.decode_layers)
 
+    def chunk_flops(self):
+        return sum(chunk_flops(L["spec"], self.pw.batch, self.chunk_seq, self.chunk_past) for L in self.chunk_layers)
+
+    def run_chunk_layer(self, L, stream):
+        m = self.mimo
+        st = m.mimo_attn_prefill_cached(L["lay"], m.BF16, self.pw.batch, self.chunk_seq, L["q"], L["k"], L["v"],
+                                        self.past_dev, self.chunk_past, L["out"], L["kc"], L["vc"],
+                                        L["kc"].shape[1], L["ws"], L["ws"].numel(), stream)
+        if st != m.OK:
+            raise m.MimoAttnError(st, "mimo_attn_prefill_cached")
+
     def decode_bytes(self):
         return sum(decode_bytes(L["spec"], self.lens) for L in self.decode_layers)
 
     def launches_per_step(self):
         n = 3 * len(self.prefill_layers)  # RoPE table + K-prep + attention
+        for L in self.chunk_layers:  # RoPE table + cache prep (1 global, 2 sliding) + attention
+            n += 3 if L["spec"].layer_type == 0 else 4
         for L in self.decode_layers:
             n += 2 if L["need"] > 0 else 1  # split kernel (+ combine)
         return n
@@ -281,6 +325,17 @@ class StackWorkload:
                 events.setdefault(kind, []).append((e0, e1))
             else:
                 self.run_prefill_layer(L, stream)
+        for L in self.chunk_layers:
+            kind = "chunk_global" if L["spec"].layer_type == 0 else "chunk_swa"
+            if events is not None:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                self.run_chunk_layer(L, stream)
+                e1.record(stream)
+                events.setdefault(kind, []).append((e0, e1))
+            else:
+                self.run_chunk_layer(L, stream)
         if self.decode_layers:
             if events is not None:
                 e0 = torch.cuda.Event(enable_timing=True)
@@ -474,7 +529,9 @@ def run_reference(args):
 def workload_config(args, reference=False):
     names = {"stack": f"{synthetic.HYBRID_PREFILL.name} + {synthetic.HYBRID_DECODE.name}",
              "swa": synthetic.SWA_PREFILL.name, "global": synthetic.GLOBAL_PREFILL.name,
-             "decode": synthetic.HYBRID_DECODE.name}
+             "decode": synthetic.HYBRID_DECODE.name,
+             "chunked": f"hybrid 8-layer stack, chunk of {CHUNK_SEQ} tokens after {CHUNK_PAST} cached, bf16 B4 "
+                        f"pattern 0,1,1,1,1,1,0,1"}
     cfg = {"workload": names[args.workload], "prefill_batch": synthetic.HYBRID_PREFILL.batch,
            "prefill_seq": synthetic.HYBRID_PREFILL.seq, "decode_batch": synthetic.HYBRID_DECODE.batch,
            "kv_len_range": list(synthetic.HYBRID_DECODE.kv_len_range), "layers": "0,1,1,1,1,1,0,1",
@@ -494,12 +551,15 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["stack", "swa", "global", "decode"], default="stack")
+    ap.add_argument("--workload", choices=["stack", "swa", "global", "decode", "chunked"], default="stack")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the decode layers one call at a time")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
+    if args.workload == "chunked":  # a NEXT-row measurement: kernels only, no host-buffer or oracle legs
+        args.no_e2e = True
+        args.no_cpu_baseline = True
     if args.impl == "reference":
         run_reference(args)
         return
@@ -548,7 +608,8 @@ def main():
     kinds = {k: [a.elapsed_time(b) for a, b in v] for k, v in events.items()}
     pflops = w.prefill_flops() if w.do_prefill else 0.0
     dflops = w.decode_flops() if w.do_decode else 0.0
-    step_flops = pflops + dflops
+    cflops = w.chunk_flops() if w.do_chunked else 0.0
+    step_flops = pflops + dflops + cflops
     value = job_value(world, step_flops, ms)
 
     parts = {}
@@ -586,6 +647,18 @@ def main():
                         "frac": ach / peaks["hbm_gbs"],
                         "traffic": committed_traffic("prefill_swa_sliding", "prefill_swa.cu"),
                         "kernel": "prefill_swa_kernel (sliding layer)", "peak_kind": f"HBM copy, {peaks['source']}"}
+    if w.do_chunked:
+        for kind, lt in (("chunk_global", 0), ("chunk_swa", 1)):
+            specs = [L["spec"] for L in w.chunk_layers if L["spec"].layer_type == lt]
+            per = statistics.mean(kinds[kind])
+            f = chunk_flops(specs[0], w.pw.batch, w.chunk_seq, w.chunk_past)
+            parts[kind + "_layer"] = {"ms_per_launch": per, "tflops": f / (per * 1e-3) / 1e12,
+                                      "frac_of_tensor_peak": f / (per * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]}
+        ach = parts["chunk_global_layer"]["tflops"]
+        roofline = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                    "frac": ach / peaks["bf16_tflops_sustained"], "traffic": None,
+                    "kernel": "prefill_ga_kernel (global layer, chunk of 4096 after 28672 cached, B4)",
+                    "peak_kind": f"bf16 dense, sustained, {peaks['source']}"}
     if w.do_decode:
         per = statistics.mean(kinds["decode_stack"])
         byt = w.decode_bytes()
