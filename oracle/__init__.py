@@ -245,3 +245,80 @@ def prefill_cached_layer(q, k, v, k_cache, v_cache, past_lens, *, layer_type: in
             slot = p if layer_type == GLOBAL else p % window
             kc[b, slot], vc[b, slot] = K[p], V[p]
     return out, kc, vc
+
+
+# ------------------------------------------------------ fp8 (e4m3) KV cache
+# The OCP 8-bit floating point format E4M3 ("OCP 8-bit Floating Point
+# Specification", FP8 E4M3): 1 sign bit, 4 exponent bits (bias 7), 3 mantissa
+# bits; exponent field 0 holds the subnormals m * 2^-9; S.1111.111 is NaN and
+# there is no infinity, so the largest finite magnitude is 1.75 * 2^8 = 448.
+# The cache stores code c for a value x as c = e4m3(x / scale) (round to
+# nearest, ties to even mantissa, saturating at +-448) and reads scale *
+# e4m3_value(c). A reading: the pages only mention "one quant" for this
+# model, without a format or a scale granularity; per-tensor scales with
+# saturation are the plainest choice.
+
+def e4m3_value(code) -> np.ndarray:
+    """Value of each E4M3 code (uint8 array-like), NaN for the two NaN codes."""
+    c = np.asarray(code, dtype=np.int64)
+    s = np.where((c >> 7) & 1, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 7
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.power(2.0, e - 7.0))
+    nan = (e == 15) & (m == 7)
+    return np.where(nan, np.nan, s * mag)
+
+
+_E4M3_POS = e4m3_value(np.arange(0, 127))  # the 127 non-negative finite codes 0x00..0x7E, increasing
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Nearest E4M3 code of each finite x (round to nearest, ties to the code
+    with an even mantissa, |x| > 448 saturating to +-448)."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), 448.0)
+    d = np.abs(a[..., None] - _E4M3_POS)  # distance to every non-negative code
+    best = np.argmin(d, axis=-1)
+    # ties: argmin takes the lower code; move to the upper one when it is
+    # equally near and has the even mantissa
+    upper = np.minimum(best + 1, 126)
+    du = np.take_along_axis(d, upper[..., None], axis=-1)[..., 0]
+    db = np.take_along_axis(d, best[..., None], axis=-1)[..., 0]
+    pick_upper = (du == db) & (upper != best) & ((upper & 1) == 0)
+    code = np.where(pick_upper, upper, best)
+    return np.where(np.signbit(x), code | 0x80, code).astype(np.uint8)
+
+
+def decode_fp8kv(q, k_new, v_new, k_codes, v_codes, L: int, rotary_dim: int, theta: float, layer_type: int,
+                 window: int, softmax_scale: float, sinks, vscale: float, k_scale: float, v_scale: float):
+    """One decode step of one (batch, KV head) over an E4M3 cache. q [n_q, Dqk],
+    k_new [Dqk], v_new [Dv] unrotated; k_codes [cap, Dqk], v_codes [cap, Dv]
+    uint8. The new token's rotated key and its value are quantized into their
+    slot first (as the cache keeps them); the query then attends the cache's
+    values (scale * code value) over its visible positions, exactly as
+    decode() does for a bf16 cache. Returns (out [n_q, Dv], k_codes', v_codes')."""
+    q = _f64(q)
+    if q.ndim == 1:
+        q = q[None, :]
+    kc = np.array(k_codes, dtype=np.uint8, copy=True)
+    vc = np.array(v_codes, dtype=np.uint8, copy=True)
+    cap = kc.shape[0]
+    if L < 1 or (layer_type == GLOBAL and L > cap) or (layer_type == SWA and cap != window):
+        raise ValueError("decode_fp8kv: bad length or capacity")
+    pos = float(L - 1)
+    slot = (L - 1) % window if layer_type == SWA else L - 1
+    kc[slot] = e4m3_encode(rope(_f64(k_new)[None, :], rotary_dim, theta, [pos])[0] / k_scale)
+    vc[slot] = e4m3_encode(_f64(v_new) / v_scale)
+    K = np.zeros((L, kc.shape[1]))
+    V = np.zeros((L, vc.shape[1]))
+    lo = max(0, L - window) if layer_type == SWA else 0
+    for p in range(lo, L):
+        sl = p % window if layer_type == SWA else p
+        K[p] = k_scale * e4m3_value(kc[sl])
+        V[p] = v_scale * e4m3_value(vc[sl])
+    q_rot = rope(q, rotary_dim, theta, np.full(q.shape[0], pos))
+    out = np.empty((q.shape[0], V.shape[1]))
+    for r in range(q.shape[0]):
+        s = None if sinks is None else float(np.asarray(sinks)[r])
+        out[r] = prefill_rows(q_rot[r:r + 1], [L - 1], K, V, layer_type, window, softmax_scale, s, vscale)[0]
+    return out, kc, vc

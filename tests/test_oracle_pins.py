@@ -395,3 +395,54 @@ def test_one_token_chunk_equals_decode(layer_type, W, P):
         np.testing.assert_allclose(out[0, 0, hs], o, rtol=0, atol=1e-13)
         np.testing.assert_allclose(kc2[0, :, kv], kcd, rtol=0, atol=1e-14)
         np.testing.assert_allclose(vc2[0, :, kv], vcd, rtol=0, atol=0)
+
+
+# ------------------------------------------------------------- fp8 KV cache
+
+def test_e4m3_values_closed_forms():
+    """Codes of the OCP E4M3 definition: largest finite 448 (0x7E), smallest
+    normal 2^-6 (0x08), smallest subnormal 2^-9 (0x01), 1.0 (0x38), sign bit,
+    and the two NaN codes. Catches a wrong bias or subnormal scale."""
+    v = oracle.e4m3_value(np.arange(256))
+    assert v[0x7E] == 448.0 and v[0x08] == 2.0 ** -6 and v[0x01] == 2.0 ** -9 and v[0x07] == 7 * 2.0 ** -9
+    assert v[0x38] == 1.0 and v[0x39] == 1.125 and v[0xB8] == -1.0 and v[0x00] == 0.0
+    assert np.isnan(v[0x7F]) and np.isnan(v[0xFF]) and np.isfinite(np.delete(v, [0x7F, 0xFF])).all()
+    pos = v[:127]
+    assert np.all(np.diff(pos) > 0)  # codes 0x00..0x7E increase
+
+
+def test_e4m3_encode_round_trip_ties_and_saturation():
+    """Every finite code round-trips; halfway values go to the even mantissa;
+    magnitudes beyond 448 saturate; values between codes go to the nearer."""
+    v = oracle.e4m3_value(np.arange(256))
+    finite = [c for c in range(256) if not np.isnan(v[c])]
+    assert np.array_equal(oracle.e4m3_encode(v[finite]), np.array(finite, dtype=np.uint8))
+    assert list(oracle.e4m3_encode([1.0625, 1.1875, 1.9375, 2.0 ** -10, 3 * 2.0 ** -11])) == [0x38, 0x3A, 0x40, 0x00, 0x01]
+    assert list(oracle.e4m3_encode([448.0, 465.0, 1e6, -1e6])) == [0x7E, 0x7E, 0x7E, 0xFE]
+    x = RNG.uniform(-400, 400, 2000)
+    got = oracle.e4m3_value(oracle.e4m3_encode(x))
+    nearest = np.array([v[finite][np.argmin(np.abs(v[finite] - xi))] for xi in x])
+    np.testing.assert_array_equal(np.abs(got - x), np.abs(nearest - x))
+
+
+@pytest.mark.parametrize("layer_type,L,W", [(0, 1, 0), (0, 40, 0), (1, 3, 8), (1, 30, 8)])
+def test_fp8_decode_equals_bf16_decode_on_representable_values(layer_type, L, W):
+    """When every cached value and the new token's rotated key and value are
+    exactly scale * (an E4M3 value), the fp8 path is the plain decode: same
+    output, and the codes written decode to the values decode() stores."""
+    Hq, D, Dv, r, theta = 2, 16, 8, 0, 1e4  # r = 0: the new key needs no rotation to stay representable
+    ks, vs = 0.5, 2.0
+    v = oracle.e4m3_value(np.arange(0, 0x7E))
+    cap = W if layer_type == 1 else L + 2
+    kc_codes = RNG.integers(0, 0x70, (cap, D)).astype(np.uint8)
+    vc_codes = RNG.integers(0, 0x70, (cap, Dv)).astype(np.uint8)
+    kn = ks * RNG.choice(v[:0x70], D) * RNG.choice([-1, 1], D)
+    vn = vs * RNG.choice(v[:0x70], Dv) * RNG.choice([-1, 1], Dv)
+    q = rnd(Hq, D)
+    sinks = rnd(Hq) if layer_type == 1 else None
+    args = (L, r, theta, layer_type, W, 1 / math.sqrt(D), sinks, 0.7)
+    o8, kc2, vc2 = oracle.decode_fp8kv(q, kn, vn, kc_codes, vc_codes, *args, ks, vs)
+    o16, kc16, vc16 = oracle.decode(q, kn, vn, ks * oracle.e4m3_value(kc_codes), vs * oracle.e4m3_value(vc_codes), *args)
+    np.testing.assert_allclose(o8, o16, rtol=0, atol=1e-13)
+    np.testing.assert_array_equal(ks * oracle.e4m3_value(kc2), kc16)
+    np.testing.assert_array_equal(vs * oracle.e4m3_value(vc2), vc16)
