@@ -1,7 +1,7 @@
 """Benchmark of the MiMo-V2-Flash hybrid attention path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload stack|swa|global|decode] [--no-e2e] [--no-cpu-baseline]
+                    [--workload stack|swa|global|decode|chunked|decode_fp8] [--no-e2e] [--no-cpu-baseline]
 
 One step = one pass of the whole hot path over the hybrid 8-layer attention
 stack (hybrid_layer_pattern 0,1,1,1,1,1,0,1: 6 sliding-window layers with
@@ -96,15 +96,17 @@ def decode_flops(spec, lens) -> float:
     return float(sum(decode_visible(spec, lens))) * spec.num_q_heads * 2 * (spec.qk_dim + spec.v_dim)
 
 
-def decode_bytes(spec, lens) -> float:
+def decode_bytes(spec, lens, cache_elem: int = 2) -> float:
     """Algorithmic HBM bytes of one decode layer: the visible cache K/V, the
-    new q/k/v, the new token's cache write, the output and the sinks."""
+    new q/k/v, the new token's cache write, the output and the sinks.
+    cache_elem: bytes per cached element (2 bf16, 1 fp8)."""
     e = 2
     B = len(lens)
-    kv_row = spec.num_kv_heads * (spec.qk_dim + spec.v_dim) * e
+    kv_elems = spec.num_kv_heads * (spec.qk_dim + spec.v_dim)
+    kv_row = kv_elems * cache_elem
     cache_read = sum(decode_visible(spec, lens)) * kv_row
     q_read = B * spec.num_q_heads * spec.qk_dim * e
-    new_rw = 2 * B * kv_row
+    new_rw = B * kv_elems * e + B * kv_row
     out_w = B * spec.num_q_heads * spec.v_dim * e
     sinks = spec.num_q_heads * 4 if spec.has_sink else 0
     return float(cache_read + q_read + new_rw + out_w + sinks)
@@ -187,7 +189,9 @@ class StackWorkload:
         elif kind == "global":
             pw = synthetic.GLOBAL_PREFILL
         self.do_prefill = kind in ("stack", "swa", "global")
-        self.do_decode = kind in ("stack", "decode")
+        self.do_decode = kind in ("stack", "decode", "decode_fp8")
+        self.fp8 = kind == "decode_fp8"
+        self.k_scale, self.v_scale = 1.0 / 16, 1.0 / 32
         self.do_chunked = kind == "chunked"
         self.pw, self.dw = pw, dw
         self.prefill_layers = []
@@ -234,6 +238,10 @@ class StackWorkload:
                                       spec.v_dim, spec.rotary_dim, spec.window, spec.theta,
                                       spec.hidden_size, sinks)
                 cap = kc.shape[1]
+                if self.fp8:  # E4M3 caches: the same N(0,1) values quantized with per-tensor scales
+                    kc = mimo.quantize_fp8(kc, self.k_scale)
+                    vc = mimo.quantize_fp8(vc, self.v_scale)
+                    torch.cuda.synchronize()
                 out = torch.empty((B, spec.num_q_heads, spec.v_dim), dtype=torch.bfloat16, device=dev)
                 need = mimo.mimo_attn_decode_workspace_size(lay, mimo.BF16, B, cap)
                 ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
@@ -259,7 +267,7 @@ class StackWorkload:
             raise m.MimoAttnError(st, "mimo_attn_prefill_cached")
 
     def decode_bytes(self):
-        return sum(decode_bytes(L["spec"], self.lens) for L in self.decode_layers)
+        return sum(decode_bytes(L["spec"], self.lens, 1 if self.fp8 else 2) for L in self.decode_layers)
 
     def launches_per_step(self):
         n = 3 * len(self.prefill_layers)  # RoPE table + K-prep + attention
@@ -278,6 +286,13 @@ class StackWorkload:
 
     def run_decode_layer(self, L, stream):
         m = self.mimo
+        if self.fp8:
+            st = m.mimo_attn_decode_fp8kv(L["lay"], self.dw.batch, L["q"], L["kn"], L["vn"], L["lens"], L["kc"],
+                                          L["vc"], L["cap"], self.k_scale, self.v_scale, L["out"], L["ws"],
+                                          L["ws"].numel(), stream)
+            if st != m.OK:
+                raise m.MimoAttnError(st, "mimo_attn_decode_fp8kv")
+            return
         st = m.mimo_attn_decode(L["lay"], m.BF16, self.dw.batch, L["q"], L["kn"], L["vn"], L["lens"], L["kc"],
                                 L["vc"], L["cap"], L["out"], L["ws"], L["ws"].numel(), stream)
         if st != m.OK:
@@ -530,6 +545,7 @@ def workload_config(args, reference=False):
     names = {"stack": f"{synthetic.HYBRID_PREFILL.name} + {synthetic.HYBRID_DECODE.name}",
              "swa": synthetic.SWA_PREFILL.name, "global": synthetic.GLOBAL_PREFILL.name,
              "decode": synthetic.HYBRID_DECODE.name,
+             "decode_fp8": synthetic.HYBRID_DECODE.name.replace("bf16", "bf16 q/out, fp8 E4M3 KV cache"),
              "chunked": f"hybrid 8-layer stack, chunk of {CHUNK_SEQ} tokens after {CHUNK_PAST} cached, bf16 B4 "
                         f"pattern 0,1,1,1,1,1,0,1"}
     cfg = {"workload": names[args.workload], "prefill_batch": synthetic.HYBRID_PREFILL.batch,
@@ -537,7 +553,7 @@ def workload_config(args, reference=False):
            "kv_len_range": list(synthetic.HYBRID_DECODE.kv_len_range), "layers": "0,1,1,1,1,1,0,1",
            "parallelism": f"replicas x{args.gpus} (weak, no collective on the data path)",
            "l2": "no flush: each step streams ~60 GB of inputs, far above the 126 MB L2"}
-    if args.workload in ("stack", "decode"):
+    if args.workload in ("stack", "decode", "decode_fp8"):
         cfg["decode_launch"] = ("direct C-ABI calls, one per layer" if args.no_graph else
                                 "the 8 layers' C-ABI calls captured once in a CUDA graph, replayed each step")
     if args.workload != "stack":
@@ -551,13 +567,13 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["stack", "swa", "global", "decode", "chunked"], default="stack")
+    ap.add_argument("--workload", choices=["stack", "swa", "global", "decode", "chunked", "decode_fp8"], default="stack")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the decode layers one call at a time")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
-    if args.workload == "chunked":  # a NEXT-row measurement: kernels only, no host-buffer or oracle legs
+    if args.workload in ("chunked", "decode_fp8"):  # NEXT-row measurements: kernels only, no host or oracle legs
         args.no_e2e = True
         args.no_cpu_baseline = True
     if args.impl == "reference":
@@ -682,7 +698,8 @@ def main():
         if roofline is None:
             ach = byt / (per * 1e-3) / 1e9
             roofline = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                        "frac": ach / peaks["hbm_gbs"], "traffic": None, "kernel": "decode_mma_kernel (8-layer stack)",
+                        "frac": ach / peaks["hbm_gbs"], "traffic": None,
+                        "kernel": "decode_mma_kernel (8-layer stack%s)" % (", fp8 KV cache" if w.fp8 else ""),
                         "peak_kind": f"HBM copy, {peaks['source']}"}
 
     # ---- e2e through the C ABI with host buffers
@@ -720,7 +737,8 @@ def main():
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(args),
+                "vs_baseline": None,
+                "dtype": "e4m3 KV cache, f16 mma, fp32 accumulate" if w.fp8 else "bf16", "data": "synthetic", "config": workload_config(args),
                 "roofline": roofline, "parts": parts, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": w.launches_per_step() * args.steps, "clocks": clocks,
                 "peaks": peaks}

@@ -37,6 +37,9 @@ EXPORTED = (
     "mimo_attn_decode_workspace_size",
     "mimo_attn_decode",
     "mimo_attn_decode_static",
+    "mimo_attn_decode_fp8kv_workspace_size",
+    "mimo_attn_decode_fp8kv",
+    "mimo_attn_quantize_fp8",
     "mimo_attn_get_device_error",
     "mimo_attn_status_string",
     "mimo_attn_debug_fail_launches",
@@ -96,6 +99,13 @@ def load() -> ctypes.CDLL:
     lib.mimo_attn_decode.restype = i32
     lib.mimo_attn_decode_static.argtypes = [lp, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp]
     lib.mimo_attn_decode_static.restype = i32
+    f32 = ctypes.c_float
+    lib.mimo_attn_decode_fp8kv_workspace_size.argtypes = [lp, i32, i32]
+    lib.mimo_attn_decode_fp8kv_workspace_size.restype = sz
+    lib.mimo_attn_decode_fp8kv.argtypes = [lp, i32, vp, vp, vp, vp, vp, vp, i32, f32, f32, vp, vp, sz, vp]
+    lib.mimo_attn_decode_fp8kv.restype = i32
+    lib.mimo_attn_quantize_fp8.argtypes = [vp, vp, sz, f32, vp]
+    lib.mimo_attn_quantize_fp8.restype = i32
     lib.mimo_attn_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     lib.mimo_attn_get_device_error.restype = i32
     lib.mimo_attn_status_string.argtypes = [i32]
@@ -222,6 +232,25 @@ def mimo_attn_decode_static(layer: mimo_attn_layer, dtype: int, batch: int, q, k
         _ptr(k_cache), _ptr(v_cache), int(cache_capacity), _ptr(out), _stream(stream)))
 
 
+def mimo_attn_decode_fp8kv_workspace_size(layer: mimo_attn_layer, batch: int, cache_capacity: int) -> int:
+    return int(load().mimo_attn_decode_fp8kv_workspace_size(ctypes.byref(layer), batch, cache_capacity))
+
+
+def mimo_attn_decode_fp8kv(layer: mimo_attn_layer, batch: int, q, k_new, v_new, kv_lens, k_cache, v_cache,
+                           cache_capacity: int, k_scale: float, v_scale: float, out, workspace=None,
+                           workspace_bytes: int = 0, stream=None) -> int:
+    """Same arguments as the C entry point; tensors in place of pointers
+    (k_cache / v_cache uint8 E4M3 codes)."""
+    return int(load().mimo_attn_decode_fp8kv(
+        ctypes.byref(layer), batch, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(kv_lens), _ptr(k_cache),
+        _ptr(v_cache), int(cache_capacity), float(k_scale), float(v_scale), _ptr(out), _ptr(workspace),
+        int(workspace_bytes), _stream(stream)))
+
+
+def mimo_attn_quantize_fp8(src, dst, n: int, scale: float, stream=None) -> int:
+    return int(load().mimo_attn_quantize_fp8(_ptr(src), _ptr(dst), int(n), float(scale), _stream(stream)))
+
+
 def mimo_attn_get_device_error() -> int:
     bits = ctypes.c_uint32(0)
     st = load().mimo_attn_get_device_error(ctypes.byref(bits))
@@ -300,4 +329,35 @@ def decode(layer: mimo_attn_layer, q: torch.Tensor, k_new: torch.Tensor, v_new: 
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     _check(mimo_attn_decode(layer, dt, B, q, k_new, v_new, kv_lens, k_cache, v_cache, cap, out, workspace,
                             0 if workspace is None else workspace.numel(), stream), "mimo_attn_decode")
+    return out
+
+
+def decode_fp8kv(layer: mimo_attn_layer, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                 kv_lens: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, k_scale: float,
+                 v_scale: float, out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """Runs mimo_attn_decode_fp8kv: bf16 q/k_new/v_new, uint8 E4M3 caches
+    (updated in place), bf16 out."""
+    B = q.shape[0]
+    cap = k_cache.shape[1]
+    if k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8:
+        raise ValueError("fp8 caches are uint8 tensors of E4M3 codes")
+    if out is None:
+        out = torch.empty((B, layer.num_q_heads, layer.v_dim), dtype=q.dtype, device=q.device)
+    need = mimo_attn_decode_fp8kv_workspace_size(layer, B, cap)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check(mimo_attn_decode_fp8kv(layer, B, q, k_new, v_new, kv_lens, k_cache, v_cache, cap, k_scale, v_scale,
+                                  out, workspace, 0 if workspace is None else workspace.numel(), stream),
+           "mimo_attn_decode_fp8kv")
+    return out
+
+
+def quantize_fp8(src: torch.Tensor, scale: float, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """E4M3 codes of src / scale (src bf16 on the GPU), same shape, uint8."""
+    if src.dtype != torch.bfloat16:
+        raise ValueError("quantize_fp8 takes bf16")
+    if out is None:
+        out = torch.empty(src.shape, dtype=torch.uint8, device=src.device)
+    _check(mimo_attn_quantize_fp8(src, out, src.numel(), scale, stream), "mimo_attn_quantize_fp8")
     return out

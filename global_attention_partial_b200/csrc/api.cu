@@ -390,6 +390,7 @@ mimo_attn_status mimo_attn_decode(const mimo_attn_layer *layer, int dtype, int b
         return MIMO_ATTN_ERR_CUDA;
 
     mimo::DecodeArgs da;
+    memset(&da, 0, sizeof(da));
     da.q = q;
     da.k_new = k_new;
     da.v_new = v_new;
@@ -405,6 +406,85 @@ mimo_attn_status mimo_attn_decode(const mimo_attn_layer *layer, int dtype, int b
     da.err = err;
     cudaError_t e = mimo::launch_decode(L, da, dtype, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MIMO_ATTN_OK : MIMO_ATTN_ERR_CUDA;
+}
+
+size_t mimo_attn_decode_fp8kv_workspace_size(const mimo_attn_layer *layer, int batch, int cache_capacity)
+{
+    return mimo_attn_decode_workspace_size(layer, MIMO_ATTN_BF16, batch, cache_capacity);
+}
+
+mimo_attn_status mimo_attn_decode_fp8kv(const mimo_attn_layer *layer, int batch, const void *q, const void *k_new,
+                                        const void *v_new, const int32_t *kv_lens, void *k_cache, void *v_cache,
+                                        int cache_capacity, float k_scale, float v_scale, void *out,
+                                        void *workspace, size_t workspace_bytes, void *stream)
+{
+    mimo::LayerArgs L;
+    mimo_attn_status st = resolve_layer(layer, MIMO_ATTN_BF16, &L);
+    if (st != MIMO_ATTN_OK)
+        return st;
+    if (batch < 0 || cache_capacity < 1)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (L.layer_type == MIMO_ATTN_SWA && cache_capacity != L.window)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (!(k_scale > 0.f) || !(v_scale > 0.f) || !isfinite(k_scale) || !isfinite(v_scale))
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (L.Dqk != 192 || L.Dv != 128 || L.G > 16)
+        return MIMO_ATTN_ERR_UNSUPPORTED;
+    if (batch == 0)
+        return MIMO_ATTN_OK;
+    if (q == nullptr || k_new == nullptr || v_new == nullptr || kv_lens == nullptr || k_cache == nullptr ||
+        v_cache == nullptr || out == nullptr)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (!(aligned16(q) && aligned16(k_new) && aligned16(v_new) && aligned16(k_cache) && aligned16(v_cache) &&
+          aligned16(out)))
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    const size_t need = mimo_attn_decode_fp8kv_workspace_size(layer, batch, cache_capacity);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+        return MIMO_ATTN_ERR_WORKSPACE;
+    if (g_fail_launches)
+        return MIMO_ATTN_ERR_CUDA;
+    unsigned *err = device_error_ptr();
+    if (err == nullptr)
+        return MIMO_ATTN_ERR_CUDA;
+    // a cached value is scale * code value: the key scale multiplies every
+    // score, the value scale the output
+    L.scale_log2 *= k_scale;
+    L.v_scale *= v_scale;
+    mimo::DecodeArgs da;
+    memset(&da, 0, sizeof(da));
+    da.q = q;
+    da.k_new = k_new;
+    da.v_new = v_new;
+    da.kv_lens = kv_lens;
+    da.k_cache = k_cache;
+    da.v_cache = v_cache;
+    da.cap = cache_capacity;
+    da.out = out;
+    da.partial = static_cast<float *>(workspace);
+    da.max_splits = mimo::decode_max_splits(L, MIMO_ATTN_BF16, cache_capacity);
+    da.chunk = mimo::decode_chunk_keys(L, MIMO_ATTN_BF16);
+    da.B = batch;
+    da.err = err;
+    da.fp8_cache = 1;
+    da.k_scale = k_scale;
+    da.v_scale = v_scale;
+    cudaError_t e = mimo::launch_decode(L, da, MIMO_ATTN_BF16, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MIMO_ATTN_OK : MIMO_ATTN_ERR_CUDA;
+}
+
+mimo_attn_status mimo_attn_quantize_fp8(const void *src, void *dst, size_t n, float scale, void *stream)
+{
+    if (!(scale > 0.f) || !isfinite(scale))
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (n == 0)
+        return MIMO_ATTN_OK;
+    if (src == nullptr || dst == nullptr)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (g_fail_launches)
+        return MIMO_ATTN_ERR_CUDA;
+    return mimo::launch_quantize_e4m3(src, dst, n, scale, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MIMO_ATTN_OK
+               : MIMO_ATTN_ERR_CUDA;
 }
 
 mimo_attn_status mimo_attn_get_device_error(uint32_t *bits)

@@ -33,10 +33,40 @@ constexpr int kChunkKeys = 2048;    // keys per split on global layers
 constexpr int kStageElems = kTileKeys * (kKStride + kVStride);
 // Ring depth x CTAs per SM: the bytes in flight per SM, (stages - 1) x 43 KB x
 // CTAs, must cover the HBM latency at full bandwidth.
-template <int ST> struct DecodeCfg {
-    static constexpr int kSmemBytes = (16 * kQStride + ST * kStageElems + kDqk + kDv) * 2;
+// fp8 (E4M3) caches: a tile lands as dense 320-byte rows (K then V), then is
+// widened to f16 into one padded compute tile (e4m3 values are exact in f16).
+constexpr int kLandRow = kDqk + kDv;             // bytes per key
+constexpr int kLandBytes = kTileKeys * kLandRow;  // 20480
+template <int ST, bool F8 = false> struct DecodeCfg {
+    static constexpr int kSmemBytes = F8 ? (16 * kQStride + kStageElems + kDqk + kDv) * 2 + ST * kLandBytes
+                                         : (16 * kQStride + ST * kStageElems + kDqk + kDv) * 2;
     static constexpr int kCtasPerSm = ST <= 2 ? 2 : 1;
 };
+
+// 16-bit operand type of the tensor-core path: bf16 for bf16 caches, f16 for
+// fp8 caches (their e4m3 values, the f16 query and the probabilities).
+template <bool F8> __device__ __forceinline__ uint32_t pack16(float lo, float hi)
+{
+    return F8 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
+}
+template <bool F8> __device__ __forceinline__ void mma16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    if (F8)
+        mma_f16_16816(d, a, b0, b1);
+    else
+        mma_bf16_16816(d, a, b0, b1);
+}
+// 8 bf16 (a 16-byte chunk) as 8 f16.
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v)
+{
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
+        w[i] = pack_f16x2(f.x, f.y);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
 constexpr int kDecodeStages = 2;
 
 struct DecodeSmem {
@@ -46,7 +76,7 @@ struct DecodeSmem {
 // Row stride (floats) of the per-warp O slices of the final merge, which
 // reuse the stage buffers: 4 x 16 rows x 136 floats = 34 KB.
 constexpr int kMergeStride = kDv + 8;
-static_assert(4 * 16 * kMergeStride * 4 <= kStageElems * 2 * 2, "merge slices fit in the stage buffers");
+static_assert(4 * 16 * kMergeStride * 4 <= kStageElems * 2, "merge slices fit in one stage buffer");
 
 __device__ __forceinline__ int visible_count(int layer_type, int Lb, int window)
 {
@@ -58,15 +88,16 @@ __device__ __forceinline__ bool kv_len_ok(int layer_type, int Lb, int cap)
     return Lb >= 1 && (layer_type == 1 || Lb <= cap);
 }
 
-template <int kStages>
-__global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
+template <int kStages, bool kFp8 = false>
+__global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm)
     decode_mma_kernel(const __grid_constant__ LayerArgs L, const __grid_constant__ DecodeArgs a)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     __nv_bfloat16 *sQ = reinterpret_cast<__nv_bfloat16 *>(smem_raw);
-    __nv_bfloat16 *sStage = sQ + 16 * kQStride;
-    __nv_bfloat16 *sKnew = sStage + kStages * kStageElems;
+    __nv_bfloat16 *sStage = sQ + 16 * kQStride;  // 16-bit elements: bf16, or f16 bits with fp8 caches
+    __nv_bfloat16 *sKnew = sStage + (kFp8 ? 1 : kStages) * kStageElems;
     __nv_bfloat16 *sVnew = sKnew + kDqk;
+    uint8_t *sLand = reinterpret_cast<uint8_t *>(sVnew + kDv);  // fp8 landing tiles (kFp8 only)
     __shared__ DecodeSmem red;
 
     const int tid = threadIdx.x;
@@ -138,9 +169,25 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
 
     // The first K/V tiles go out before the query preparation below.
     const int n_tiles = (key_end - key_begin + kTileKeys - 1) / kTileKeys;
+    const uint8_t *kc8 = reinterpret_cast<const uint8_t *>(a.k_cache) + ((size_t)b * a.cap * kv_row + kvh) * kDqk;
+    const uint8_t *vc8 = reinterpret_cast<const uint8_t *>(a.v_cache) + ((size_t)b * a.cap * kv_row + kvh) * kDv;
     auto issue = [&](int t) {
-        __nv_bfloat16 *st = sStage + (t % kStages) * kStageElems;
         const int base_key = key_begin + t * kTileKeys;
+        if (kFp8) {
+            // 20 chunks of 16 bytes per key: 12 of K, 8 of V
+            uint8_t *land = sLand + (t % kStages) * kLandBytes;
+            for (int c = tid; c < kTileKeys * 20; c += kThreads) {
+                const int r = c / 20;
+                const int ch = c - r * 20;
+                const int key = base_key + r;
+                const bool valid = key < key_end && key != slot_new;
+                const size_t ks = (size_t)(valid ? key : key_begin) * kv_row;
+                const uint8_t *src = ch < 12 ? kc8 + ks * kDqk + ch * 16 : vc8 + ks * kDv + (ch - 12) * 16;
+                cp_async16(land + r * kLandRow + ch * 16, src, valid ? 16u : 0u);
+            }
+            return;
+        }
+        __nv_bfloat16 *st = sStage + (t % kStages) * kStageElems;
         for (int c = tid; c < kTileKeys * 40; c += kThreads) {
             const int r = c / 40;
             const int ch = c - r * 40;
@@ -200,13 +247,13 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
                     const float2 c1 = s_cs[w * 8 + 2 * e + 1];
                     const float2 xa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pa[e]));
                     const float2 xb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pb[e]));
-                    qa[e] = pack_bf16x2(xa.x * c0.x - xb.x * c0.y, xa.y * c1.x - xb.y * c1.y);
-                    qb[e] = pack_bf16x2(xb.x * c0.x + xa.x * c0.y, xb.y * c1.x + xa.y * c1.y);
+                    qa[e] = pack16<kFp8>(xa.x * c0.x - xb.x * c0.y, xa.y * c1.x - xb.y * c1.y);
+                    qb[e] = pack16<kFp8>(xb.x * c0.x + xa.x * c0.y, xb.y * c1.x + xa.y * c1.y);
                 }
                 dst[w] = ya;
                 dst[w + npair] = yb;
             } else {
-                dst[npair + w] = va[k];
+                dst[npair + w] = kFp8 ? bf16x8_to_f16x8(va[k]) : va[k];
             }
         }
     } else {
@@ -226,12 +273,47 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
                     y = __bfloat162float(qr[e]);
                 }
             }
-            sQ[r * kQStride + e] = __float2bfloat16_rn(y);
+            if (kFp8)
+                reinterpret_cast<__half *>(sQ)[r * kQStride + e] = __float2half_rn(y);
+            else
+                sQ[r * kQStride + e] = __float2bfloat16_rn(y);
         }
     }
     // New token (CTA-uniform branch): rotate k from its raw copy, then write k
     // and v into the cache slot and keep the rotated copy for the tile.
-    if (owns_new) {
+    // rotated element e of the new key, from its raw copy in sKnew
+    auto rot_new_k = [&](int e) -> float {
+        if (e < L.rope.rotary_dim) {
+            const int j = e < half ? e : e - half;
+            const float2 cs = s_cs[j];
+            const float xa = __bfloat162float(sKnew[j]);
+            const float xb = __bfloat162float(sKnew[j + half]);
+            return e < half ? xa * cs.x - xb * cs.y : xb * cs.x + xa * cs.y;
+        }
+        return __bfloat162float(sKnew[e]);
+    };
+    if (owns_new && kFp8) {
+        // fp8 caches: the rotated key and the value are quantized (divided by
+        // their scales, nearest E4M3, saturating) two elements at a time; the
+        // tile uses the stored codes' values, as every other cached key.
+        uint8_t *kdst = reinterpret_cast<uint8_t *>(a.k_cache) + (((size_t)b * a.cap + slot_new) * kv_row + kvh) * kDqk;
+        uint8_t *vdst = reinterpret_cast<uint8_t *>(a.v_cache) + (((size_t)b * a.cap + slot_new) * kv_row + kvh) * kDv;
+        uint16_t kq = 0, vq = 0;
+        if (tid < kDqk / 2)
+            kq = f32x2_to_e4m3x2(rot_new_k(2 * tid) / a.k_scale, rot_new_k(2 * tid + 1) / a.k_scale);
+        if (tid < kDv / 2)
+            vq = f32x2_to_e4m3x2(__bfloat162float(sVnew[2 * tid]) / a.v_scale,
+                                 __bfloat162float(sVnew[2 * tid + 1]) / a.v_scale);
+        __syncthreads();  // every raw element read before any is overwritten
+        if (tid < kDqk / 2) {
+            reinterpret_cast<uint16_t *>(kdst)[tid] = kq;
+            reinterpret_cast<uint32_t *>(sKnew)[tid] = e4m3x2_to_f16x2(kq);
+        }
+        if (tid < kDv / 2) {
+            reinterpret_cast<uint16_t *>(vdst)[tid] = vq;
+            reinterpret_cast<uint32_t *>(sVnew)[tid] = e4m3x2_to_f16x2(vq);
+        }
+    } else if (owns_new) {
         __nv_bfloat16 *kdst = reinterpret_cast<__nv_bfloat16 *>(a.k_cache) +
                               (((size_t)b * a.cap + slot_new) * kv_row + kvh) * kDqk;
         __nv_bfloat16 *vdst = reinterpret_cast<__nv_bfloat16 *>(a.v_cache) +
@@ -240,19 +322,7 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
             const int e = tid + k * kThreads;
-            float y = 0.f;
-            if (e < kDqk) {
-                if (e < L.rope.rotary_dim) {
-                    const int j = e < half ? e : e - half;
-                    const float2 cs = s_cs[j];
-                    const float xa = __bfloat162float(sKnew[j]);
-                    const float xb = __bfloat162float(sKnew[j + half]);
-                    y = e < half ? xa * cs.x - xb * cs.y : xb * cs.x + xa * cs.y;
-                } else {
-                    y = __bfloat162float(sKnew[e]);
-                }
-            }
-            yk[k] = __float2bfloat16_rn(y);
+            yk[k] = __float2bfloat16_rn(e < kDqk ? rot_new_k(e) : 0.f);
         }
         __syncthreads();  // every raw element read before any is overwritten
 #pragma unroll
@@ -298,8 +368,27 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
         cp_async_commit();
         cp_async_wait<kStages - 1>();
         __syncthreads();
-        __nv_bfloat16 *st = sStage + (t % kStages) * kStageElems;
+        __nv_bfloat16 *st = kFp8 ? sStage : sStage + (t % kStages) * kStageElems;
         const int base_key = key_begin + t * kTileKeys;
+        if (kFp8) {
+            // widen the landed e4m3 tile into the padded f16 compute tile
+            const uint8_t *land = sLand + (t % kStages) * kLandBytes;
+            for (int c = tid; c < kTileKeys * 20; c += kThreads) {
+                const int r = c / 20;
+                const int ch = c - r * 20;
+                const uint4 w = *reinterpret_cast<const uint4 *>(land + r * kLandRow + ch * 16);
+                uint4 h0, h1;
+                e4m3x4_to_f16x4(w.x, h0.x, h0.y);
+                e4m3x4_to_f16x4(w.y, h0.z, h0.w);
+                e4m3x4_to_f16x4(w.z, h1.x, h1.y);
+                e4m3x4_to_f16x4(w.w, h1.z, h1.w);
+                uint4 *dst = reinterpret_cast<uint4 *>(
+                    ch < 12 ? st + r * kKStride + ch * 16 : st + kTileKeys * kKStride + r * kVStride + (ch - 12) * 16);
+                dst[0] = h0;
+                dst[1] = h1;
+            }
+            __syncthreads();
+        }
         if (owns_new && slot_new >= base_key && slot_new < base_key + kTileKeys) {
             const int r = slot_new - base_key;
             if (tid < 24)
@@ -323,8 +412,8 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
             for (int ks = 0; ks < 12; ++ks) {
                 uint32_t b0, b1, b2, b3;
                 ldmatrix_x4(base + ks * 32, b0, b1, b2, b3);
-                mma_bf16_16816(s_acc[0], qa[ks], b0, b1);
-                mma_bf16_16816(s_acc[1], qa[ks], b2, b3);
+                mma16<kFp8>(s_acc[0], qa[ks], b0, b1);
+                mma16<kFp8>(s_acc[1], qa[ks], b2, b3);
             }
         }
         // Scale, mask keys past the end of the range, online softmax.
@@ -374,10 +463,10 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
             o[d][3] *= c1;
         }
         uint32_t pa[4];
-        pa[0] = pack_bf16x2(p[0][0], p[0][1]);
-        pa[1] = pack_bf16x2(p[0][2], p[0][3]);
-        pa[2] = pack_bf16x2(p[1][0], p[1][1]);
-        pa[3] = pack_bf16x2(p[1][2], p[1][3]);
+        pa[0] = pack16<kFp8>(p[0][0], p[0][1]);
+        pa[1] = pack16<kFp8>(p[0][2], p[0][3]);
+        pa[2] = pack16<kFp8>(p[1][0], p[1][1]);
+        pa[3] = pack16<kFp8>(p[1][2], p[1][3]);
         // O += P V over these 16 keys.
         {
             const int mi = lane >> 3;
@@ -388,8 +477,8 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages>::kCtasPerSm)
             for (int dp = 0; dp < 8; ++dp) {
                 uint32_t b0, b1, b2, b3;
                 ldmatrix_x4_trans(base + dp * 32, b0, b1, b2, b3);
-                mma_bf16_16816(o[2 * dp], pa, b0, b1);
-                mma_bf16_16816(o[2 * dp + 1], pa, b2, b3);
+                mma16<kFp8>(o[2 * dp], pa, b0, b1);
+                mma16<kFp8>(o[2 * dp + 1], pa, b2, b3);
             }
         }
     }
@@ -684,20 +773,56 @@ int decode_max_splits(const LayerArgs &L, int dtype, int cap)
     return (cap + chunk - 1) / chunk;
 }
 
+namespace {
+__global__ void quantize_e4m3_kernel(const __nv_bfloat16 *src, uint8_t *dst, size_t n, float scale)
+{
+    for (size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 2; i < n; i += (size_t)gridDim.x * blockDim.x * 2) {
+        const float x0 = __bfloat162float(src[i]) / scale;
+        if (i + 1 < n) {
+            const uint16_t c = f32x2_to_e4m3x2(x0, __bfloat162float(src[i + 1]) / scale);
+            dst[i] = (uint8_t)(c & 0xFF);
+            dst[i + 1] = (uint8_t)(c >> 8);
+        } else {
+            dst[i] = (uint8_t)(f32x2_to_e4m3x2(x0, 0.f) & 0xFF);
+        }
+    }
+}
+} // namespace
+
+cudaError_t launch_quantize_e4m3(const void *src, void *dst, size_t n, float scale, cudaStream_t stream)
+{
+    const size_t pairs = (n + 1) / 2;
+    const size_t blocks = (pairs + 255) / 256;
+    quantize_e4m3_kernel<<<(unsigned)(blocks < 65536 ? blocks : 65536), 256, 0, stream>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(src), reinterpret_cast<uint8_t *>(dst), n, scale);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_decode(const LayerArgs &L, const DecodeArgs &a, int dtype, cudaStream_t stream)
 {
+    if (a.fp8_cache && !decode_mma_supported(L, dtype))
+        return cudaErrorInvalidValue;
     if (decode_mma_supported(L, dtype)) {
-        static bool attr_set = false;
-        if (!attr_set) {
-            cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<kDecodeStages>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 DecodeCfg<kDecodeStages>::kSmemBytes);
+        static bool attr_set[2] = {false, false};
+        const int f = a.fp8_cache ? 1 : 0;
+        if (!attr_set[f]) {
+            cudaError_t e = f ? cudaFuncSetAttribute(decode_mma_kernel<kDecodeStages, true>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     DecodeCfg<kDecodeStages, true>::kSmemBytes)
+                              : cudaFuncSetAttribute(decode_mma_kernel<kDecodeStages, false>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     DecodeCfg<kDecodeStages, false>::kSmemBytes);
             if (e != cudaSuccess)
                 return e;
-            attr_set = true;
+            attr_set[f] = true;
         }
         dim3 grid(a.max_splits, L.Hkv, a.B);
-        decode_mma_kernel<kDecodeStages><<<grid, kThreads, DecodeCfg<kDecodeStages>::kSmemBytes, stream>>>(L, a);
+        if (f)
+            decode_mma_kernel<kDecodeStages, true>
+                <<<grid, kThreads, DecodeCfg<kDecodeStages, true>::kSmemBytes, stream>>>(L, a);
+        else
+            decode_mma_kernel<kDecodeStages, false>
+                <<<grid, kThreads, DecodeCfg<kDecodeStages, false>::kSmemBytes, stream>>>(L, a);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess || a.max_splits <= 1)
             return e;

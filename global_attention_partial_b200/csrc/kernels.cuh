@@ -129,7 +129,15 @@ struct DecodeArgs {
     int chunk;       // keys per split
     int B;
     unsigned *err;
+    // E4M3 caches (bytes): a cached value is scale * e4m3(code); the new
+    // token's rotated key and value are stored as e4m3(x / scale). The
+    // scales also multiply the scores (k_scale) and the output (v_scale):
+    // the caller folds them into the layer's softmax and V scales.
+    int fp8_cache;
+    float k_scale, v_scale;
 };
+// dst[i] = e4m3(src[i] / scale) (bf16 in, E4M3 codes out; nearest, saturating).
+cudaError_t launch_quantize_e4m3(const void *src, void *dst, size_t n, float scale, cudaStream_t stream);
 int decode_chunk_keys(const LayerArgs &L, int dtype);
 int decode_max_splits(const LayerArgs &L, int dtype, int cap);
 cudaError_t launch_decode(const LayerArgs &L, const DecodeArgs &a, int dtype, cudaStream_t stream);

@@ -215,6 +215,45 @@ MIMO_ATTN_API mimo_attn_status mimo_attn_decode_static(const mimo_attn_layer *la
                                          const int32_t *kv_lens, void *k_cache, void *v_cache,
                                          int cache_capacity, void *out, void *stream);
 
+/* Bytes of workspace mimo_attn_decode_fp8kv needs (the same split-KV partial
+ * results as the bf16 decode). */
+MIMO_ATTN_API size_t mimo_attn_decode_fp8kv_workspace_size(const mimo_attn_layer *layer, int batch,
+                                                           int cache_capacity);
+
+/* Decode over an fp8 KV cache. The pages ("Add Xiaomi MiMo-V2", section
+ * "Additional useful info") note that the model ships a quantized variant
+ * without saying what is quantized or how; this entry point is the plainest
+ * reading for the decode hot path: the caches hold OCP FP8 E4M3 codes with
+ * one scale per tensor (a cached key is k_scale * e4m3 value, a cached value
+ * v_scale * e4m3 value), everything else is the bf16 decode.
+ *   q [batch, Hq, Dqk], k_new [batch, Hkv, Dqk], v_new [batch, Hkv, Dv]:
+ *          bf16, unrotated, as in mimo_attn_decode.
+ *   kv_lens, cache_capacity, layouts: as in mimo_attn_decode, with one byte
+ *          per element in k_cache / v_cache ([batch, cap, Hkv, D] uint8).
+ *   k_scale, v_scale: finite, > 0.
+ *   The new token's key, rotated in fp32, is divided by k_scale and
+ *          stored as its E4M3 code (round to nearest even, saturating at
+ *          +-448); v_new likewise with v_scale. Its own score and value use
+ *          the stored codes, so the result is the attention over the cache as
+ *          it stands after the call.
+ *   out [batch, Hq, Dv] bf16. Scores and the PV product are computed from
+ *          f16 operands (every E4M3 value is exact in f16) with fp32
+ *          accumulation; the query is rounded to f16.
+ * Supported: Dqk 192, Dv 128, Hq/Hkv <= 16 (else MIMO_ATTN_ERR_UNSUPPORTED).
+ * q, k_new, v_new, out and both caches must be 16-byte aligned. */
+MIMO_ATTN_API mimo_attn_status mimo_attn_decode_fp8kv(const mimo_attn_layer *layer, int batch, const void *q,
+                                                      const void *k_new, const void *v_new,
+                                                      const int32_t *kv_lens, void *k_cache, void *v_cache,
+                                                      int cache_capacity, float k_scale, float v_scale,
+                                                      void *out, void *workspace, size_t workspace_bytes,
+                                                      void *stream);
+
+/* dst[i] = E4M3 code of src[i] / scale for i < n (src bf16, dst uint8;
+ * round to nearest even, saturating at +-448, NaN stays NaN). Fills an fp8
+ * cache from bf16 keys and values (keys already rotated). scale finite, > 0. */
+MIMO_ATTN_API mimo_attn_status mimo_attn_quantize_fp8(const void *src, void *dst, size_t n, float scale,
+                                                      void *stream);
+
 /* Device error word bits (sticky until read). */
 #define MIMO_ATTN_DEVERR_KV_LEN 0x1u   /* a kv_lens entry was out of range */
 #define MIMO_ATTN_DEVERR_TIMEOUT 0x2u  /* a kernel pipeline wait hit its iteration limit */

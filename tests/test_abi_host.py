@@ -23,7 +23,7 @@ def lib():
 def header_functions():
     text = open(os.path.join(ROOT, "include", "mimo_attn.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(mimo_attn_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(mimo_attn_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_library_exports_every_declared_function(lib):
@@ -217,3 +217,32 @@ def test_prefill_cached_workspace_sizes(lib):
     assert mimo.mimo_attn_prefill_cached_workspace_size(w17, mimo.FP32, 1, 10, 0) == \
         256 * math.ceil(10 * 32 * 8 / 256) + 256 * math.ceil(rows * 192 * 4 / 256) + 256 * math.ceil(rows * 128 * 4 / 256)
     assert mimo.mimo_attn_prefill_cached_workspace_size(ga, mimo.BF16, 1, 8, -1) == 0
+
+
+def fp8_status(l, batch=2, cap=128, ws=1 << 30, ks=1.0, vs=1.0):
+    return mimo.mimo_attn_decode_fp8kv(l, batch, T(), T(), T(), T(), T(), T(), cap, ks, vs, T(), T(), ws, 0)
+
+
+def test_decode_fp8kv_argument_checks(lib):
+    mimo.mimo_attn_debug_fail_launches(True)
+    try:
+        l = layer()
+        assert fp8_status(l, cap=64) == mimo.ERR_INVALID_ARG                 # ring must equal window
+        for bad in (0.0, -1.0, float("inf"), float("nan")):
+            assert fp8_status(l, ks=bad) == mimo.ERR_INVALID_ARG
+            assert fp8_status(l, vs=bad) == mimo.ERR_INVALID_ARG
+        assert fp8_status(layer(qk_dim=128, rotary_dim=42)) == mimo.ERR_UNSUPPORTED
+        assert fp8_status(layer(num_kv_heads=2)) == mimo.ERR_UNSUPPORTED  # G = 32 > 16
+        assert fp8_status(l, batch=0) == mimo.OK
+        assert fp8_status(l) == mimo.ERR_CUDA
+        g = layer(layer_type=mimo.GLOBAL, num_kv_heads=4)
+        need = mimo.mimo_attn_decode_fp8kv_workspace_size(g, 64, 32768)
+        assert need == mimo.mimo_attn_decode_workspace_size(g, mimo.BF16, 64, 32768)
+        assert fp8_status(g, batch=64, cap=32768, ws=need - 1) == mimo.ERR_WORKSPACE
+        assert fp8_status(g, batch=64, cap=32768, ws=need) == mimo.ERR_CUDA
+        assert mimo.mimo_attn_quantize_fp8(T(), T(), 10, 0.0, 0) == mimo.ERR_INVALID_ARG
+        assert mimo.mimo_attn_quantize_fp8(None, T(), 10, 1.0, 0) == mimo.ERR_INVALID_ARG
+        assert mimo.mimo_attn_quantize_fp8(None, None, 0, 1.0, 0) == mimo.OK
+        assert mimo.mimo_attn_quantize_fp8(T(), T(), 10, 1.0, 0) == mimo.ERR_CUDA
+    finally:
+        mimo.mimo_attn_debug_fail_launches(False)
