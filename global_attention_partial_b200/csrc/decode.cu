@@ -37,11 +37,15 @@ constexpr int kStageElems = kTileKeys * (kKStride + kVStride);
 // widened to f16 into one padded compute tile (e4m3 values are exact in f16).
 constexpr int kLandRow = kDqk + kDv;             // bytes per key
 constexpr int kLandBytes = kTileKeys * kLandRow;  // 20480
+// With fp8 caches the query rows are staged in the compute tile (they are
+// read into registers before the first tile is widened there), so a 3-deep
+// landing ring still leaves room for 2 CTAs per SM.
 template <int ST, bool F8 = false> struct DecodeCfg {
-    static constexpr int kSmemBytes = F8 ? (16 * kQStride + kStageElems + kDqk + kDv) * 2 + ST * kLandBytes
+    static constexpr int kSmemBytes = F8 ? (kStageElems + kDqk + kDv) * 2 + ST * kLandBytes
                                          : (16 * kQStride + ST * kStageElems + kDqk + kDv) * 2;
-    static constexpr int kCtasPerSm = ST <= 2 ? 2 : 1;
+    static constexpr int kCtasPerSm = (F8 ? ST <= 3 : ST <= 2) ? 2 : 1;
 };
+static_assert(16 * kQStride <= kStageElems, "query rows fit in the compute tile");
 
 // 16-bit operand type of the tensor-core path: bf16 for bf16 caches, f16 for
 // fp8 caches (their e4m3 values, the f16 query and the probabilities).
@@ -68,6 +72,8 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v)
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 constexpr int kDecodeStages = 2;
+constexpr int kDecodeStagesFp8 = 3;  // 20 KB landing tiles: 2 in flight while one is computed
+static_assert(DecodeCfg<kDecodeStagesFp8, true>::kSmemBytes <= 110 * 1024, "2 CTAs per SM");
 
 struct DecodeSmem {
     float wm[4][16];
@@ -93,8 +99,9 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
     decode_mma_kernel(const __grid_constant__ LayerArgs L, const __grid_constant__ DecodeArgs a)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    __nv_bfloat16 *sQ = reinterpret_cast<__nv_bfloat16 *>(smem_raw);
-    __nv_bfloat16 *sStage = sQ + 16 * kQStride;  // 16-bit elements: bf16, or f16 bits with fp8 caches
+    // 16-bit elements: bf16, or f16 bits with fp8 caches
+    __nv_bfloat16 *sStage = reinterpret_cast<__nv_bfloat16 *>(smem_raw) + (kFp8 ? 0 : 16 * kQStride);
+    __nv_bfloat16 *sQ = kFp8 ? sStage : reinterpret_cast<__nv_bfloat16 *>(smem_raw);
     __nv_bfloat16 *sKnew = sStage + (kFp8 ? 1 : kStages) * kStageElems;
     __nv_bfloat16 *sVnew = sKnew + kDqk;
     uint8_t *sLand = reinterpret_cast<uint8_t *>(sVnew + kDv);  // fp8 landing tiles (kFp8 only)
@@ -806,9 +813,9 @@ cudaError_t launch_decode(const LayerArgs &L, const DecodeArgs &a, int dtype, cu
         static bool attr_set[2] = {false, false};
         const int f = a.fp8_cache ? 1 : 0;
         if (!attr_set[f]) {
-            cudaError_t e = f ? cudaFuncSetAttribute(decode_mma_kernel<kDecodeStages, true>,
+            cudaError_t e = f ? cudaFuncSetAttribute(decode_mma_kernel<kDecodeStagesFp8, true>,
                                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                     DecodeCfg<kDecodeStages, true>::kSmemBytes)
+                                                     DecodeCfg<kDecodeStagesFp8, true>::kSmemBytes)
                               : cudaFuncSetAttribute(decode_mma_kernel<kDecodeStages, false>,
                                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                      DecodeCfg<kDecodeStages, false>::kSmemBytes);
@@ -818,8 +825,8 @@ cudaError_t launch_decode(const LayerArgs &L, const DecodeArgs &a, int dtype, cu
         }
         dim3 grid(a.max_splits, L.Hkv, a.B);
         if (f)
-            decode_mma_kernel<kDecodeStages, true>
-                <<<grid, kThreads, DecodeCfg<kDecodeStages, true>::kSmemBytes, stream>>>(L, a);
+            decode_mma_kernel<kDecodeStagesFp8, true>
+                <<<grid, kThreads, DecodeCfg<kDecodeStagesFp8, true>::kSmemBytes, stream>>>(L, a);
         else
             decode_mma_kernel<kDecodeStages, false>
                 <<<grid, kThreads, DecodeCfg<kDecodeStages, false>::kSmemBytes, stream>>>(L, a);
