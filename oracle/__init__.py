@@ -322,3 +322,46 @@ def decode_fp8kv(q, k_new, v_new, k_codes, v_codes, L: int, rotary_dim: int, the
         s = None if sinks is None else float(np.asarray(sinks)[r])
         out[r] = prefill_rows(q_rot[r:r + 1], [L - 1], K, V, layer_type, window, softmax_scale, s, vscale)[0]
     return out, kc, vc
+
+
+def qkv_project(x, w_qkv, positions, *, num_q_heads: int, num_kv_heads: int, qk_dim: int, v_dim: int,
+                rotary_dim: int, theta: float):
+    """The step before attention: the token's hidden state x ([T, hidden])
+    times the stacked projection weight w_qkv ([Hq*Dqk + Hkv*Dqk + Hkv*Dv,
+    hidden]: the rows of W_q, then W_k, then W_v, each in the [out, in]
+    layout of a linear layer, no bias), split into query, key and value heads;
+    queries and keys then get the layer's partial RoPE at the token's
+    position, values are left as they are (PR 45144, "Additional useful
+    info": partial RoPE, decoupled V head dim). Returns q [T, Hq, Dqk],
+    k [T, Hkv, Dqk] (both rotated) and v [T, Hkv, Dv]."""
+    x = _f64(x)
+    w = _f64(w_qkv)
+    T = x.shape[0]
+    nq, nk, nv = num_q_heads * qk_dim, num_kv_heads * qk_dim, num_kv_heads * v_dim
+    if w.shape != (nq + nk + nv, x.shape[1]):
+        raise ValueError("qkv_project: weight shape")
+    y = x @ w.T  # one product per (token, output feature)
+    pos = np.asarray(positions, dtype=np.float64).reshape(T)
+    q = y[:, :nq].reshape(T, num_q_heads, qk_dim)
+    k = y[:, nq:nq + nk].reshape(T, num_kv_heads, qk_dim)
+    v = y[:, nq + nk:].reshape(T, num_kv_heads, v_dim).copy()
+    q_rot = rope(q.reshape(T * num_q_heads, qk_dim), rotary_dim, theta,
+                 np.repeat(pos, num_q_heads)).reshape(T, num_q_heads, qk_dim)
+    k_rot = rope(k.reshape(T * num_kv_heads, qk_dim), rotary_dim, theta,
+                 np.repeat(pos, num_kv_heads)).reshape(T, num_kv_heads, qk_dim)
+    return q_rot, k_rot, v
+
+
+def cache_write(k_cache, v_cache, k, v, positions, *, layer_type: int, window: int):
+    """Stores each token's (rotated) key and value in its cache slot, tokens
+    in order, so a later token that maps to the same slot wins: slot = position
+    in a global layer's linear cache, position mod window in a sliding
+    layer's ring (issue 842, "Implementation plan": rotating cache).
+    k_cache/v_cache [cap, Hkv, D]; k/v [T, Hkv, D]. Returns new arrays."""
+    kc = _f64(k_cache).copy()
+    vc = _f64(v_cache).copy()
+    for t, p in enumerate(np.asarray(positions).reshape(-1)):
+        slot = int(p) % window if layer_type == SWA else int(p)
+        kc[slot] = k[t]
+        vc[slot] = v[t]
+    return kc, vc

@@ -419,6 +419,8 @@ def test_e4m3_encode_round_trip_ties_and_saturation():
     assert np.array_equal(oracle.e4m3_encode(v[finite]), np.array(finite, dtype=np.uint8))
     assert list(oracle.e4m3_encode([1.0625, 1.1875, 1.9375, 2.0 ** -10, 3 * 2.0 ** -11])) == [0x38, 0x3A, 0x40, 0x00, 0x01]
     assert list(oracle.e4m3_encode([448.0, 465.0, 1e6, -1e6])) == [0x7E, 0x7E, 0x7E, 0xFE]
+    # a value that rounds to zero keeps its sign, as an IEEE-style conversion does
+    assert list(oracle.e4m3_encode([0.0, -0.0, -1e-9, 1e-9])) == [0x00, 0x80, 0x80, 0x00]
     x = RNG.uniform(-400, 400, 2000)
     got = oracle.e4m3_value(oracle.e4m3_encode(x))
     nearest = np.array([v[finite][np.argmin(np.abs(v[finite] - xi))] for xi in x])
@@ -446,3 +448,91 @@ def test_fp8_decode_equals_bf16_decode_on_representable_values(layer_type, L, W)
     np.testing.assert_allclose(o8, o16, rtol=0, atol=1e-13)
     np.testing.assert_array_equal(ks * oracle.e4m3_value(kc2), kc16)
     np.testing.assert_array_equal(vs * oracle.e4m3_value(vc2), vc16)
+
+
+# ------------------------------------------------- QKV projection step pins
+
+def test_qkv_project_brute_force_at_position_zero():
+    """At position 0 RoPE is the identity, so every output is one dot product
+    of the token's hidden state with one weight row, written out as a loop:
+    query head h, dim d is row h*Dqk + d; key head j is row Hq*Dqk + j*Dqk + d;
+    value head j is row (Hq + Hkv)*Dqk + j*Dv + d. Catches a transposed
+    weight and the q/k/v blocks in the wrong order."""
+    T, hidden, Hq, Hkv, Dqk, Dv = 3, 5, 2, 1, 4, 2
+    x = rnd(T, hidden)
+    w = rnd(Hq * Dqk + Hkv * Dqk + Hkv * Dv, hidden)
+    q, k, v = oracle.qkv_project(x, w, np.zeros(T), num_q_heads=Hq, num_kv_heads=Hkv, qk_dim=Dqk, v_dim=Dv,
+                                 rotary_dim=2, theta=1e4)
+
+    def dot(t, row):
+        return sum(x[t, i] * w[row, i] for i in range(hidden))
+
+    for t in range(T):
+        for h in range(Hq):
+            for d in range(Dqk):
+                assert abs(q[t, h, d] - dot(t, h * Dqk + d)) < 1e-12
+        for j in range(Hkv):
+            for d in range(Dqk):
+                assert abs(k[t, j, d] - dot(t, Hq * Dqk + j * Dqk + d)) < 1e-12
+            for d in range(Dv):
+                assert abs(v[t, j, d] - dot(t, (Hq + Hkv) * Dqk + j * Dv + d)) < 1e-12
+
+
+def test_qkv_project_rope_closed_form():
+    """Selection weights (W_q = I, W_k = 2I, W_v = the first Dv rows of I)
+    make the projections the hidden state itself, so the outputs at position
+    p are the rotation written out: pair (j, j + r/2) of the first r dims
+    turns by p * theta^(-2j/r); the rest and V pass through. Catches a wrong
+    pairing, sign or frequency in the projection's RoPE, and a rotated V."""
+    D, Dv, r, theta, p = 8, 4, 4, 100.0, 3.0
+    x = rnd(1, D)
+    w = np.concatenate([np.eye(D), 2 * np.eye(D), np.eye(D)[:Dv]])
+    q, k, v = oracle.qkv_project(x, w, [p], num_q_heads=1, num_kv_heads=1, qk_dim=D, v_dim=Dv,
+                                 rotary_dim=r, theta=theta)
+    for j in range(r // 2):
+        phi = p * theta ** (-2 * j / r)
+        a, b = x[0, j], x[0, j + r // 2]
+        z = complex(a, b) * cmath.exp(1j * phi)
+        assert abs(q[0, 0, j] - z.real) < 1e-12 and abs(q[0, 0, j + r // 2] - z.imag) < 1e-12
+        assert abs(k[0, 0, j] - 2 * z.real) < 1e-12 and abs(k[0, 0, j + r // 2] - 2 * z.imag) < 1e-12
+    np.testing.assert_array_equal(q[0, 0, r:], x[0, r:])
+    np.testing.assert_array_equal(v[0, 0], x[0, :Dv])
+
+
+@pytest.mark.parametrize("layer_type", [0, 1])
+def test_qkv_then_attention_without_rope_is_the_layer(layer_type):
+    """Projection outputs are already rotated, so attention over them with
+    rotary_dim 0 equals the layer (attention with RoPE) over the unrotated
+    projections x W^T. Ties the projection's RoPE to the attention's own,
+    independently pinned, and fixes how the two calls compose."""
+    B, S, hidden, Hq, Hkv, Dqk, Dv, r, W = 1, 9, 6, 4, 2, 8, 4, 4, 3
+    x = rnd(B * S, hidden)
+    w = rnd(Hq * Dqk + Hkv * (Dqk + Dv), hidden)
+    pos = np.arange(S, dtype=np.float64)
+    q, k, v = oracle.qkv_project(x, w, pos, num_q_heads=Hq, num_kv_heads=Hkv, qk_dim=Dqk, v_dim=Dv,
+                                 rotary_dim=r, theta=1e4)
+    y = x @ w.T
+    q0 = y[:, :Hq * Dqk].reshape(B, S, Hq, Dqk)
+    k0 = y[:, Hq * Dqk:(Hq + Hkv) * Dqk].reshape(B, S, Hkv, Dqk)
+    v0 = y[:, (Hq + Hkv) * Dqk:].reshape(B, S, Hkv, Dv)
+    sinks = rnd(Hq) if layer_type == 1 else None
+    kw = dict(layer_type=layer_type, num_kv_heads=Hkv, theta=1e4, window=W, sinks=sinks, hidden_size=64)
+    want = oracle.prefill_layer(q0, k0, v0, rotary_dim=r, **kw)
+    got = oracle.prefill_layer(q.reshape(B, S, Hq, Dqk), k.reshape(B, S, Hkv, Dqk), v.reshape(B, S, Hkv, Dv),
+                               rotary_dim=0, **kw)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_cache_write_slots():
+    """A global cache holds position p in slot p; a ring of W slots holds, in
+    slot s, the latest token whose position is s mod W (later tokens
+    overwrite earlier ones)."""
+    T, W = 10, 4
+    k = np.arange(T, dtype=np.float64).reshape(T, 1, 1) + 100
+    v = -k
+    kc, vc = oracle.cache_write(np.zeros((T, 1, 1)), np.zeros((T, 1, 1)), k, v, np.arange(T),
+                                layer_type=0, window=W)
+    assert list(kc[:, 0, 0]) == [100 + p for p in range(T)] and np.array_equal(vc, -kc)
+    kc, vc = oracle.cache_write(np.zeros((W, 1, 1)), np.zeros((W, 1, 1)), k, v, np.arange(T),
+                                layer_type=1, window=W)
+    assert list(kc[:, 0, 0]) == [108, 109, 106, 107] and np.array_equal(vc, -kc)
