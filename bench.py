@@ -1,7 +1,7 @@
 """Benchmark of the MiMo-V2-Flash hybrid attention path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload stack|swa|global|decode|chunked|decode_fp8] [--no-e2e] [--no-cpu-baseline]
+                    [--workload stack|swa|global|decode|chunked|decode_fp8|qkv] [--no-e2e] [--no-cpu-baseline]
 
 One step = one pass of the whole hot path over the hybrid 8-layer attention
 stack (hybrid_layer_pattern 0,1,1,1,1,1,0,1: 6 sliding-window layers with
@@ -79,6 +79,12 @@ def chunk_flops(spec, B: int, S: int, past: int) -> float:
     else:
         pairs = sum(min(past + t + 1, spec.window) for t in range(S))
     return float(B) * spec.num_q_heads * pairs * 2 * (spec.qk_dim + spec.v_dim)
+
+
+def qkv_flops(spec, B: int, S: int) -> float:
+    """FLOPs of one layer's QKV projection: 2 per multiply-add of x W^T."""
+    n = spec.num_q_heads * spec.qk_dim + spec.num_kv_heads * (spec.qk_dim + spec.v_dim)
+    return 2.0 * B * S * n * spec.hidden_size
 
 
 def prefill_bytes(spec, B: int, S: int) -> float:
@@ -193,6 +199,7 @@ class StackWorkload:
         self.fp8 = kind == "decode_fp8"
         self.k_scale, self.v_scale = 1.0 / 16, 1.0 / 32
         self.do_chunked = kind == "chunked"
+        self.do_qkv = kind == "qkv"
         self.pw, self.dw = pw, dw
         self.prefill_layers = []
         if self.do_prefill:
@@ -225,6 +232,28 @@ class StackWorkload:
                 need = mimo.mimo_attn_prefill_cached_workspace_size(lay, mimo.BF16, B, S, P)
                 ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
                 self.chunk_layers.append(dict(spec=spec, lay=lay, q=q, k=k, v=v, kc=kc, vc=vc, out=out, ws=ws))
+        # qkv: every layer's fused QKV projection of the stack's prefill tokens
+        # (outputs and the cache write; x and the output buffers are shared
+        # by the layers, each layer has its own weights and caches)
+        self.qkv_layers = []
+        if self.do_qkv:
+            B, S = pw.batch, pw.seq
+            spec0 = pw.layers[0]
+            self.qkv_x, _ = synthetic.projection_inputs(spec0, B, S, seed=seed, layer=0, device=dev)
+            self.qkv_q = torch.empty((B, S, spec0.num_q_heads, spec0.qk_dim), dtype=torch.bfloat16, device=dev)
+            kv_heads = max(s.num_kv_heads for s in pw.layers)
+            self.qkv_k = torch.empty((B, S, kv_heads, spec0.qk_dim), dtype=torch.bfloat16, device=dev)
+            self.qkv_v = torch.empty((B, S, kv_heads, spec0.v_dim), dtype=torch.bfloat16, device=dev)
+            for li, spec in enumerate(pw.layers):
+                _, w = synthetic.projection_inputs(spec, 1, 1, seed=seed, layer=li, device=dev)
+                lay = mimo.make_layer(spec.layer_type, spec.num_q_heads, spec.num_kv_heads, spec.qk_dim,
+                                      spec.v_dim, spec.rotary_dim, spec.window, spec.theta, spec.hidden_size, None)
+                cap = spec.window if spec.layer_type == 1 else S
+                kc = torch.empty((B, cap, spec.num_kv_heads, spec.qk_dim), dtype=torch.bfloat16, device=dev)
+                vc = torch.empty((B, cap, spec.num_kv_heads, spec.v_dim), dtype=torch.bfloat16, device=dev)
+                need = mimo.mimo_attn_qkv_project_workspace_size(lay, B, S, 0)
+                ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+                self.qkv_layers.append(dict(spec=spec, lay=lay, w=w, kc=kc, vc=vc, cap=cap, ws=ws))
         self.decode_layers = []
         if self.do_decode:
             B = dw.batch
@@ -255,6 +284,17 @@ class StackWorkload:
     def decode_flops(self):
         return sum(decode_flops(L["spec"], self.lens) for L in self.decode_layers)
 
+    def qkv_flops(self):
+        return sum(qkv_flops(L["spec"], self.pw.batch, self.pw.seq) for L in self.qkv_layers)
+
+    def run_qkv_layer(self, L, stream):
+        m = self.mimo
+        st = m.mimo_attn_qkv_project(L["lay"], self.pw.batch, self.pw.seq, self.qkv_x, L["w"], None, 0, self.qkv_q,
+                                     self.qkv_k, self.qkv_v, L["kc"], L["vc"], L["cap"], L["ws"], L["ws"].numel(),
+                                     stream)
+        if st != m.OK:
+            raise m.MimoAttnError(st, "mimo_attn_qkv_project")
+
     def chunk_flops(self):
         return sum(chunk_flops(L["spec"], self.pw.batch, self.chunk_seq, self.chunk_past) for L in self.chunk_layers)
 
@@ -275,6 +315,7 @@ class StackWorkload:
             n += 3 if L["spec"].layer_type == 0 else 4
         for L in self.decode_layers:
             n += 2 if L["need"] > 0 else 1  # split kernel (+ combine)
+        n += 2 * len(self.qkv_layers)  # RoPE table + projection
         return n
 
     def run_prefill_layer(self, L, stream):
@@ -351,6 +392,17 @@ class StackWorkload:
                 events.setdefault(kind, []).append((e0, e1))
             else:
                 self.run_chunk_layer(L, stream)
+        for L in self.qkv_layers:
+            kind = "qkv_global" if L["spec"].layer_type == 0 else "qkv_swa"
+            if events is not None:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                self.run_qkv_layer(L, stream)
+                e1.record(stream)
+                events.setdefault(kind, []).append((e0, e1))
+            else:
+                self.run_qkv_layer(L, stream)
         if self.decode_layers:
             if events is not None:
                 e0 = torch.cuda.Event(enable_timing=True)
@@ -546,6 +598,8 @@ def workload_config(args, reference=False):
              "swa": synthetic.SWA_PREFILL.name, "global": synthetic.GLOBAL_PREFILL.name,
              "decode": synthetic.HYBRID_DECODE.name,
              "decode_fp8": synthetic.HYBRID_DECODE.name.replace("bf16", "bf16 q/out, fp8 E4M3 KV cache"),
+             "qkv": "hybrid 8-layer stack QKV projection (x W^T + RoPE + q/k/v and cache stores) bf16 B4 S32768 "
+                    "hidden 4096 pattern 0,1,1,1,1,1,0,1",
              "chunked": f"hybrid 8-layer stack, chunk of {CHUNK_SEQ} tokens after {CHUNK_PAST} cached, bf16 B4 "
                         f"pattern 0,1,1,1,1,1,0,1"}
     cfg = {"workload": names[args.workload], "prefill_batch": synthetic.HYBRID_PREFILL.batch,
@@ -567,13 +621,13 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["stack", "swa", "global", "decode", "chunked", "decode_fp8"], default="stack")
+    ap.add_argument("--workload", choices=["stack", "swa", "global", "decode", "chunked", "decode_fp8", "qkv"], default="stack")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the decode layers one call at a time")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
-    if args.workload in ("chunked", "decode_fp8"):  # NEXT-row measurements: kernels only, no host or oracle legs
+    if args.workload in ("chunked", "decode_fp8", "qkv"):  # NEXT-row measurements: kernels only, no host or oracle legs
         args.no_e2e = True
         args.no_cpu_baseline = True
     if args.impl == "reference":
@@ -625,7 +679,8 @@ def main():
     pflops = w.prefill_flops() if w.do_prefill else 0.0
     dflops = w.decode_flops() if w.do_decode else 0.0
     cflops = w.chunk_flops() if w.do_chunked else 0.0
-    step_flops = pflops + dflops + cflops
+    qflops = w.qkv_flops() if w.do_qkv else 0.0
+    step_flops = pflops + dflops + cflops + qflops
     value = job_value(world, step_flops, ms)
 
     parts = {}
@@ -674,6 +729,18 @@ def main():
         roofline = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                     "frac": ach / peaks["bf16_tflops_sustained"], "traffic": None,
                     "kernel": "prefill_ga_kernel (global layer, chunk of 4096 after 28672 cached, B4)",
+                    "peak_kind": f"bf16 dense, sustained, {peaks['source']}"}
+    if w.do_qkv:
+        for kind, lt in (("qkv_global", 0), ("qkv_swa", 1)):
+            spec = [L["spec"] for L in w.qkv_layers if L["spec"].layer_type == lt][0]
+            per = statistics.mean(kinds[kind])
+            f = qkv_flops(spec, w.pw.batch, w.pw.seq)
+            parts[kind + "_layer"] = {"ms_per_launch": per, "tflops": f / (per * 1e-3) / 1e12,
+                                      "frac_of_tensor_peak": f / (per * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]}
+        ach = parts["qkv_swa_layer"]["tflops"]
+        roofline = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                    "frac": ach / peaks["bf16_tflops_sustained"], "traffic": None,
+                    "kernel": "qkv_proj_kernel (sliding layer: 14848 features, B4 S32768, hidden 4096)",
                     "peak_kind": f"bf16 dense, sustained, {peaks['source']}"}
     if w.do_decode:
         per = statistics.mean(kinds["decode_stack"])

@@ -37,6 +37,8 @@ EXPORTED = (
     "mimo_attn_decode_workspace_size",
     "mimo_attn_decode",
     "mimo_attn_decode_static",
+    "mimo_attn_qkv_project_workspace_size",
+    "mimo_attn_qkv_project",
     "mimo_attn_decode_fp8kv_workspace_size",
     "mimo_attn_decode_fp8kv",
     "mimo_attn_quantize_fp8",
@@ -100,6 +102,10 @@ def load() -> ctypes.CDLL:
     lib.mimo_attn_decode_static.argtypes = [lp, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp]
     lib.mimo_attn_decode_static.restype = i32
     f32 = ctypes.c_float
+    lib.mimo_attn_qkv_project_workspace_size.argtypes = [lp, i32, i32, i32]
+    lib.mimo_attn_qkv_project_workspace_size.restype = sz
+    lib.mimo_attn_qkv_project.argtypes = [lp, i32, i32, vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, vp, sz, vp]
+    lib.mimo_attn_qkv_project.restype = i32
     lib.mimo_attn_decode_fp8kv_workspace_size.argtypes = [lp, i32, i32]
     lib.mimo_attn_decode_fp8kv_workspace_size.restype = sz
     lib.mimo_attn_decode_fp8kv.argtypes = [lp, i32, vp, vp, vp, vp, vp, vp, i32, f32, f32, vp, vp, sz, vp]
@@ -232,6 +238,20 @@ def mimo_attn_decode_static(layer: mimo_attn_layer, dtype: int, batch: int, q, k
         _ptr(k_cache), _ptr(v_cache), int(cache_capacity), _ptr(out), _stream(stream)))
 
 
+def mimo_attn_qkv_project_workspace_size(layer: mimo_attn_layer, batch: int, seq: int, max_past_len: int) -> int:
+    return int(load().mimo_attn_qkv_project_workspace_size(ctypes.byref(layer), batch, seq, int(max_past_len)))
+
+
+def mimo_attn_qkv_project(layer: mimo_attn_layer, batch: int, seq: int, x, w_qkv, past_lens, max_past_len: int,
+                          q_out, k_out, v_out, k_cache, v_cache, cache_capacity: int, workspace=None,
+                          workspace_bytes: int = 0, stream=None) -> int:
+    """Same arguments as the C entry point; tensors (or None) in place of pointers."""
+    return int(load().mimo_attn_qkv_project(
+        ctypes.byref(layer), batch, seq, _ptr(x), _ptr(w_qkv), _ptr(past_lens), int(max_past_len), _ptr(q_out),
+        _ptr(k_out), _ptr(v_out), _ptr(k_cache), _ptr(v_cache), int(cache_capacity), _ptr(workspace),
+        int(workspace_bytes), _stream(stream)))
+
+
 def mimo_attn_decode_fp8kv_workspace_size(layer: mimo_attn_layer, batch: int, cache_capacity: int) -> int:
     return int(load().mimo_attn_decode_fp8kv_workspace_size(ctypes.byref(layer), batch, cache_capacity))
 
@@ -361,3 +381,26 @@ def quantize_fp8(src: torch.Tensor, scale: float, out: Optional[torch.Tensor] = 
         out = torch.empty(src.shape, dtype=torch.uint8, device=src.device)
     _check(mimo_attn_quantize_fp8(src, out, src.numel(), scale, stream), "mimo_attn_quantize_fp8")
     return out
+
+
+def qkv_project(layer: mimo_attn_layer, x: torch.Tensor, w_qkv: torch.Tensor, past_lens: Optional[torch.Tensor] = None,
+                max_past_len: Optional[int] = None, k_cache: Optional[torch.Tensor] = None,
+                v_cache: Optional[torch.Tensor] = None, want_kv: bool = True, stream=None):
+    """Runs mimo_attn_qkv_project on x [B, S, hidden]: returns (q, k, v) with q
+    and k rotated ([B, S, H, D]; k and v are None when want_kv is False) and
+    fills the caches when given. max_past_len defaults to max(past_lens), read
+    on the host."""
+    B, S = x.shape[0], x.shape[1]
+    if max_past_len is None:
+        max_past_len = int(past_lens.max().item()) if past_lens is not None and past_lens.numel() else 0
+    q = torch.empty((B, S, layer.num_q_heads, layer.qk_dim), dtype=x.dtype, device=x.device)
+    k = v = None
+    if want_kv:
+        k = torch.empty((B, S, layer.num_kv_heads, layer.qk_dim), dtype=x.dtype, device=x.device)
+        v = torch.empty((B, S, layer.num_kv_heads, layer.v_dim), dtype=x.dtype, device=x.device)
+    need = mimo_attn_qkv_project_workspace_size(layer, B, S, max_past_len)
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    cap = 0 if k_cache is None else k_cache.shape[1]
+    _check(mimo_attn_qkv_project(layer, B, S, x, w_qkv, past_lens, max_past_len, q, k, v, k_cache, v_cache, cap,
+                                 ws, ws.numel(), stream), "mimo_attn_qkv_project")
+    return q, k, v

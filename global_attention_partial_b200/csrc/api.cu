@@ -408,6 +408,74 @@ mimo_attn_status mimo_attn_decode(const mimo_attn_layer *layer, int dtype, int b
     return e == cudaSuccess ? MIMO_ATTN_OK : MIMO_ATTN_ERR_CUDA;
 }
 
+size_t mimo_attn_qkv_project_workspace_size(const mimo_attn_layer *layer, int batch, int seq, int max_past_len)
+{
+    mimo::LayerArgs L;
+    if (resolve_layer(layer, MIMO_ATTN_BF16, &L) != MIMO_ATTN_OK || batch < 0 || seq < 0 || max_past_len < 0)
+        return 0;
+    // the RoPE table of positions 0 .. max_past + seq - 1
+    return round_up(((size_t)max_past_len + seq) * L.rope.half * sizeof(float2), 256);
+}
+
+mimo_attn_status mimo_attn_qkv_project(const mimo_attn_layer *layer, int batch, int seq, const void *x,
+                                       const void *w_qkv, const int32_t *past_lens, int max_past_len, void *q_out,
+                                       void *k_out, void *v_out, void *k_cache, void *v_cache, int cache_capacity,
+                                       void *workspace, size_t workspace_bytes, void *stream)
+{
+    mimo::LayerArgs L;
+    mimo_attn_status st = resolve_layer(layer, MIMO_ATTN_BF16, &L);
+    if (st != MIMO_ATTN_OK)
+        return st;
+    if (batch < 0 || seq < 0 || max_past_len < 0)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (past_lens == nullptr && max_past_len != 0)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if ((k_cache == nullptr) != (v_cache == nullptr))
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (k_cache != nullptr) {
+        if (L.layer_type == MIMO_ATTN_SWA && cache_capacity != L.window)
+            return MIMO_ATTN_ERR_INVALID_ARG;
+        if (L.layer_type == MIMO_ATTN_GLOBAL && (cache_capacity < 1 || (long long)max_past_len + seq > cache_capacity))
+            return MIMO_ATTN_ERR_INVALID_ARG;
+    }
+    if (!mimo::qkv_proj_supported(L, layer->hidden_size))
+        return MIMO_ATTN_ERR_UNSUPPORTED;
+    if (batch == 0 || seq == 0)
+        return MIMO_ATTN_OK;
+    if (x == nullptr || w_qkv == nullptr || q_out == nullptr)
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    if (!(aligned16(x) && aligned16(w_qkv) && aligned16(q_out) && aligned16(k_out) && aligned16(v_out) &&
+          aligned16(k_cache) && aligned16(v_cache)))
+        return MIMO_ATTN_ERR_INVALID_ARG;
+    const size_t need = mimo_attn_qkv_project_workspace_size(layer, batch, seq, max_past_len);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+        return MIMO_ATTN_ERR_WORKSPACE;
+    if (g_fail_launches)
+        return MIMO_ATTN_ERR_CUDA;
+    unsigned *err = device_error_ptr();
+    if (err == nullptr)
+        return MIMO_ATTN_ERR_CUDA;
+    mimo::QkvArgs a;
+    memset(&a, 0, sizeof(a));
+    a.x = x;
+    a.w = w_qkv;
+    a.past_lens = past_lens;
+    a.max_past = max_past_len;
+    a.q = q_out;
+    a.k = k_out;
+    a.v = v_out;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.cap = cache_capacity;
+    a.B = batch;
+    a.S = seq;
+    a.hidden = layer->hidden_size;
+    a.rope_table = L.rope.half > 0 ? static_cast<float2 *>(workspace) : nullptr;
+    a.err = err;
+    cudaError_t e = mimo::launch_qkv_proj(L, a, num_sms(), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MIMO_ATTN_OK : MIMO_ATTN_ERR_CUDA;
+}
+
 size_t mimo_attn_decode_fp8kv_workspace_size(const mimo_attn_layer *layer, int batch, int cache_capacity)
 {
     return mimo_attn_decode_workspace_size(layer, MIMO_ATTN_BF16, batch, cache_capacity);

@@ -136,6 +136,26 @@ struct DecodeArgs {
     int fp8_cache;
     float k_scale, v_scale;
 };
+// QKV projection with the fused RoPE / store epilogue (csrc/qkv_proj.cu).
+// x [B*S, hidden] and w [Hq*Dqk + Hkv*(Dqk+Dv), hidden] bf16; q [B, S, Hq,
+// Dqk], k / v [B, S, Hkv, D] (k, v may be null), caches as in the cached
+// prefill (both or neither). rope_table: max_past + S rows of 32 (cos, sin)
+// pairs, filled here.
+struct QkvArgs {
+    const void *x;
+    const void *w;
+    const int *past_lens;  // nullptr: position = sequence index
+    int max_past;
+    void *q, *k, *v;
+    void *k_cache, *v_cache;
+    int cap;
+    int B, S, hidden;
+    float2 *rope_table;
+    unsigned *err;
+};
+bool qkv_proj_supported(const LayerArgs &L, int hidden);
+cudaError_t launch_qkv_proj(const LayerArgs &L, const QkvArgs &a, int num_sms, cudaStream_t stream);
+
 // dst[i] = e4m3(src[i] / scale) (bf16 in, E4M3 codes out; nearest, saturating).
 cudaError_t launch_quantize_e4m3(const void *src, void *dst, size_t n, float scale, cudaStream_t stream);
 int decode_chunk_keys(const LayerArgs &L, int dtype);

@@ -28,11 +28,13 @@ def _mix(seed: int, tensor_id: int) -> int:
     return z & ((1 << 63) - 1)
 
 
-def normal(shape, *, seed: int, tensor_id: int, dtype=torch.bfloat16, device="cpu") -> torch.Tensor:
-    """N(0,1) tensor of `shape`, rounded to `dtype`, drawn on `device`."""
+def normal(shape, *, seed: int, tensor_id: int, dtype=torch.bfloat16, device="cpu", std: float = 1.0) -> torch.Tensor:
+    """N(0, std^2) tensor of `shape`, rounded to `dtype`, drawn on `device`."""
     g = torch.Generator(device=device)
     g.manual_seed(_mix(seed, tensor_id))
     x = torch.randn(tuple(shape), generator=g, device=device, dtype=torch.float32)
+    if std != 1.0:
+        x = x * std
     return x if dtype == torch.float32 else x.to(dtype)
 
 
@@ -44,7 +46,7 @@ def uniform_int(n: int, lo: int, hi: int, *, seed: int, tensor_id: int) -> torch
 
 
 # tensor ids: layer l uses 16*l + role
-ROLE_Q, ROLE_K, ROLE_V, ROLE_SINK, ROLE_KCACHE, ROLE_VCACHE, ROLE_KNEW, ROLE_VNEW, ROLE_LENS = range(9)
+ROLE_Q, ROLE_K, ROLE_V, ROLE_SINK, ROLE_KCACHE, ROLE_VCACHE, ROLE_KNEW, ROLE_VNEW, ROLE_LENS, ROLE_X, ROLE_WQKV = range(11)
 
 
 def tensor_id(layer: int, role: int) -> int:
@@ -171,3 +173,15 @@ def cached_prefill_inputs(spec: LayerSpec, batch: int, seq: int, capacity: int, 
 def decode_kv_lens(batch: int, lo: int, hi: int, *, seed: int) -> torch.Tensor:
     """KV lengths (counting the new token) uniform in [lo, hi], int32 on the CPU."""
     return uniform_int(batch, lo, hi, seed=seed, tensor_id=tensor_id(255, ROLE_LENS))
+
+
+def projection_inputs(spec: LayerSpec, batch: int, seq: int, *, seed: int, layer: int, device="cpu"):
+    """(x, w_qkv) for the QKV projection of one layer: hidden states x
+    [batch, seq, hidden] N(0,1) and the stacked weight [Hq*Dqk + Hkv*(Dqk+Dv),
+    hidden] N(0, 1/hidden) (the usual fan-in initialisation scale, so the
+    projections come out near N(0,1)), both bf16."""
+    x = normal((batch, seq, spec.hidden_size), seed=seed, tensor_id=tensor_id(layer, ROLE_X), device=device)
+    n = spec.num_q_heads * spec.qk_dim + spec.num_kv_heads * (spec.qk_dim + spec.v_dim)
+    w = normal((n, spec.hidden_size), seed=seed, tensor_id=tensor_id(layer, ROLE_WQKV), device=device,
+               std=spec.hidden_size ** -0.5)
+    return x, w

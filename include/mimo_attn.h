@@ -215,6 +215,43 @@ MIMO_ATTN_API mimo_attn_status mimo_attn_decode_static(const mimo_attn_layer *la
                                          const int32_t *kv_lens, void *k_cache, void *v_cache,
                                          int cache_capacity, void *out, void *stream);
 
+/* Bytes of workspace mimo_attn_qkv_project needs: the RoPE cos/sin table of
+ * positions 0 .. max_past_len + seq - 1. */
+MIMO_ATTN_API size_t mimo_attn_qkv_project_workspace_size(const mimo_attn_layer *layer, int batch, int seq,
+                                                          int max_past_len);
+
+/* The step before attention, fused: the QKV projection of a chunk of tokens
+ * with partial RoPE and the cache write in its epilogue.
+ *   y = x W^T with W = w_qkv (no bias), then y's columns split into Hq query
+ *   heads of Dqk, Hkv key heads of Dqk and Hkv value heads of Dv; query and
+ *   key heads get the layer's partial RoPE at the token's position ("Add
+ *   Xiaomi MiMo-V2", "Additional useful info"); values pass through.
+ *   x      [batch, seq, hidden_size] bf16.
+ *   w_qkv  [Hq*Dqk + Hkv*Dqk + Hkv*Dv, hidden_size] bf16: the rows of W_q,
+ *          then W_k, then W_v, each in a linear layer's [out, in] layout.
+ *   past_lens: device int32 [batch] or NULL (= all 0): token t of sequence b
+ *          sits at position past_lens[b] + t. max_past_len >= every entry
+ *          (0 when past_lens is NULL); an entry outside [0, max_past_len]
+ *          sets MIMO_ATTN_DEVERR_KV_LEN and that sequence is skipped.
+ *   q_out  [batch, seq, Hq, Dqk] bf16: rotated queries (required).
+ *   k_out  [batch, seq, Hkv, Dqk] rotated keys, v_out [batch, seq, Hkv, Dv]
+ *          values: optional (NULL = not stored).
+ *   k_cache, v_cache: optional, both or neither, laid out as in
+ *          mimo_attn_prefill_cached (GLOBAL: linear, cache_capacity >=
+ *          max_past_len + seq; SWA: ring, cache_capacity == window, which
+ *          receives the chunk's last `window` tokens).
+ * The outputs are rotated already: attention over them takes a copy of the
+ * layer with rotary_dim = 0 (mimo_attn_prefill, or decode-time reads of the
+ * caches, which always hold rotated keys).
+ * Supported: bf16; Dqk and Dv multiples of 64; rotary_dim 0 or 64;
+ * hidden_size a multiple of 64 (else MIMO_ATTN_ERR_UNSUPPORTED). Pointers
+ * 16-byte aligned; 32-byte aligned outputs take 32-byte stores. */
+MIMO_ATTN_API mimo_attn_status mimo_attn_qkv_project(const mimo_attn_layer *layer, int batch, int seq,
+                                                     const void *x, const void *w_qkv, const int32_t *past_lens,
+                                                     int max_past_len, void *q_out, void *k_out, void *v_out,
+                                                     void *k_cache, void *v_cache, int cache_capacity,
+                                                     void *workspace, size_t workspace_bytes, void *stream);
+
 /* Bytes of workspace mimo_attn_decode_fp8kv needs (the same split-KV partial
  * results as the bf16 decode). */
 MIMO_ATTN_API size_t mimo_attn_decode_fp8kv_workspace_size(const mimo_attn_layer *layer, int batch,

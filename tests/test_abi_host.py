@@ -246,3 +246,37 @@ def test_decode_fp8kv_argument_checks(lib):
         assert mimo.mimo_attn_quantize_fp8(T(), T(), 10, 1.0, 0) == mimo.ERR_CUDA
     finally:
         mimo.mimo_attn_debug_fail_launches(False)
+
+
+def qkv_status(l, batch=2, seq=64, past=True, max_past=10, caches=False, cap=None, ws=1 << 30, kv=True):
+    if cap is None:
+        cap = l.window if l.layer_type == mimo.SWA else max_past + seq
+    return mimo.mimo_attn_qkv_project(l, batch, seq, T(), T(), T() if past else None, max_past, T(),
+                                      T() if kv else None, T() if kv else None, T() if caches else None,
+                                      T() if caches else None, cap, T(), ws, 0)
+
+
+def test_qkv_project_argument_checks(lib):
+    mimo.mimo_attn_debug_fail_launches(True)
+    try:
+        swa = layer()
+        ga = layer(layer_type=mimo.GLOBAL, num_kv_heads=4)
+        assert qkv_status(ga, past=False) == mimo.ERR_INVALID_ARG             # max_past without past_lens
+        assert qkv_status(ga, past=False, max_past=0) == mimo.ERR_CUDA
+        assert qkv_status(swa, caches=True, cap=64) == mimo.ERR_INVALID_ARG  # ring must equal the window
+        assert qkv_status(ga, caches=True, cap=10 + 64 - 1) == mimo.ERR_INVALID_ARG
+        assert qkv_status(ga, caches=True) == mimo.ERR_CUDA
+        assert qkv_status(ga, max_past=-1) == mimo.ERR_INVALID_ARG
+        assert qkv_status(layer(rotary_dim=32)) == mimo.ERR_UNSUPPORTED     # the epilogue rotates 64 or 0 dims
+        assert qkv_status(layer(hidden_size=4000)) == mimo.ERR_UNSUPPORTED  # hidden not a multiple of 64
+        assert qkv_status(layer(qk_dim=96, rotary_dim=32)) == mimo.ERR_UNSUPPORTED
+        assert qkv_status(ga, batch=0) == mimo.OK
+        assert qkv_status(ga, seq=0) == mimo.OK
+        assert qkv_status(ga, ws=100) == mimo.ERR_WORKSPACE
+        assert qkv_status(ga, kv=False) == mimo.ERR_CUDA
+        assert qkv_status(swa) == mimo.ERR_CUDA
+        # the RoPE table of positions 0 .. max_past + seq - 1
+        assert mimo.mimo_attn_qkv_project_workspace_size(ga, 2, 64, 10) == 256 * math.ceil(74 * 32 * 8 / 256)
+        assert mimo.mimo_attn_qkv_project_workspace_size(layer(rotary_dim=0), 2, 64, 10) == 0
+    finally:
+        mimo.mimo_attn_debug_fail_launches(False)
