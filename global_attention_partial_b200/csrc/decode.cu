@@ -72,6 +72,7 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v)
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 constexpr int kDecodeStages = 2;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kDecodeStagesFp8 = 3;  // 20 KB landing tiles: 2 in flight while one is computed
 static_assert(DecodeCfg<kDecodeStagesFp8, true>::kSmemBytes <= 110 * 1024, "2 CTAs per SM");
 
@@ -178,37 +179,59 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
     const int n_tiles = (key_end - key_begin + kTileKeys - 1) / kTileKeys;
     const uint8_t *kc8 = reinterpret_cast<const uint8_t *>(a.k_cache) + ((size_t)b * a.cap * kv_row + kvh) * kDqk;
     const uint8_t *vc8 = reinterpret_cast<const uint8_t *>(a.v_cache) + ((size_t)b * a.cap * kv_row + kvh) * kDv;
+    // Each thread copies a fixed pattern of 16-byte chunks in every tile, so
+    // the shared-memory offsets are compile-time steps from one base and only
+    // the key rows change per tile. Rows past the range and the new token's
+    // slot are zero-filled (the new token comes from its own copy).
+    // bf16: K rows are 24 chunks: thread (key kr + 16i, chunk kch + 8j); V rows
+    // are 16 chunks: thread (key vr + 8i, chunk vch).
+    // fp8: K rows are 12 chunks: thread (key fr + 32i, chunk fch + 4j); V rows
+    // are 8 chunks: thread (key gr + 16i, chunk gch). The widening below walks
+    // the same chunks, so a thread only widens what it copied itself.
+    const int kr = tid >> 3, kch = tid & 7;
+    const int vr = tid >> 4, vch = tid & 15;
+    const int fr = tid >> 2, fch = tid & 3;
+    const int gr = tid >> 3, gch = tid & 7;
+    const size_t k_rstride = kv_row * kDqk;  // elements (bf16) or bytes (fp8) between key rows
+    const size_t v_rstride = kv_row * kDv;
+    auto row_of = [&](int key) { return (size_t)(key < key_end && key != slot_new ? key : key_begin); };
+    auto ok_of = [&](int key) { return key < key_end && key != slot_new ? 16u : 0u; };
     auto issue = [&](int t) {
         const int base_key = key_begin + t * kTileKeys;
         if (kFp8) {
-            // 20 chunks of 16 bytes per key: 12 of K, 8 of V
             uint8_t *land = sLand + (t % kStages) * kLandBytes;
-            for (int c = tid; c < kTileKeys * 20; c += kThreads) {
-                const int r = c / 20;
-                const int ch = c - r * 20;
-                const int key = base_key + r;
-                const bool valid = key < key_end && key != slot_new;
-                const size_t ks = (size_t)(valid ? key : key_begin) * kv_row;
-                const uint8_t *src = ch < 12 ? kc8 + ks * kDqk + ch * 16 : vc8 + ks * kDv + (ch - 12) * 16;
-                cp_async16(land + r * kLandRow + ch * 16, src, valid ? 16u : 0u);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int key = base_key + fr + 32 * i;
+                const uint8_t *src = kc8 + row_of(key) * k_rstride + fch * 16;
+                const uint32_t n = ok_of(key);
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+                    cp_async16(land + (fr + 32 * i) * kLandRow + (fch + 4 * j) * 16, src + j * 64, n);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int key = base_key + gr + 16 * i;
+                cp_async16(land + (gr + 16 * i) * kLandRow + kDqk + gch * 16,
+                           vc8 + row_of(key) * v_rstride + gch * 16, ok_of(key));
             }
             return;
         }
         __nv_bfloat16 *st = sStage + (t % kStages) * kStageElems;
-        for (int c = tid; c < kTileKeys * 40; c += kThreads) {
-            const int r = c / 40;
-            const int ch = c - r * 40;
-            const int key = base_key + r;
-            const bool valid = key < key_end && key != slot_new;
-            const int ks = valid ? key : key_begin;
-            if (ch < 24) {
-                cp_async16(st + r * kKStride + ch * 8, kc + (size_t)ks * kv_row * kDqk + ch * 8,
-                           valid ? 16u : 0u);
-            } else {
-                const int cv = ch - 24;
-                cp_async16(st + kTileKeys * kKStride + r * kVStride + cv * 8,
-                           vc + (size_t)ks * kv_row * kDv + cv * 8, valid ? 16u : 0u);
-            }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int key = base_key + kr + 16 * i;
+            const __nv_bfloat16 *src = kc + row_of(key) * k_rstride + kch * 8;
+            const uint32_t n = ok_of(key);
+#pragma unroll
+            for (int j = 0; j < 3; ++j)
+                cp_async16(st + (kr + 16 * i) * kKStride + (kch + 8 * j) * 8, src + j * 64, n);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int key = base_key + vr + 8 * i;
+            cp_async16(st + kTileKeys * kKStride + (vr + 8 * i) * kVStride + vch * 8,
+                       vc + row_of(key) * v_rstride + vch * 8, ok_of(key));
         }
     };
 #pragma unroll
@@ -374,28 +397,34 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
             issue(t + kStages - 1);
         cp_async_commit();
         cp_async_wait<kStages - 1>();
-        __syncthreads();
         __nv_bfloat16 *st = kFp8 ? sStage : sStage + (t % kStages) * kStageElems;
         const int base_key = key_begin + t * kTileKeys;
         if (kFp8) {
-            // widen the landed e4m3 tile into the padded f16 compute tile
+            // widen this thread's own landed e4m3 chunks (complete after its
+            // wait) into the padded f16 compute tile
             const uint8_t *land = sLand + (t % kStages) * kLandBytes;
-            for (int c = tid; c < kTileKeys * 20; c += kThreads) {
-                const int r = c / 20;
-                const int ch = c - r * 20;
-                const uint4 w = *reinterpret_cast<const uint4 *>(land + r * kLandRow + ch * 16);
+            auto widen = [&](const uint8_t *src, __nv_bfloat16 *dst) {
+                const uint4 w = *reinterpret_cast<const uint4 *>(src);
                 uint4 h0, h1;
                 e4m3x4_to_f16x4(w.x, h0.x, h0.y);
                 e4m3x4_to_f16x4(w.y, h0.z, h0.w);
                 e4m3x4_to_f16x4(w.z, h1.x, h1.y);
                 e4m3x4_to_f16x4(w.w, h1.z, h1.w);
-                uint4 *dst = reinterpret_cast<uint4 *>(
-                    ch < 12 ? st + r * kKStride + ch * 16 : st + kTileKeys * kKStride + r * kVStride + (ch - 12) * 16);
-                dst[0] = h0;
-                dst[1] = h1;
-            }
-            __syncthreads();
+                reinterpret_cast<uint4 *>(dst)[0] = h0;
+                reinterpret_cast<uint4 *>(dst)[1] = h1;
+            };
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+                    widen(land + (fr + 32 * i) * kLandRow + (fch + 4 * j) * 16,
+                          st + (fr + 32 * i) * kKStride + (fch + 4 * j) * 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                widen(land + (gr + 16 * i) * kLandRow + kDqk + gch * 16,
+                      st + kTileKeys * kKStride + (gr + 16 * i) * kVStride + gch * 16);
         }
+        __syncthreads();
         if (owns_new && slot_new >= base_key && slot_new < base_key + kTileKeys) {
             const int r = slot_new - base_key;
             if (tid < 24)
@@ -423,14 +452,16 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
                 mma16<kFp8>(s_acc[1], qa[ks], b2, b3);
             }
         }
-        // Scale, mask keys past the end of the range, online softmax.
+        // Scale, mask keys past the end of the range (only the range's last
+        // tile has any), online softmax.
         float mx0 = -INFINITY, mx1 = -INFINITY;
+        const bool full_tile = base_key + kTileKeys <= key_end;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int key = base_key + kb + nt * 8 + 2 * tq + e;
-                const bool valid = key < key_end;
+                const bool valid = full_tile || key < key_end;
                 s_acc[nt][e] = valid ? s_acc[nt][e] * L.scale_log2 : -INFINITY;
                 s_acc[nt][2 + e] = valid ? s_acc[nt][2 + e] * L.scale_log2 : -INFINITY;
                 mx0 = fmaxf(mx0, s_acc[nt][e]);
@@ -441,14 +472,20 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float mn0 = fmaxf(m0, mx0);
-        const float mn1 = fmaxf(m1, mx1);
-        const float c0 = (mn0 == -INFINITY) ? 1.f : exp2f(m0 - mn0);
-        const float c1 = (mn1 == -INFINITY) ? 1.f : exp2f(m1 - mn1);
-        const float u0 = (mn0 == -INFINITY) ? 0.f : mn0;
-        const float u1 = (mn1 == -INFINITY) ? 0.f : mn1;
-        m0 = mn0;
-        m1 = mn1;
+        // The reference max of a row only moves when the block's max exceeds
+        // it by more than 2^8 (probabilities stay <= 256, exact in the 16-bit
+        // operand types), so O is rescaled rarely: m and l always describe the
+        // same reference, and the merge / combine use them as they are.
+        const bool up0 = mx0 > m0 + kRescaleThreshold || (m0 == -INFINITY && mx0 > -INFINITY);
+        const bool up1 = mx1 > m1 + kRescaleThreshold || (m1 == -INFINITY && mx1 > -INFINITY);
+        const float c0 = up0 && m0 != -INFINITY ? exp2f(m0 - mx0) : 1.f;
+        const float c1 = up1 && m1 != -INFINITY ? exp2f(m1 - mx1) : 1.f;
+        if (up0)
+            m0 = mx0;
+        if (up1)
+            m1 = mx1;
+        const float u0 = (m0 == -INFINITY) ? 0.f : m0;
+        const float u1 = (m1 == -INFINITY) ? 0.f : m1;
         float p[2][4];
         float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
@@ -462,12 +499,14 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
         }
         l0 = l0 * c0 + rs0;
         l1 = l1 * c1 + rs1;
+        if (__any_sync(0xffffffffu, c0 != 1.f || c1 != 1.f)) {
 #pragma unroll
-        for (int d = 0; d < 16; ++d) {
-            o[d][0] *= c0;
-            o[d][1] *= c0;
-            o[d][2] *= c1;
-            o[d][3] *= c1;
+            for (int d = 0; d < 16; ++d) {
+                o[d][0] *= c0;
+                o[d][1] *= c0;
+                o[d][2] *= c1;
+                o[d][3] *= c1;
+            }
         }
         uint32_t pa[4];
         pa[0] = pack16<kFp8>(p[0][0], p[0][1]);
