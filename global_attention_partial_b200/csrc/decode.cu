@@ -33,32 +33,24 @@ constexpr int kChunkKeys = 2048;    // keys per split on global layers
 constexpr int kStageElems = kTileKeys * (kKStride + kVStride);
 // Ring depth x CTAs per SM: the bytes in flight per SM, (stages - 1) x 43 KB x
 // CTAs, must cover the HBM latency at full bandwidth.
-// fp8 (E4M3) caches: a tile lands as dense 320-byte rows (K then V), then is
-// widened to f16 into one padded compute tile (e4m3 values are exact in f16).
+// fp8 (E4M3) caches: each warp streams its own 16 keys of every tile as dense
+// 320-byte rows (K then V) through a private ring and builds its mma operands
+// straight from those bytes (every E4M3 value is exact in f16), so the loop
+// has no CTA barrier and no widening pass.
 constexpr int kLandRow = kDqk + kDv;             // bytes per key
-constexpr int kLandBytes = kTileKeys * kLandRow;  // 20480
-// With fp8 caches the query rows are staged in the compute tile (they are
-// read into registers before the first tile is widened there), so a 3-deep
-// landing ring still leaves room for 2 CTAs per SM.
+constexpr int kWarpLand = 16 * kLandRow;         // one warp's 16 keys: 5120
+constexpr int kLandBytes = kTileKeys * kLandRow;  // one stage of the CTA: 20480
 template <int ST, bool F8 = false> struct DecodeCfg {
-    static constexpr int kSmemBytes = F8 ? (kStageElems + kDqk + kDv) * 2 + ST * kLandBytes
+    static constexpr int kSmemBytes = F8 ? (16 * kQStride + kDqk + kDv) * 2 + kLandRow + ST * kLandBytes
                                          : (16 * kQStride + ST * kStageElems + kDqk + kDv) * 2;
-    static constexpr int kCtasPerSm = (F8 ? ST <= 3 : ST <= 2) ? 2 : 1;
+    static constexpr int kCtasPerSm = (F8 ? ST <= 4 : ST <= 2) ? 2 : 1;
 };
-static_assert(16 * kQStride <= kStageElems, "query rows fit in the compute tile");
 
 // 16-bit operand type of the tensor-core path: bf16 for bf16 caches, f16 for
 // fp8 caches (their e4m3 values, the f16 query and the probabilities).
 template <bool F8> __device__ __forceinline__ uint32_t pack16(float lo, float hi)
 {
     return F8 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
-}
-template <bool F8> __device__ __forceinline__ void mma16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
-{
-    if (F8)
-        mma_f16_16816(d, a, b0, b1);
-    else
-        mma_bf16_16816(d, a, b0, b1);
 }
 // 8 bf16 (a 16-byte chunk) as 8 f16.
 __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v)
@@ -73,7 +65,7 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v)
 }
 constexpr int kDecodeStages = 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kDecodeStagesFp8 = 3;  // 20 KB landing tiles: 2 in flight while one is computed
+constexpr int kDecodeStagesFp8 = 4;  // 5 KB per warp and stage: 3 tiles in flight while one is computed
 static_assert(DecodeCfg<kDecodeStagesFp8, true>::kSmemBytes <= 110 * 1024, "2 CTAs per SM");
 
 struct DecodeSmem {
@@ -84,6 +76,7 @@ struct DecodeSmem {
 // reuse the stage buffers: 4 x 16 rows x 136 floats = 34 KB.
 constexpr int kMergeStride = kDv + 8;
 static_assert(4 * 16 * kMergeStride * 4 <= kStageElems * 2, "merge slices fit in one stage buffer");
+static_assert(4 * 16 * kMergeStride * 4 <= kDecodeStagesFp8 * kLandBytes, "merge slices fit in the fp8 rings");
 
 __device__ __forceinline__ int visible_count(int layer_type, int Lb, int window)
 {
@@ -100,12 +93,16 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
     decode_mma_kernel(const __grid_constant__ LayerArgs L, const __grid_constant__ DecodeArgs a)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    // 16-bit elements: bf16, or f16 bits with fp8 caches
-    __nv_bfloat16 *sStage = reinterpret_cast<__nv_bfloat16 *>(smem_raw) + (kFp8 ? 0 : 16 * kQStride);
-    __nv_bfloat16 *sQ = kFp8 ? sStage : reinterpret_cast<__nv_bfloat16 *>(smem_raw);
-    __nv_bfloat16 *sKnew = sStage + (kFp8 ? 1 : kStages) * kStageElems;
+    // Query rows: bf16, or f16 with fp8 caches. bf16: then the K/V stage
+    // ring and the raw new k/v. fp8: the raw new k/v, the new token's codes
+    // (K then V) and the per-warp landing rings (warp w, stage s at
+    // (w * kStages + s) * kWarpLand).
+    __nv_bfloat16 *sQ = reinterpret_cast<__nv_bfloat16 *>(smem_raw);
+    __nv_bfloat16 *sStage = sQ + 16 * kQStride;
+    __nv_bfloat16 *sKnew = sStage + (kFp8 ? 0 : kStages * kStageElems);
     __nv_bfloat16 *sVnew = sKnew + kDqk;
-    uint8_t *sLand = reinterpret_cast<uint8_t *>(sVnew + kDv);  // fp8 landing tiles (kFp8 only)
+    uint8_t *sNew8 = reinterpret_cast<uint8_t *>(sVnew + kDv);
+    uint8_t *sLand = sNew8 + kLandRow;
     __shared__ DecodeSmem red;
 
     const int tid = threadIdx.x;
@@ -185,13 +182,12 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
     // slot are zero-filled (the new token comes from its own copy).
     // bf16: K rows are 24 chunks: thread (key kr + 16i, chunk kch + 8j); V rows
     // are 16 chunks: thread (key vr + 8i, chunk vch).
-    // fp8: K rows are 12 chunks: thread (key fr + 32i, chunk fch + 4j); V rows
-    // are 8 chunks: thread (key gr + 16i, chunk gch). The widening below walks
-    // the same chunks, so a thread only widens what it copied itself.
+    // fp8, per warp and its 16 keys: K rows are 12 chunks: lane (key fr + 8i,
+    // chunk fch + 4j); V rows are 8 chunks: lane (key gr + 4i, chunk gch).
     const int kr = tid >> 3, kch = tid & 7;
     const int vr = tid >> 4, vch = tid & 15;
-    const int fr = tid >> 2, fch = tid & 3;
-    const int gr = tid >> 3, gch = tid & 7;
+    const int fr = lane >> 2, fch = lane & 3;
+    const int gr = lane >> 3, gch = lane & 7;
     const size_t k_rstride = kv_row * kDqk;  // elements (bf16) or bytes (fp8) between key rows
     const size_t v_rstride = kv_row * kDv;
     auto row_of = [&](int key) { return (size_t)(key < key_end && key != slot_new ? key : key_begin); };
@@ -199,20 +195,21 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
     auto issue = [&](int t) {
         const int base_key = key_begin + t * kTileKeys;
         if (kFp8) {
-            uint8_t *land = sLand + (t % kStages) * kLandBytes;
+            const int wkey = base_key + warp * 16;
+            uint8_t *land = sLand + (warp * kStages + t % kStages) * kWarpLand;
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
-                const int key = base_key + fr + 32 * i;
+                const int key = wkey + fr + 8 * i;
                 const uint8_t *src = kc8 + row_of(key) * k_rstride + fch * 16;
                 const uint32_t n = ok_of(key);
 #pragma unroll
                 for (int j = 0; j < 3; ++j)
-                    cp_async16(land + (fr + 32 * i) * kLandRow + (fch + 4 * j) * 16, src + j * 64, n);
+                    cp_async16(land + (fr + 8 * i) * kLandRow + (fch + 4 * j) * 16, src + j * 64, n);
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int key = base_key + gr + 16 * i;
-                cp_async16(land + (gr + 16 * i) * kLandRow + kDqk + gch * 16,
+                const int key = wkey + gr + 4 * i;
+                cp_async16(land + (gr + 4 * i) * kLandRow + kDqk + gch * 16,
                            vc8 + row_of(key) * v_rstride + gch * 16, ok_of(key));
             }
             return;
@@ -337,11 +334,11 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
         __syncthreads();  // every raw element read before any is overwritten
         if (tid < kDqk / 2) {
             reinterpret_cast<uint16_t *>(kdst)[tid] = kq;
-            reinterpret_cast<uint32_t *>(sKnew)[tid] = e4m3x2_to_f16x2(kq);
+            reinterpret_cast<uint16_t *>(sNew8)[tid] = kq;
         }
         if (tid < kDv / 2) {
             reinterpret_cast<uint16_t *>(vdst)[tid] = vq;
-            reinterpret_cast<uint32_t *>(sVnew)[tid] = e4m3x2_to_f16x2(vq);
+            reinterpret_cast<uint16_t *>(sNew8 + kDqk)[tid] = vq;
         }
     } else if (owns_new) {
         __nv_bfloat16 *kdst = reinterpret_cast<__nv_bfloat16 *>(a.k_cache) +
@@ -368,9 +365,25 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
     }
     __syncthreads();
 
-    // Query fragments (A operand, 16 heads x 192) for the 12 k-steps.
+    const int g = lane >> 2;  // row (head) g and g + 8
+    const int tq = lane & 3;
+    // Query fragments (A operand, 16 heads x 192) for the 12 k-steps. fp8:
+    // the QK dot product runs over a permutation of the 192 dims that lets a
+    // lane read its key operands as whole words: in k-step ks, lane (g, tq)
+    // holds dims tq*48 + 4*ks + {0, 1} (fragment k = 2tq, 2tq+1) and
+    // tq*48 + 4*ks + {2, 3} (k = 2tq+8, 2tq+9), for the query as for the key.
     uint32_t qa[12][4];
-    {
+    if constexpr (kFp8) {
+        const uint32_t *q0 = reinterpret_cast<const uint32_t *>(sQ + g * kQStride + tq * 48);
+        const uint32_t *q1 = reinterpret_cast<const uint32_t *>(sQ + (g + 8) * kQStride + tq * 48);
+#pragma unroll
+        for (int ks = 0; ks < 12; ++ks) {
+            qa[ks][0] = q0[2 * ks];
+            qa[ks][1] = q1[2 * ks];
+            qa[ks][2] = q0[2 * ks + 1];
+            qa[ks][3] = q1[2 * ks + 1];
+        }
+    } else {
         const int mi = lane >> 3;
         const int r = (lane & 7) + (mi & 1) * 8;
         const uint32_t base = smem_u32(sQ) + (uint32_t)(r * kQStride + (mi >> 1) * 8) * 2u;
@@ -378,9 +391,6 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
         for (int ks = 0; ks < 12; ++ks)
             ldmatrix_x4(base + ks * 32, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
     }
-
-    const int g = lane >> 2;  // row (head) g and g + 8
-    const int tq = lane & 3;
     float m0 = -INFINITY, m1 = -INFINITY;  // running max of rows g, g+8 (base 2)
     float l0 = 0.f, l1 = 0.f;              // this thread's partial sums
     float o[16][4];
@@ -389,58 +399,67 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
         o[d][0] = o[d][1] = o[d][2] = o[d][3] = 0.f;
 
     for (int t = 0; t < n_tiles; ++t) {
-        // Tile t + kStages - 1 goes out before the wait for tile t, so kStages
-        // tiles are in flight during it; the barrier first makes sure every
-        // warp is done with the buffer it refills (that of tile t - 1).
-        __syncthreads();
-        if (t + kStages - 1 < n_tiles)
-            issue(t + kStages - 1);
-        cp_async_commit();
-        cp_async_wait<kStages - 1>();
-        __nv_bfloat16 *st = kFp8 ? sStage : sStage + (t % kStages) * kStageElems;
         const int base_key = key_begin + t * kTileKeys;
-        if (kFp8) {
-            // widen this thread's own landed e4m3 chunks (complete after its
-            // wait) into the padded f16 compute tile
-            const uint8_t *land = sLand + (t % kStages) * kLandBytes;
-            auto widen = [&](const uint8_t *src, __nv_bfloat16 *dst) {
-                const uint4 w = *reinterpret_cast<const uint4 *>(src);
-                uint4 h0, h1;
-                e4m3x4_to_f16x4(w.x, h0.x, h0.y);
-                e4m3x4_to_f16x4(w.y, h0.z, h0.w);
-                e4m3x4_to_f16x4(w.z, h1.x, h1.y);
-                e4m3x4_to_f16x4(w.w, h1.z, h1.w);
-                reinterpret_cast<uint4 *>(dst)[0] = h0;
-                reinterpret_cast<uint4 *>(dst)[1] = h1;
-            };
-#pragma unroll
-            for (int i = 0; i < 2; ++i)
-#pragma unroll
-                for (int j = 0; j < 3; ++j)
-                    widen(land + (fr + 32 * i) * kLandRow + (fch + 4 * j) * 16,
-                          st + (fr + 32 * i) * kKStride + (fch + 4 * j) * 16);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                widen(land + (gr + 16 * i) * kLandRow + kDqk + gch * 16,
-                      st + kTileKeys * kKStride + (gr + 16 * i) * kVStride + gch * 16);
-        }
-        __syncthreads();
-        if (owns_new && slot_new >= base_key && slot_new < base_key + kTileKeys) {
-            const int r = slot_new - base_key;
-            if (tid < 24)
-                *reinterpret_cast<uint4 *>(st + r * kKStride + tid * 8) =
-                    *reinterpret_cast<const uint4 *>(sKnew + tid * 8);
-            else if (tid < 40)
-                *reinterpret_cast<uint4 *>(st + kTileKeys * kKStride + r * kVStride + (tid - 24) * 8) =
-                    *reinterpret_cast<const uint4 *>(sVnew + (tid - 24) * 8);
-            __syncthreads();
-        }
         const int kb = warp * 16;  // this warp's 16 keys within the tile
-        if (base_key + kb >= key_end)
-            continue;
-        // S = Q K^T for 16 heads x 16 keys.
         float s_acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        {
+        const uint8_t *land = nullptr;       // fp8: this warp's landed rows of tile t
+        const __nv_bfloat16 *st = nullptr;   // bf16: the CTA's stage of tile t
+        if constexpr (kFp8) {
+            // The warp refills the ring entry of tile t - 1 once all its lanes
+            // are done with it, then waits for its own copies of tile t.
+            __syncwarp();
+            if (t + kStages - 1 < n_tiles)
+                issue(t + kStages - 1);
+            cp_async_commit();
+            cp_async_wait<kStages - 1>();
+            __syncwarp();
+            if (base_key + kb >= key_end)
+                continue;
+            land = sLand + (warp * kStages + t % kStages) * kWarpLand;
+            if (owns_new && slot_new >= base_key + kb && slot_new < base_key + kb + 16) {
+                if (lane < kLandRow / 16)
+                    *reinterpret_cast<uint4 *>(const_cast<uint8_t *>(land) + (slot_new - base_key - kb) * kLandRow +
+                                               lane * 16) = *reinterpret_cast<const uint4 *>(sNew8 + lane * 16);
+                __syncwarp();
+            }
+            // S = Q K^T: lane (g, tq) reads its 48 key bytes tq*48 .. of key
+            // g (n-tile 0) and 8 + g (n-tile 1); word ks holds the four dims of
+            // k-step ks (low half: b0, high half: b1).
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const uint4 *kr4 = reinterpret_cast<const uint4 *>(land + (nt * 8 + g) * kLandRow + tq * 48);
+                const uint4 w0 = kr4[0], w1 = kr4[1], w2 = kr4[2];
+                const uint32_t kw[12] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w, w2.x, w2.y, w2.z, w2.w};
+#pragma unroll
+                for (int ks = 0; ks < 12; ++ks)
+                    mma_f16_16816(s_acc[nt], qa[ks], e4m3x2_to_f16x2((uint16_t)(kw[ks] & 0xFFFFu)),
+                                  e4m3x2_to_f16x2((uint16_t)(kw[ks] >> 16)));
+            }
+        } else {
+            // Tile t + kStages - 1 goes out before the wait for tile t, so
+            // kStages tiles are in flight during it; the barrier first makes
+            // sure every warp is done with the buffer it refills (tile t - 1's).
+            __syncthreads();
+            if (t + kStages - 1 < n_tiles)
+                issue(t + kStages - 1);
+            cp_async_commit();
+            cp_async_wait<kStages - 1>();
+            __syncthreads();
+            __nv_bfloat16 *stw = sStage + (t % kStages) * kStageElems;
+            if (owns_new && slot_new >= base_key && slot_new < base_key + kTileKeys) {
+                const int r = slot_new - base_key;
+                if (tid < 24)
+                    *reinterpret_cast<uint4 *>(stw + r * kKStride + tid * 8) =
+                        *reinterpret_cast<const uint4 *>(sKnew + tid * 8);
+                else if (tid < 40)
+                    *reinterpret_cast<uint4 *>(stw + kTileKeys * kKStride + r * kVStride + (tid - 24) * 8) =
+                        *reinterpret_cast<const uint4 *>(sVnew + (tid - 24) * 8);
+                __syncthreads();
+            }
+            st = stw;
+            if (base_key + kb >= key_end)
+                continue;
+            // S = Q K^T for 16 heads x 16 keys.
             const int mi = lane >> 3;
             const int key = kb + (mi >> 1) * 8 + (lane & 7);
             const uint32_t base = smem_u32(st) + (uint32_t)(key * kKStride + (mi & 1) * 8) * 2u;
@@ -448,8 +467,8 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
             for (int ks = 0; ks < 12; ++ks) {
                 uint32_t b0, b1, b2, b3;
                 ldmatrix_x4(base + ks * 32, b0, b1, b2, b3);
-                mma16<kFp8>(s_acc[0], qa[ks], b0, b1);
-                mma16<kFp8>(s_acc[1], qa[ks], b2, b3);
+                mma_bf16_16816(s_acc[0], qa[ks], b0, b1);
+                mma_bf16_16816(s_acc[1], qa[ks], b2, b3);
             }
         }
         // Scale, mask keys past the end of the range (only the range's last
@@ -514,7 +533,32 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
         pa[2] = pack16<kFp8>(p[1][0], p[1][1]);
         pa[3] = pack16<kFp8>(p[1][2], p[1][3]);
         // O += P V over these 16 keys.
-        {
+        if constexpr (kFp8) {
+            // Output dims are permuted: n-tile dp, column n holds dim n*16 + dp.
+            // Lane (g, tq) reads value bytes g*16 .. g*16+15 of keys 2tq, 2tq+1
+            // (b0) and 2tq+8, 2tq+9 (b1); prmt pairs the two keys' bytes of one
+            // dim, lower key in the low byte.
+            const uint8_t *vb = land + kDqk + g * 16;
+            const uint4 va = *reinterpret_cast<const uint4 *>(vb + (2 * tq) * kLandRow);
+            const uint4 vb1 = *reinterpret_cast<const uint4 *>(vb + (2 * tq + 1) * kLandRow);
+            const uint4 vc2 = *reinterpret_cast<const uint4 *>(vb + (2 * tq + 8) * kLandRow);
+            const uint4 vd3 = *reinterpret_cast<const uint4 *>(vb + (2 * tq + 9) * kLandRow);
+            const uint32_t A[4] = {va.x, va.y, va.z, va.w}, B[4] = {vb1.x, vb1.y, vb1.z, vb1.w};
+            const uint32_t C[4] = {vc2.x, vc2.y, vc2.z, vc2.w}, D[4] = {vd3.x, vd3.y, vd3.z, vd3.w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const uint32_t lo01 = __byte_perm(A[w], B[w], 0x5140u), hi01 = __byte_perm(C[w], D[w], 0x5140u);
+                const uint32_t lo23 = __byte_perm(A[w], B[w], 0x7362u), hi23 = __byte_perm(C[w], D[w], 0x7362u);
+                mma_f16_16816(o[4 * w], pa, e4m3x2_to_f16x2((uint16_t)(lo01 & 0xFFFFu)),
+                              e4m3x2_to_f16x2((uint16_t)(hi01 & 0xFFFFu)));
+                mma_f16_16816(o[4 * w + 1], pa, e4m3x2_to_f16x2((uint16_t)(lo01 >> 16)),
+                              e4m3x2_to_f16x2((uint16_t)(hi01 >> 16)));
+                mma_f16_16816(o[4 * w + 2], pa, e4m3x2_to_f16x2((uint16_t)(lo23 & 0xFFFFu)),
+                              e4m3x2_to_f16x2((uint16_t)(hi23 & 0xFFFFu)));
+                mma_f16_16816(o[4 * w + 3], pa, e4m3x2_to_f16x2((uint16_t)(lo23 >> 16)),
+                              e4m3x2_to_f16x2((uint16_t)(hi23 >> 16)));
+            }
+        } else {
             const int mi = lane >> 3;
             const int key = kb + (mi & 1) * 8 + (lane & 7);
             const uint32_t base = smem_u32(st + kTileKeys * kKStride) +
@@ -523,8 +567,8 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
             for (int dp = 0; dp < 8; ++dp) {
                 uint32_t b0, b1, b2, b3;
                 ldmatrix_x4_trans(base + dp * 32, b0, b1, b2, b3);
-                mma16<kFp8>(o[2 * dp], pa, b0, b1);
-                mma16<kFp8>(o[2 * dp + 1], pa, b2, b3);
+                mma_bf16_16816(o[2 * dp], pa, b0, b1);
+                mma_bf16_16816(o[2 * dp + 1], pa, b2, b3);
             }
         }
     }
@@ -553,14 +597,24 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
     // Each warp writes its rescaled partial O into its own slice (rows padded
     // to kMergeStride floats: the 8 rows of a warp's access fall in different
     // banks), then one pass sums the four slices.
-    float *slices = reinterpret_cast<float *>(sStage);
+    float *slices = reinterpret_cast<float *>(kFp8 ? sLand : reinterpret_cast<uint8_t *>(sStage));
     {
         float *sl = slices + warp * 16 * kMergeStride;
 #pragma unroll
         for (int d = 0; d < 16; ++d) {
-            const int col = d * 8 + 2 * tq;
-            *reinterpret_cast<float2 *>(sl + g * kMergeStride + col) = make_float2(o[d][0] * f0, o[d][1] * f0);
-            *reinterpret_cast<float2 *>(sl + (g + 8) * kMergeStride + col) = make_float2(o[d][2] * f1, o[d][3] * f1);
+            if constexpr (kFp8) {
+                // undo the output-dim permutation: n-tile d, column n is dim n*16 + d
+                const int c0 = (2 * tq) * 16 + d, c1 = (2 * tq + 1) * 16 + d;
+                sl[g * kMergeStride + c0] = o[d][0] * f0;
+                sl[g * kMergeStride + c1] = o[d][1] * f0;
+                sl[(g + 8) * kMergeStride + c0] = o[d][2] * f1;
+                sl[(g + 8) * kMergeStride + c1] = o[d][3] * f1;
+            } else {
+                const int col = d * 8 + 2 * tq;
+                *reinterpret_cast<float2 *>(sl + g * kMergeStride + col) = make_float2(o[d][0] * f0, o[d][1] * f0);
+                *reinterpret_cast<float2 *>(sl + (g + 8) * kMergeStride + col) =
+                    make_float2(o[d][2] * f1, o[d][3] * f1);
+            }
         }
     }
     __syncthreads();
