@@ -158,6 +158,70 @@ __global__ void kprep_bf16_vec_kernel(const __grid_constant__ KprepArgs a)
     }
 }
 
+// K rows of 192 bf16 (24 chunks of 16 bytes) with rotary_dim 64, rotated
+// into dst_k only (no cache copies): the rows are one flat array of chunks,
+// 32 consecutive chunks per warp, four per thread in flight. A row starts at
+// a multiple of 8 chunks, so its 8 rotary chunks (dims 0-63: chunk c < 4
+// pairs with c + 4) sit in one aligned group of 8 lanes and a lane gets its
+// partner chunk from lane ^ 4 by shuffle.
+constexpr int kKprepChunks = 24;
+constexpr int kKprepUnroll = 4;
+__global__ void kprep_r64_kernel(const __grid_constant__ KprepArgs a)
+{
+    const long long total = (long long)a.B * a.S * a.Hkv * kKprepChunks;
+    const int lane = threadIdx.x & 31;
+    const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.k);
+    uint4 *dst = reinterpret_cast<uint4 *>(a.dst_k);
+    for (long long w = warp0 * kKprepUnroll; w * 32 < total; w += nwarps * kKprepUnroll) {
+        uint4 x[kKprepUnroll];
+#pragma unroll
+        for (int u = 0; u < kKprepUnroll; ++u) {
+            const long long g = (w + u) * 32 + lane;
+            x[u] = g < total ? __ldg(src + g) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kKprepUnroll; ++u) {
+            const long long g = (w + u) * 32 + lane;
+            const long long row = g / kKprepChunks;
+            const int c = (int)(g - row * kKprepChunks);
+            // partner chunk of the rotary half (meaningful for c < 8 only);
+            // every lane takes part in the shuffles
+            uint4 y;
+            y.x = __shfl_xor_sync(0xffffffffu, x[u].x, 4);
+            y.y = __shfl_xor_sync(0xffffffffu, x[u].y, 4);
+            y.z = __shfl_xor_sync(0xffffffffu, x[u].z, 4);
+            y.w = __shfl_xor_sync(0xffffffffu, x[u].w, 4);
+            if (g >= total)
+                continue;
+            const long long bi = row / a.Hkv;
+            const int i = (int)(bi % a.S);
+            const int b = (int)(bi / a.S);
+            const int kv = (int)(row - bi * a.Hkv);
+            uint4 out = x[u];
+            if (c < 8) {
+                const bool first = c < 4;
+                // own dims are 8c.. (first half) or 32 + 8(c-4).. (second half):
+                // pairs 8(c & 3) .. 8(c & 3) + 7
+                const float4 *cs = reinterpret_cast<const float4 *>(a.rope_table + (long long)i * 32 + (c & 3) * 8);
+                const uint32_t *own = reinterpret_cast<const uint32_t *>(&x[u]);
+                const uint32_t *oth = reinterpret_cast<const uint32_t *>(&y);
+                uint32_t *o = reinterpret_cast<uint32_t *>(&out);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float4 cc = __ldg(cs + e);  // (cos, sin) of pairs 2e and 2e + 1 of the chunk
+                    const float2 xa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(first ? &own[e] : &oth[e]));
+                    const float2 xb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(first ? &oth[e] : &own[e]));
+                    o[e] = first ? pack_bf16x2(xa.x * cc.x - xb.x * cc.y, xa.y * cc.z - xb.y * cc.w)
+                                 : pack_bf16x2(xb.x * cc.x + xa.x * cc.y, xb.y * cc.z + xa.y * cc.w);
+                }
+            }
+            dst[(((long long)b * a.dst_rows + i) * a.Hkv + kv) * kKprepChunks + c] = out;
+        }
+    }
+}
+
 template <typename T>
 __global__ void prefill_simt_kernel(const __grid_constant__ LayerArgs L, const __grid_constant__ PrefillArgs a)
 {
@@ -253,6 +317,14 @@ cudaError_t launch_kprep(const KprepArgs &a, int dtype, cudaStream_t stream)
         rope_table_kernel<<<(unsigned)(tb < 4096 ? tb : 4096), 256, 0, stream>>>(a);
     }
     const int threads = 256;
+    if (dtype == kDtypeBf16 && a.rope.rotary_dim == 64 && a.Dqk == 192 && a.ring_k == nullptr &&
+        a.ring_v == nullptr && a.lin_v == nullptr) {
+        const long long warps = (rows * kKprepChunks + 32 * kKprepUnroll - 1) / (32 * kKprepUnroll);
+        const long long need = (warps + threads / 32 - 1) / (threads / 32);
+        const long long cap = 148LL * 16;  // grid-stride beyond 16 blocks per SM
+        kprep_r64_kernel<<<(unsigned)(need < cap ? need : cap), threads, 0, stream>>>(a);
+        return cudaGetLastError();
+    }
     const long long blocks = (rows + (threads / 32) - 1) / (threads / 32);
     const bool vec = dtype == kDtypeBf16 && a.rope.rotary_dim % 16 == 0 && a.Dqk % 8 == 0 && a.Dv % 8 == 0 &&
                      (a.rope.half / 8) + (a.Dqk - a.rope.rotary_dim) / 8 + a.Dv / 8 <= 32 * 64;
