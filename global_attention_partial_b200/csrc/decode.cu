@@ -13,6 +13,11 @@
 //   through shared memory; a sequence with one split is finished in place
 //   (sink folded, V scale applied), otherwise the (m, l, O) partials go to the
 //   workspace and a combine kernel merges them.
+// fp8 (E4M3) caches, same kernel with kFp8: each warp streams its own 16 keys
+//   of every tile through a private cp.async ring and builds its f16 mma
+//   operands from the landed bytes in registers (QK over a permuted order of
+//   the 192 dims, PV with permuted output dims, undone at the merge); the new
+//   token is quantized into its slot and read back as codes.
 // Other dtypes / dims: a CUDA-core path (one warp per query head) after a
 // separate new-token write.
 #include "kernels.cuh"
