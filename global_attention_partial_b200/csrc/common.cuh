@@ -64,20 +64,6 @@ __device__ __forceinline__ float fast_exp2(float x)
     return y;
 }
 
-// 2^a and 2^b from one MUFU operation on f16 arguments: the arguments are
-// rounded to f16 (11-bit significand: at |x| < 16 the result is off by at
-// most a factor 2^(2^-8), 0.27 %, about the bf16 rounding the probabilities
-// get anyway), the results converted back to fp32 exactly. For exponents
-// in [-24, 8] as the softmax kernels produce them; -inf gives 0.
-__device__ __forceinline__ float2 exp2_pair_f16(float a, float b)
-{
-    uint32_t h, e;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(b), "f"(a));
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
-    const __half2 v = *reinterpret_cast<const __half2 *>(&e);
-    return __half22float2(v);
-}
-
 // Branch-free test lo <= c <= hi (one unsigned compare; empty when hi < lo).
 __device__ __forceinline__ bool in_range(int c, int lo, int hi)
 {

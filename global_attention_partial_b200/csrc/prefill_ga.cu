@@ -407,10 +407,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_ga_kernel(const __grid_co
                 uint32_t r[8];
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    // two exponentials per MUFU operation
-                    const float2 e = exp2_pair_f16(fmaf(x[c0 + 2 * c], sc, -m_use), fmaf(x[c0 + 2 * c + 1], sc, -m_use));
-                    rsv[c & 3] += e.x + e.y;
-                    r[c] = pack_bf16x2(e.x, e.y);
+                    const float e0 = fast_exp2(fmaf(x[c0 + 2 * c], sc, -m_use));
+                    const float e1 = fast_exp2(fmaf(x[c0 + 2 * c + 1], sc, -m_use));
+                    rsv[c & 3] += e0 + e1;
+                    r[c] = pack_bf16x2(e0, e1);
                 }
                 tmem_st8(s_addr + c0 / 2, r);
             }

@@ -493,9 +493,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 uint32_t pk[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const float2 ex = exp2_pair_f16(fmaf(x[16 * q + 2 * e], sc, -mu), fmaf(x[16 * q + 2 * e + 1], sc, -mu));
-                    rsv[e & 3] += ex.x + ex.y;
-                    pk[e] = pack_bf16x2(ex.x, ex.y);
+                    const float e0 = fast_exp2(fmaf(x[16 * q + 2 * e], sc, -mu));
+                    const float e1 = fast_exp2(fmaf(x[16 * q + 2 * e + 1], sc, -mu));
+                    rsv[e & 3] += e0 + e1;
+                    pk[e] = pack_bf16x2(e0, e1);
                 }
                 tmem_st8(s_addr + 8 * q, pk);
             }
