@@ -222,3 +222,14 @@ def test_decode_fp8_bad_length_sets_error_and_skips():
     assert torch.equal(kc[1], kc0[1]) and torch.equal(vc[1], vc0[1])
     assert torch.all(out[1] == 0)
     _check_fp8(spec, out, q, kn, vn, kc0, vc0, kc, vc, None, [0], lens)
+
+
+@pytest.mark.parametrize("layer_type", [0, 1])
+def test_decode_fp8_small_groups(layer_type):
+    """G = 2 (global) and G = 4 with a sink (sliding): query rows beyond G in
+    the 16-row mma tile are zero and must not leak into the output."""
+    spec = synthetic.LayerSpec(layer_type, 8 if layer_type == 0 else 16, 4, 192, 128, 64, 128,
+                               5e6 if layer_type == 0 else 1e4, 1024, layer_type == 1)
+    lens = [1, 17, 128, 129, 700]
+    out, (q, kn, vn, kc0, vc0, kc, vc, sinks) = _run_fp8(spec, len(lens), 700, lens, seed=8)
+    _check_fp8(spec, out, q, kn, vn, kc0, vc0, kc, vc, sinks, range(len(lens)), lens)

@@ -147,3 +147,10 @@ def test_qkv_project_bad_past_sets_error_and_skips():
     assert torch.all(q[1] == 0)
     oq, _, _ = _oracle(spec, x[0], w, 3 + np.arange(64), spec.rotary_dim)
     _check(compare(f64(q[0]).ravel(), oq.ravel()), "q of the valid sequence")
+
+
+def test_qkv_project_one_k_block_short_ring():
+    """hidden 64 (a single k-block), three sequences of 40 tokens on a
+    sliding layer whose 128-slot ring is only partly written."""
+    spec = synthetic.LayerSpec(1, 8, 2, 192, 128, 64, 128, 1e4, 64, True)
+    _run_and_check(spec, 3, 40, [0, 100, 7], cap=128)
