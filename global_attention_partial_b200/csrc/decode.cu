@@ -48,7 +48,7 @@ constexpr int kLandBytes = kTileKeys * kLandRow;  // one stage of the CTA: 20480
 template <int ST, bool F8 = false> struct DecodeCfg {
     static constexpr int kSmemBytes = F8 ? (16 * kQStride + kDqk + kDv) * 2 + kLandRow + ST * kLandBytes
                                          : (16 * kQStride + ST * kStageElems + kDqk + kDv) * 2;
-    static constexpr int kCtasPerSm = (F8 ? ST <= 4 : ST <= 2) ? 2 : 1;
+    static constexpr int kCtasPerSm = F8 ? (ST <= 3 ? 3 : 2) : (ST <= 2 ? 2 : 1);
 };
 
 // 16-bit operand type of the tensor-core path: bf16 for bf16 caches, f16 for
@@ -70,8 +70,8 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v)
 }
 constexpr int kDecodeStages = 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kDecodeStagesFp8 = 4;  // 5 KB per warp and stage: 3 tiles in flight while one is computed
-static_assert(DecodeCfg<kDecodeStagesFp8, true>::kSmemBytes <= 110 * 1024, "2 CTAs per SM");
+constexpr int kDecodeStagesFp8 = 3;  // 5 KB per warp and stage; 69 KB per CTA: 3 CTAs (12 warps) per SM
+static_assert(DecodeCfg<kDecodeStagesFp8, true>::kSmemBytes <= 72 * 1024, "3 CTAs per SM");
 
 struct DecodeSmem {
     float wm[4][16];
