@@ -908,18 +908,15 @@ cudaError_t launch_decode(const LayerArgs &L, const DecodeArgs &a, int dtype, cu
     if (a.fp8_cache && !decode_mma_supported(L, dtype))
         return cudaErrorInvalidValue;
     if (decode_mma_supported(L, dtype)) {
-        static bool attr_set[2] = {false, false};
+        static std::atomic<unsigned long long> prepared[2] = {{0}, {0}};
         const int f = a.fp8_cache ? 1 : 0;
-        if (!attr_set[f]) {
-            cudaError_t e = f ? cudaFuncSetAttribute(decode_mma_kernel<kDecodeStagesFp8, true>,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                     DecodeCfg<kDecodeStagesFp8, true>::kSmemBytes)
-                              : cudaFuncSetAttribute(decode_mma_kernel<kDecodeStages, false>,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                     DecodeCfg<kDecodeStages, false>::kSmemBytes);
+        {
+            cudaError_t e = f ? prepare_kernel_once(decode_mma_kernel<kDecodeStagesFp8, true>,
+                                                    DecodeCfg<kDecodeStagesFp8, true>::kSmemBytes, prepared[1])
+                              : prepare_kernel_once(decode_mma_kernel<kDecodeStages, false>,
+                                                    DecodeCfg<kDecodeStages, false>::kSmemBytes, prepared[0]);
             if (e != cudaSuccess)
                 return e;
-            attr_set[f] = true;
         }
         dim3 grid(a.max_splits, L.Hkv, a.B);
         if (f)

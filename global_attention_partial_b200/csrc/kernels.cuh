@@ -3,7 +3,41 @@
 
 #include "common.cuh"
 
+#include <atomic>
+
 namespace mimo {
+
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` once per device
+// (the attribute belongs to the device's copy of the kernel). When
+// `launch_regs` > 0 it first checks that the kernel was compiled with exactly
+// that many registers per thread: the warp-specialised kernels split the
+// block's register pool with setmaxnreg and must not launch with a smaller
+// one. `done` is one bit per device ordinal (< 64), shared by the host
+// threads that call the launcher.
+template <typename K>
+inline cudaError_t prepare_kernel_once(K kernel, int bytes, std::atomic<unsigned long long> &done, int launch_regs = 0)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit)
+        return cudaSuccess;
+    if (launch_regs > 0) {
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, kernel);
+        if (e != cudaSuccess)
+            return e;
+        if (fa.numRegs != launch_regs)
+            return cudaErrorInvalidConfiguration;
+    }
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess)
+        done.fetch_or(bit, std::memory_order_release);
+    return e;
+}
+
 
 enum { kDtypeBf16 = 0, kDtypeFp32 = 1 };
 

@@ -498,20 +498,11 @@ cudaError_t launch_prefill_ga(const LayerArgs &L, const PrefillArgs &a, cudaStre
     p.scale_log2 = L.scale_log2;
     p.v_scale = L.v_scale;
 
-    static bool attr_set = false;
-    if (!attr_set) {
-        // The setmaxnreg split needs a launch with exactly kLaunchRegs registers.
-        cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, prefill_ga_kernel);
-        if (e != cudaSuccess)
-            return e;
-        if (fa.numRegs != kLaunchRegs)
-            return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(prefill_ga_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess)
-            return e;
-        attr_set = true;
-    }
+    // The setmaxnreg split needs a launch with exactly kLaunchRegs registers.
+    static std::atomic<unsigned long long> prepared{0};
+    cudaError_t e = prepare_kernel_once(prefill_ga_kernel, kSmemBytes, prepared, kLaunchRegs);
+    if (e != cudaSuccess)
+        return e;
     dim3 grid(p.num_p_tiles, p.num_pairs, a.B);
     prefill_ga_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p);
     return cudaGetLastError();

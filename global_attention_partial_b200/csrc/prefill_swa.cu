@@ -618,22 +618,13 @@ cudaError_t launch_prefill_swa(const LayerArgs &L, const PrefillArgs &a, const f
     p.scale_log2 = L.scale_log2;
     p.v_scale = L.v_scale;
 
-    static bool attr_set = false;
-    if (!attr_set) {
-        // The setmaxnreg split assumes the block launches with exactly
-        // kLaunchRegs registers per thread; refuse to launch otherwise (a
-        // smaller pool would leave setmaxnreg.inc waiting forever).
-        cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, prefill_swa_kernel);
-        if (e != cudaSuccess)
-            return e;
-        if (fa.numRegs != kLaunchRegs)
-            return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(prefill_swa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess)
-            return e;
-        attr_set = true;
-    }
+    // The setmaxnreg split assumes the block launches with exactly
+    // kLaunchRegs registers per thread; refuse to launch otherwise (a smaller
+    // pool would leave setmaxnreg.inc waiting forever).
+    static std::atomic<unsigned long long> prepared{0};
+    cudaError_t e = prepare_kernel_once(prefill_swa_kernel, kSmemBytes, prepared, kLaunchRegs);
+    if (e != cudaSuccess)
+        return e;
     const int grid = (p.num_tiles + p.tiles_per_cta - 1) / p.tiles_per_cta;
     prefill_swa_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p);
     return cudaGetLastError();

@@ -501,15 +501,10 @@ cudaError_t launch_prefill_tc(const LayerArgs &L, const PrefillArgs &a, cudaStre
     p.v_scale = L.v_scale;
     p.rope = L.rope;
 
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<kBN, kStages>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             TileCfg<kBN, kStages>::kSmemBytes);
-        if (e != cudaSuccess)
-            return e;
-        attr_set = true;
-    }
+    static std::atomic<unsigned long long> prepared{0};
+    cudaError_t e = prepare_kernel_once(prefill_tc_kernel<kBN, kStages>, TileCfg<kBN, kStages>::kSmemBytes, prepared);
+    if (e != cudaSuccess)
+        return e;
     dim3 grid(p.num_p_tiles, L.Hkv * p.num_g_tiles, a.B);
     prefill_tc_kernel<kBN, kStages><<<grid, kThreads, TileCfg<kBN, kStages>::kSmemBytes, stream>>>(p);
     return cudaGetLastError();

@@ -336,13 +336,10 @@ cudaError_t launch_qkv_proj(const LayerArgs &L, const QkvArgs &a, int num_sms, c
     p.v_cache = reinterpret_cast<__nv_bfloat16 *>(a.v_cache);
     p.v8 = aligned32(a.q) && aligned32(a.k) && aligned32(a.v) && aligned32(a.k_cache) && aligned32(a.v_cache);
     p.err = a.err;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(qkv_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess)
-            return e;
-        attr_set = true;
-    }
+    static std::atomic<unsigned long long> prepared{0};
+    cudaError_t e = prepare_kernel_once(qkv_proj_kernel, kSmemBytes, prepared);
+    if (e != cudaSuccess)
+        return e;
     const long long tiles = (long long)p.tiles_m * p.tiles_n;
     const int grid = (int)(tiles < num_sms ? tiles : num_sms);
     qkv_proj_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p);
