@@ -64,12 +64,6 @@ __device__ __forceinline__ float fast_exp2(float x)
     return y;
 }
 
-// Branch-free test lo <= c <= hi (one unsigned compare; empty when hi < lo).
-__device__ __forceinline__ bool in_range(int c, int lo, int hi)
-{
-    return (unsigned)(c - lo) <= (unsigned)(hi - lo) && hi >= lo;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -132,20 +126,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     uint32_t ok;
     asm volatile("{\n\t.reg .pred p;\n\t"
                  "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}\n"
-                 : "=r"(ok)
-                 : "r"(smem_u32(bar)), "r"(parity)
-                 : "memory");
-    return ok != 0;
-}
-
-// Non-blocking probe of a phase (never suspends the thread): for polling
-// loops that must not stall on one barrier while another is ready.
-__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
                  "selp.u32 %0, 1, 0, p;\n\t}\n"
                  : "=r"(ok)
                  : "r"(smem_u32(bar)), "r"(parity)
@@ -216,22 +196,6 @@ __device__ __forceinline__ void tma_load_4d(void *smem_dst, const CUtensorMap *m
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
         "r"(smem_u32(bar))
         : "memory");
-}
-
-// Prefetch of one tensor box into L2 (no shared memory, no completion
-// signal): starts the DRAM read of a tile that a later load will need.
-__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-                 : "memory");
-}
-
-// Prefetch of `bytes` (a multiple of 16) contiguous global bytes into L2.
-__device__ __forceinline__ void prefetch_l2_bulk(const void *gmem, uint32_t bytes)
-{
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem), "r"(bytes) : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05
@@ -520,13 +484,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes)
     uint32_t r;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(codes));
     return r;
-}
-
-// Four E4M3 codes of a 32-bit word to two f16x2 words (elements 0-1, 2-3).
-__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t &lo, uint32_t &hi)
-{
-    lo = e4m3x2_to_f16x2((uint16_t)(w & 0xFFFFu));
-    hi = e4m3x2_to_f16x2((uint16_t)(w >> 16));
 }
 
 // Nearest E4M3 codes of two floats (round to nearest even, saturating at
