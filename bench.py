@@ -466,15 +466,46 @@ def oracle_sample(seconds: float, seed: int = 1, kind: str = "stack"):
     oracle.build()
     rng = np.random.default_rng(seed)
     flops, t_total, rows_done, groups_done = 0.0, 0.0, 0, 0
-    pw = {"stack": synthetic.HYBRID_PREFILL, "swa": synthetic.SWA_PREFILL,
-          "global": synthetic.GLOBAL_PREFILL}.get(kind)
-    dw = synthetic.HYBRID_DECODE if kind in ("stack", "decode") else None
+    if kind not in ("stack", "swa", "global", "decode", "decode_fp8", "chunked", "qkv"):
+        raise ValueError(f"no oracle sample for workload {kind!r}")
+    pw = {"stack": synthetic.HYBRID_PREFILL, "swa": synthetic.SWA_PREFILL, "global": synthetic.GLOBAL_PREFILL,
+          "chunked": synthetic.HYBRID_PREFILL}.get(kind)
+    dw = synthetic.HYBRID_DECODE if kind in ("stack", "decode", "decode_fp8") else None
+    fp8 = kind == "decode_fp8"
+    # chunked: query rows are the stack's last CHUNK_SEQ positions
+    row_lo = CHUNK_PAST if kind == "chunked" else 0
+    tables = {}
+
+    def e4m3_of(x, scale):
+        # the oracle's codes of bf16 values, through one table over all 65536 patterns
+        if scale not in tables:
+            with np.errstate(all="ignore"):
+                quot = (np.arange(65536, dtype=np.uint32) << 16).view(np.float32) / np.float32(scale)
+            tables[scale] = oracle.e4m3_encode(np.nan_to_num(quot, nan=0.0).astype(np.float64))
+        return tables[scale][x.view(torch.int16).numpy().astype(np.int64) & 0xFFFF]
+
+    proj = None
+    if kind == "qkv":
+        spec = synthetic.HYBRID_PREFILL.layers[0]
+        x16, w16 = synthetic.projection_inputs(spec, 1, 16, seed=seed, layer=0)
+        proj = (spec, x16[0].double().numpy(), w16.double().numpy())
     t_start = time.perf_counter()
     while time.perf_counter() - t_start < seconds:
+        if proj is not None:
+            from threadpoolctl import threadpool_limits
+            spec, x, w = proj
+            with threadpool_limits(limits=1):  # one core, like the C oracle
+                t0 = time.perf_counter()
+                oracle.qkv_project(x, w, np.arange(x.shape[0]), num_q_heads=spec.num_q_heads,
+                                   num_kv_heads=spec.num_kv_heads, qk_dim=spec.qk_dim, v_dim=spec.v_dim,
+                                   rotary_dim=spec.rotary_dim, theta=spec.theta)
+                t_total += time.perf_counter() - t0
+            flops += 2.0 * x.shape[0] * w.shape[0] * x.shape[1]
+            rows_done += x.shape[0]
         if pw is not None:
             for li, spec in enumerate(pw.layers):
                 S = pw.seq
-                i = int(rng.integers(0, S))
+                i = int(rng.integers(row_lo, S))
                 lo = 0 if spec.layer_type == 0 else max(0, i - spec.window + 1)
                 n = i - lo + 1
                 k = synthetic.normal((n, spec.qk_dim), seed=seed, tensor_id=1000 + li, dtype=torch.bfloat16)
@@ -500,16 +531,27 @@ def oracle_sample(seconds: float, seed: int = 1, kind: str = "stack"):
                 kn = synthetic.normal((spec.qk_dim,), seed=seed, tensor_id=7000 + li, dtype=torch.bfloat16)
                 vn = synthetic.normal((spec.v_dim,), seed=seed, tensor_id=8000 + li, dtype=torch.bfloat16)
                 sinks = np.zeros(G) if spec.has_sink else None
-                t0 = time.perf_counter()
-                oracle.decode(q.double().numpy(), kn.double().numpy(), vn.double().numpy(), kc.double().numpy(),
-                              vc.double().numpy(), L, spec.rotary_dim, spec.theta, spec.layer_type, spec.window,
-                              1 / math.sqrt(spec.qk_dim), sinks, 0.7)
+                if fp8:
+                    kc8, vc8 = e4m3_of(kc, 1 / 16), e4m3_of(vc, 1 / 32)
+                    t0 = time.perf_counter()
+                    oracle.decode_fp8kv(q.double().numpy(), kn.double().numpy(), vn.double().numpy(), kc8, vc8, L,
+                                        spec.rotary_dim, spec.theta, spec.layer_type, spec.window,
+                                        1 / math.sqrt(spec.qk_dim), sinks, 0.7, 1 / 16, 1 / 32)
+                else:
+                    t0 = time.perf_counter()
+                    oracle.decode(q.double().numpy(), kn.double().numpy(), vn.double().numpy(), kc.double().numpy(),
+                                  vc.double().numpy(), L, spec.rotary_dim, spec.theta, spec.layer_type, spec.window,
+                                  1 / math.sqrt(spec.qk_dim), sinks, 0.7)
                 t_total += time.perf_counter() - t0
                 flops += G * (min(L, spec.window) if spec.layer_type == 1 else L) * 2 * (spec.qk_dim + spec.v_dim)
                 groups_done += 1
-    desc = (f"{rows_done} prefill query rows (uniform positions, all visible keys, every layer of the stack) "
-            f"+ {groups_done} decode KV groups (one sequence, all query heads of the group); "
-            f"fp64 C oracle, single thread")
+    if proj is not None:
+        desc = (f"{rows_done} tokens of the global layer's QKV projection (all 13568 features, RoPE); "
+                f"fp64 oracle (numpy matmul on one BLAS thread)")
+    else:
+        desc = (f"{rows_done} prefill query rows (uniform positions{' in the chunk' if row_lo else ''}, all visible "
+                f"keys, every layer of the stack) + {groups_done} decode KV groups (one sequence, all query heads "
+                f"of the group{', E4M3 caches' if fp8 else ''}); fp64 C oracle, single thread")
     return flops, t_total, desc
 
 
@@ -627,9 +669,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="launch the decode layers one call at a time")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
-    if args.workload in ("chunked", "decode_fp8", "qkv"):  # NEXT-row measurements: kernels only, no host or oracle legs
+    if args.workload in ("chunked", "decode_fp8", "qkv"):  # NEXT-row measurements: no host-buffer leg
         args.no_e2e = True
-        args.no_cpu_baseline = True
     if args.impl == "reference":
         run_reference(args)
         return
