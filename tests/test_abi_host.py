@@ -280,3 +280,17 @@ def test_qkv_project_argument_checks(lib):
         assert mimo.mimo_attn_qkv_project_workspace_size(layer(rotary_dim=0), 2, 64, 10) == 0
     finally:
         mimo.mimo_attn_debug_fail_launches(False)
+
+
+def test_python_conveniences_check_dtypes(lib):
+    """decode_fp8kv wants uint8 caches and quantize_fp8 wants bf16 input; both
+    refuse before touching the device."""
+    import torch
+    l = layer()
+    q = torch.zeros((1, 64, 192), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        mimo.decode_fp8kv(l, q, q[:, :8], q[:, :8, :128], torch.ones(1, dtype=torch.int32),
+                          torch.zeros((1, 128, 8, 192), dtype=torch.bfloat16),
+                          torch.zeros((1, 128, 8, 128), dtype=torch.uint8), 1.0, 1.0)
+    with pytest.raises(ValueError):
+        mimo.quantize_fp8(torch.zeros(8, dtype=torch.float32), 1.0)
