@@ -183,7 +183,11 @@ CHUNK_PAST, CHUNK_SEQ = 28672, 4096
 class StackWorkload:
     """Device-resident inputs, outputs, caches and workspaces of the step."""
 
-    def __init__(self, kind: str, seed: int = 0):
+    def __init__(self, kind: str, seed: int = 0, layers=None, batch=None, seq=None):
+        """layers: indices of the workload's layers to keep (all by default);
+        batch / seq: override the prefill batch and length (prefill and
+        projection workloads), e.g. to profile one kernel on a smaller case."""
+        import dataclasses
         import global_attention_partial_b200 as mimo
         self.mimo = mimo
         self.kind = kind
@@ -194,6 +198,15 @@ class StackWorkload:
             pw = synthetic.SWA_PREFILL
         elif kind == "global":
             pw = synthetic.GLOBAL_PREFILL
+        if layers is not None:
+            pw = dataclasses.replace(pw, layers=tuple(pw.layers[i] for i in layers if i < len(pw.layers)))
+            dw = dataclasses.replace(dw, layers=tuple(dw.layers[i] for i in layers if i < len(dw.layers)))
+        if batch is not None:
+            pw = dataclasses.replace(pw, batch=batch)
+        if seq is not None:
+            pw = dataclasses.replace(pw, seq=seq)
+        # seeds follow each layer's index in the full workload
+        self.layer_ids = list(layers) if layers is not None else list(range(len(synthetic.HYBRID_PATTERN)))
         self.do_prefill = kind in ("stack", "swa", "global")
         self.do_decode = kind in ("stack", "decode", "decode_fp8")
         self.fp8 = kind == "decode_fp8"
@@ -204,7 +217,7 @@ class StackWorkload:
         self.prefill_layers = []
         if self.do_prefill:
             B, S = pw.batch, pw.seq
-            for li, spec in enumerate(pw.layers):
+            for li, spec in zip(self.layer_ids, pw.layers):
                 q, k, v, sinks = synthetic.prefill_inputs(spec, B, S, seed=seed, layer=li, device=dev)
                 sinks = sinks if spec.layer_type == 1 else None
                 lay = mimo.make_layer(spec.layer_type, spec.num_q_heads, spec.num_kv_heads, spec.qk_dim,
@@ -221,7 +234,7 @@ class StackWorkload:
         if self.do_chunked:
             B, S, P = pw.batch, CHUNK_SEQ, CHUNK_PAST
             self.past_dev = torch.full((B,), P, dtype=torch.int32, device=dev)
-            for li, spec in enumerate(pw.layers):
+            for li, spec in zip(self.layer_ids, pw.layers):
                 q, k, v, kc, vc, sinks = synthetic.cached_prefill_inputs(spec, B, S, P + S, seed=seed, layer=li,
                                                                          device=dev)
                 sinks = sinks if spec.layer_type == 1 else None
@@ -244,7 +257,7 @@ class StackWorkload:
             kv_heads = max(s.num_kv_heads for s in pw.layers)
             self.qkv_k = torch.empty((B, S, kv_heads, spec0.qk_dim), dtype=torch.bfloat16, device=dev)
             self.qkv_v = torch.empty((B, S, kv_heads, spec0.v_dim), dtype=torch.bfloat16, device=dev)
-            for li, spec in enumerate(pw.layers):
+            for li, spec in zip(self.layer_ids, pw.layers):
                 _, w = synthetic.projection_inputs(spec, 1, 1, seed=seed, layer=li, device=dev)
                 lay = mimo.make_layer(spec.layer_type, spec.num_q_heads, spec.num_kv_heads, spec.qk_dim,
                                       spec.v_dim, spec.rotary_dim, spec.window, spec.theta, spec.hidden_size, None)
@@ -259,7 +272,7 @@ class StackWorkload:
             B = dw.batch
             self.lens = synthetic.decode_kv_lens(B, *dw.kv_len_range, seed=seed).tolist()
             lens_dev = torch.tensor(self.lens, dtype=torch.int32, device=dev)
-            for li, spec in enumerate(dw.layers):
+            for li, spec in zip(self.layer_ids, dw.layers):
                 q, kn, vn, kc, vc, sinks = synthetic.decode_inputs(spec, B, dw.seq, torch.tensor(self.lens),
                                                                    seed=seed, layer=100 + li, device=dev)
                 sinks = sinks if spec.layer_type == 1 else None
@@ -457,23 +470,139 @@ class HostInputs:
 
 
 # ------------------------------------------------------------------ oracle
-def oracle_sample(seconds: float, seed: int = 1, kind: str = "stack"):
-    """Times the fp64 oracle on a bounded sample of the workload: for every
-    prefill layer, query rows at uniform positions against their whole
-    visible key range; for every decode layer, one KV group of one sequence.
-    Returns (unmasked FLOPs done, seconds, description)."""
+def host_cores() -> int:
+    """Cores this process may run on (the oracle's thread count)."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
+def cpu_model() -> str:
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.lower().startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _run_parallel(tasks, threads: int, seconds: float = None):
+    """Runs the callables of `tasks` (an iterator; each returns its FLOPs) on
+    `threads` host threads, until the iterator ends or, when `seconds` is
+    given, until that much wall time has passed (tasks already started
+    finish). The oracle's C routines release the GIL, so the threads run on
+    separate cores. Returns (FLOPs, wall seconds, tasks run)."""
+    from concurrent.futures import FIRST_COMPLETED, ThreadPoolExecutor, wait
+    flops, n = 0.0, 0
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        live = set()
+        it = iter(tasks)
+        exhausted = False
+        while True:
+            while not exhausted and len(live) < 2 * threads and (
+                    seconds is None or time.perf_counter() - t0 < seconds):
+                try:
+                    live.add(ex.submit(next(it)))
+                except StopIteration:
+                    exhausted = True
+            if not live:
+                break
+            done, live = wait(live, return_when=FIRST_COMPLETED)
+            for f in done:
+                flops += f.result()
+                n += 1
+            if seconds is not None and time.perf_counter() - t0 >= seconds:
+                exhausted = True
+    return flops, time.perf_counter() - t0, n
+
+
+class _OracleInputs:
+    """Host copies of synthetic inputs for the oracle's timing runs, drawn
+    once per layer kind before the clock starts (values N(0,1) rounded to
+    bf16, as on the device)."""
+
+    def __init__(self, seed: int):
+        self.seed = seed
+        self.cache = {}
+
+    def get(self, key, shape, tid):
+        if key not in self.cache:
+            self.cache[key] = synthetic.normal(shape, seed=self.seed, tensor_id=tid,
+                                               dtype=torch.bfloat16).double().numpy()
+        return self.cache[key]
+
+
+def _prefill_row_task(inp, spec, S, i, li):
+    """One query row of one head: rotate its visible keys and the query, attend."""
+    import oracle
+    lo = 0 if spec.layer_type == 0 else max(0, i - spec.window + 1)
+    k = inp.get(("k", spec.layer_type, S), (S, spec.qk_dim), 1000 + spec.layer_type)
+    v = inp.get(("v", spec.layer_type, S), (S, spec.v_dim), 2000 + spec.layer_type)
+    q = inp.get(("q", spec.layer_type), (64, spec.qk_dim), 3000 + spec.layer_type)
+
+    def run():
+        pos = np.arange(lo, i + 1, dtype=np.float64)
+        kr = oracle.rope(k[lo:i + 1], spec.rotary_dim, spec.theta, pos)
+        qr = oracle.rope(q[li % 64:li % 64 + 1], spec.rotary_dim, spec.theta, [float(i)])
+        oracle.prefill_rows(qr, [i - lo], kr, v[lo:i + 1], spec.layer_type, spec.window,
+                            1 / math.sqrt(spec.qk_dim), 0.5 if spec.has_sink else None, 0.7)
+        return (i - lo + 1) * 2.0 * (spec.qk_dim + spec.v_dim)
+    return run
+
+
+def _decode_group_task(inp, spec, L, li, fp8, e4m3_of):
+    """One KV group of one sequence: the G query heads against the cache."""
+    import oracle
+    cap = spec.window if spec.layer_type == 1 else 32768
+    G = spec.num_q_heads // spec.num_kv_heads
+    kc = inp.get(("kc", spec.layer_type), (cap, spec.qk_dim), 4000 + spec.layer_type)
+    vc = inp.get(("vc", spec.layer_type), (cap, spec.v_dim), 5000 + spec.layer_type)
+    q = inp.get(("dq", spec.layer_type), (G, spec.qk_dim), 6000 + spec.layer_type)
+    kn = inp.get(("kn", spec.layer_type), (spec.qk_dim,), 7000 + spec.layer_type)
+    vn = inp.get(("vn", spec.layer_type), (spec.v_dim,), 8000 + spec.layer_type)
+    sinks = np.zeros(G) if spec.has_sink else None
+    c = cap if spec.layer_type == 1 else L
+    if fp8:
+        for key, src, scale in ((("kc8", spec.layer_type), kc, 1 / 16), (("vc8", spec.layer_type), vc, 1 / 32)):
+            if key not in inp.cache:
+                inp.cache[key] = e4m3_of(src, scale)
+        kc8, vc8 = inp.cache[("kc8", spec.layer_type)], inp.cache[("vc8", spec.layer_type)]
+
+    def run():
+        if fp8:
+            oracle.decode_fp8kv(q, kn, vn, kc8[:c], vc8[:c], L, spec.rotary_dim, spec.theta, spec.layer_type,
+                                spec.window, 1 / math.sqrt(spec.qk_dim), sinks, 0.7, 1 / 16, 1 / 32)
+        else:
+            oracle.decode(q, kn, vn, kc[:c], vc[:c], L, spec.rotary_dim, spec.theta, spec.layer_type,
+                          spec.window, 1 / math.sqrt(spec.qk_dim), sinks, 0.7)
+        n = min(L, spec.window) if spec.layer_type == 1 else L
+        return G * n * 2.0 * (spec.qk_dim + spec.v_dim)
+    return run
+
+
+def oracle_sample(seconds: float, seed: int = 1, kind: str = "stack", threads: int = None):
+    """Times the fp64 oracle, threaded over all host cores, on a bounded
+    sample of the workload: for every prefill layer in turn, query rows at
+    uniform positions against their whole visible key range; for every
+    decode layer, one KV group of one sequence of uniform length. Inputs are
+    drawn before the clock starts. Returns (unmasked FLOPs done, wall
+    seconds, description, threads)."""
     import oracle
     oracle.build()
-    rng = np.random.default_rng(seed)
-    flops, t_total, rows_done, groups_done = 0.0, 0.0, 0, 0
+    threads = threads or host_cores()
     if kind not in ("stack", "swa", "global", "decode", "decode_fp8", "chunked", "qkv"):
         raise ValueError(f"no oracle sample for workload {kind!r}")
+    rng = np.random.default_rng(seed)
     pw = {"stack": synthetic.HYBRID_PREFILL, "swa": synthetic.SWA_PREFILL, "global": synthetic.GLOBAL_PREFILL,
           "chunked": synthetic.HYBRID_PREFILL}.get(kind)
     dw = synthetic.HYBRID_DECODE if kind in ("stack", "decode", "decode_fp8") else None
     fp8 = kind == "decode_fp8"
-    # chunked: query rows are the stack's last CHUNK_SEQ positions
-    row_lo = CHUNK_PAST if kind == "chunked" else 0
+    row_lo = CHUNK_PAST if kind == "chunked" else 0  # chunked: rows in the stack's last CHUNK_SEQ positions
+    inp = _OracleInputs(seed)
     tables = {}
 
     def e4m3_of(x, scale):
@@ -482,84 +611,63 @@ def oracle_sample(seconds: float, seed: int = 1, kind: str = "stack"):
             with np.errstate(all="ignore"):
                 quot = (np.arange(65536, dtype=np.uint32) << 16).view(np.float32) / np.float32(scale)
             tables[scale] = oracle.e4m3_encode(np.nan_to_num(quot, nan=0.0).astype(np.float64))
-        return tables[scale][x.view(torch.int16).numpy().astype(np.int64) & 0xFFFF]
+        bits = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().astype(np.int64) & 0xFFFF
+        return tables[scale][bits]
 
-    proj = None
     if kind == "qkv":
+        from threadpoolctl import threadpool_limits
         spec = synthetic.HYBRID_PREFILL.layers[0]
-        x16, w16 = synthetic.projection_inputs(spec, 1, 16, seed=seed, layer=0)
-        proj = (spec, x16[0].double().numpy(), w16.double().numpy())
-    t_start = time.perf_counter()
-    while time.perf_counter() - t_start < seconds:
-        if proj is not None:
-            from threadpoolctl import threadpool_limits
-            spec, x, w = proj
-            with threadpool_limits(limits=1):  # one core, like the C oracle
-                t0 = time.perf_counter()
+        x16, w16 = synthetic.projection_inputs(spec, 1, 64, seed=seed, layer=0)
+        x, w = x16[0].double().numpy(), w16.double().numpy()
+        flops, rows = 0.0, 0
+        with threadpool_limits(limits=threads):  # numpy's BLAS on every core
+            t0 = time.perf_counter()
+            while time.perf_counter() - t0 < seconds:
                 oracle.qkv_project(x, w, np.arange(x.shape[0]), num_q_heads=spec.num_q_heads,
                                    num_kv_heads=spec.num_kv_heads, qk_dim=spec.qk_dim, v_dim=spec.v_dim,
                                    rotary_dim=spec.rotary_dim, theta=spec.theta)
-                t_total += time.perf_counter() - t0
-            flops += 2.0 * x.shape[0] * w.shape[0] * x.shape[1]
-            rows_done += x.shape[0]
-        if pw is not None:
-            for li, spec in enumerate(pw.layers):
-                S = pw.seq
-                i = int(rng.integers(row_lo, S))
-                lo = 0 if spec.layer_type == 0 else max(0, i - spec.window + 1)
-                n = i - lo + 1
-                k = synthetic.normal((n, spec.qk_dim), seed=seed, tensor_id=1000 + li, dtype=torch.bfloat16)
-                v = synthetic.normal((n, spec.v_dim), seed=seed, tensor_id=2000 + li, dtype=torch.bfloat16)
-                q = synthetic.normal((1, spec.qk_dim), seed=seed, tensor_id=3000 + li, dtype=torch.bfloat16)
-                pos = np.arange(lo, i + 1, dtype=np.float64)
-                t0 = time.perf_counter()
-                kr = oracle.rope(k.double().numpy(), spec.rotary_dim, spec.theta, pos)
-                qr = oracle.rope(q.double().numpy(), spec.rotary_dim, spec.theta, [float(i)])
-                oracle.prefill_rows(qr, [n - 1], kr, v.double().numpy(), spec.layer_type, spec.window,
-                                    1 / math.sqrt(spec.qk_dim), 0.5 if spec.has_sink else None, 0.7)
-                t_total += time.perf_counter() - t0
-                flops += n * 2 * (spec.qk_dim + spec.v_dim)
-                rows_done += 1
-        if dw is not None:
-            for li, spec in enumerate(dw.layers):
-                L = int(rng.integers(dw.kv_len_range[0], dw.kv_len_range[1] + 1))
-                cap = spec.window if spec.layer_type == 1 else L
-                G = spec.num_q_heads // spec.num_kv_heads
-                kc = synthetic.normal((cap, spec.qk_dim), seed=seed, tensor_id=4000 + li, dtype=torch.bfloat16)
-                vc = synthetic.normal((cap, spec.v_dim), seed=seed, tensor_id=5000 + li, dtype=torch.bfloat16)
-                q = synthetic.normal((G, spec.qk_dim), seed=seed, tensor_id=6000 + li, dtype=torch.bfloat16)
-                kn = synthetic.normal((spec.qk_dim,), seed=seed, tensor_id=7000 + li, dtype=torch.bfloat16)
-                vn = synthetic.normal((spec.v_dim,), seed=seed, tensor_id=8000 + li, dtype=torch.bfloat16)
-                sinks = np.zeros(G) if spec.has_sink else None
-                if fp8:
-                    kc8, vc8 = e4m3_of(kc, 1 / 16), e4m3_of(vc, 1 / 32)
-                    t0 = time.perf_counter()
-                    oracle.decode_fp8kv(q.double().numpy(), kn.double().numpy(), vn.double().numpy(), kc8, vc8, L,
-                                        spec.rotary_dim, spec.theta, spec.layer_type, spec.window,
-                                        1 / math.sqrt(spec.qk_dim), sinks, 0.7, 1 / 16, 1 / 32)
-                else:
-                    t0 = time.perf_counter()
-                    oracle.decode(q.double().numpy(), kn.double().numpy(), vn.double().numpy(), kc.double().numpy(),
-                                  vc.double().numpy(), L, spec.rotary_dim, spec.theta, spec.layer_type, spec.window,
-                                  1 / math.sqrt(spec.qk_dim), sinks, 0.7)
-                t_total += time.perf_counter() - t0
-                flops += G * (min(L, spec.window) if spec.layer_type == 1 else L) * 2 * (spec.qk_dim + spec.v_dim)
-                groups_done += 1
-    if proj is not None:
-        desc = (f"{rows_done} tokens of the global layer's QKV projection (all 13568 features, RoPE); "
-                f"fp64 oracle (numpy matmul on one BLAS thread)")
-    else:
-        desc = (f"{rows_done} prefill query rows (uniform positions{' in the chunk' if row_lo else ''}, all visible "
-                f"keys, every layer of the stack) + {groups_done} decode KV groups (one sequence, all query heads "
-                f"of the group{', E4M3 caches' if fp8 else ''}); fp64 C oracle, single thread")
-    return flops, t_total, desc
+                flops += 2.0 * x.shape[0] * w.shape[0] * x.shape[1]
+                rows += x.shape[0]
+            t = time.perf_counter() - t0
+        return flops, t, (f"{rows} tokens of the global layer's QKV projection (all 13568 features, RoPE); fp64 "
+                          f"oracle, numpy matmul on {threads} BLAS threads"), threads
+
+    def tasks():
+        n = 0
+        while True:
+            if pw is not None:
+                for li, spec in enumerate(pw.layers):
+                    yield _prefill_row_task(inp, spec, pw.seq, int(rng.integers(row_lo, pw.seq)), n + li)
+            if dw is not None:
+                for li, spec in enumerate(dw.layers):
+                    L = int(rng.integers(dw.kv_len_range[0], dw.kv_len_range[1] + 1))
+                    yield _decode_group_task(inp, spec, L, li, fp8, e4m3_of)
+            n += 1
+
+    # draw the inputs of every layer kind before the clock starts
+    warm = tasks()
+    for _ in range((len(pw.layers) if pw else 0) + (len(dw.layers) if dw else 0)):
+        next(warm)
+    flops, t, n = _run_parallel(tasks(), threads, seconds)
+    what = []
+    if pw is not None:
+        what.append(f"prefill query rows at uniform positions{' in the chunk' if row_lo else ''} (all visible keys, "
+                    f"every layer of the workload in turn)")
+    if dw is not None:
+        what.append(f"decode KV groups (one sequence of uniform length, all query heads of the group"
+                    f"{', E4M3 caches' if fp8 else ''})")
+    desc = f"{n} units: " + " + ".join(what) + f"; fp64 C oracle on {threads} threads ({cpu_model()})"
+    return flops, t, desc, threads
 
 
 # ------------------------------------------------------------------ traffic
-def committed_traffic(kernel_tag: str, source: str):
+def committed_traffic(kernel_tag: str, source: str, tokens: int):
     """Per-launch DRAM bytes from the committed ncu summary profiles/<kernel_tag>.md,
     valid only while the kernel's source file (csrc/<source>) still matches the
-    hash recorded there."""
+    hash recorded there. The summary gives the bytes of its capture and the
+    tokens (batch x sequence) the captured launch processed; this kernel's
+    traffic grows with the tokens (Q, K, V read once, O written once), so the
+    capture is scaled to `tokens`."""
     import hashlib
     path = os.path.join(ROOT, "profiles", f"{kernel_tag}.md")
     src = os.path.join(ROOT, "global_attention_partial_b200", "csrc", source)
@@ -574,8 +682,8 @@ def committed_traffic(kernel_tag: str, source: str):
     if vals.get("source_sha256_16") != sha:
         return None
     try:
-        return float(vals["dram_bytes_per_full_launch"])
-    except (KeyError, ValueError):
+        return float(vals["dram_bytes_per_capture"]) * tokens / float(vals["tokens_per_capture"])
+    except (KeyError, ValueError, ZeroDivisionError):
         return None
 
 
@@ -613,16 +721,20 @@ def job_value(world: int, units_per_rank: float, ms_max: float) -> float:
 
 
 def run_reference(args):
-    """CPU oracle arm: rank 0 times the oracle on bounded samples."""
+    """CPU oracle arm: rank 0 times the oracle, threaded over the host cores,
+    on bounded samples of the workload."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
+        return
+    if args.oracle_table:
+        print(json.dumps(oracle_table(args)), flush=True)
         return
     per_step = float(os.environ.get("MIMO_REF_STEP_SECONDS", "6"))
     for _ in range(args.warmup):
         oracle_sample(min(per_step, 1.0), seed=99, kind=args.workload)
-    vals, flops_total, t_total, desc = [], 0.0, 0.0, ""
+    flops_total, t_total, desc, threads = 0.0, 0.0, "", 1
     for s in range(args.steps):
-        f, t, desc = oracle_sample(per_step, seed=s, kind=args.workload)
+        f, t, desc, threads = oracle_sample(per_step, seed=s, kind=args.workload)
         flops_total += f
         t_total += t
     value = flops_total / t_total / 1e12
@@ -630,12 +742,110 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * t_total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(args, reference=True),
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
+                             "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def workload_config(args, reference=False):
+def oracle_table(args):
+    """Wall time of the fp64 oracle over whole configurations, threaded over
+    the host cores: the tiny fp32 pair, the SWA layer (B1 S4096) and the
+    hybrid decode (B64, every layer) in full; the global layer (B2 S8192)
+    and the hybrid prefill stack (B4 S32768) on a sample of query rows,
+    extrapolated by unmasked FLOPs (each row's cost is proportional to its
+    visible keys). The inputs are the synthetic ones (CPU draws, bf16)."""
+    import oracle
+    oracle.build()
+    threads = host_cores()
+    res = {"cores": threads, "cpu_model": cpu_model(), "configs": {}}
+    seed = 0
+
+    def time_layer(spec, B, S, rows_per_head, dtype=torch.bfloat16, batches=None):
+        """Times one layer in the oracle's own order (oracle.prefill_layer):
+        rotate each (batch, KV head)'s keys once, then per (batch, query head)
+        rotate the query rows and attend them. Both phases run on the thread
+        pool. `batches` limits the timed sequences (the others are alike);
+        rows_per_head(b, h) picks the rows (all, or a sample). Returns
+        (estimated seconds for all B sequences and all rows, measured
+        seconds, attention FLOPs done)."""
+        Hq, G = spec.num_q_heads, spec.num_q_heads // spec.num_kv_heads
+        nb = B if batches is None else batches
+        q, k, v, sinks = synthetic.prefill_inputs(spec, nb, S, seed=seed, layer=0, dtype=dtype)
+        sn = None if sinks is None else sinks.double().numpy()
+        pos = np.arange(S, dtype=np.float64)
+        scale = 1 / math.sqrt(spec.qk_dim)
+        vs = oracle.v_scale(spec.hidden_size, Hq, spec.v_dim)
+        k_rot = {}
+
+        def rotate(b, kv):
+            def run():
+                k_rot[(b, kv)] = (oracle.rope(k[b, :, kv].double().numpy(), spec.rotary_dim, spec.theta, pos),
+                                  v[b, :, kv].double().numpy())
+                return 0.0
+            return run
+
+        def attend(b, h, rows):
+            def run():
+                kr, vv = k_rot[(b, h // G)]
+                qr = oracle.rope(q[b, rows, h].double().numpy(), spec.rotary_dim, spec.theta, pos[rows])
+                oracle.prefill_rows(qr, rows, kr, vv, spec.layer_type, spec.window, scale,
+                                    None if sn is None else float(sn[h]), vs)
+                lo = np.maximum(0, rows - spec.window + 1) if spec.layer_type == 1 else 0
+                return float(np.sum(rows - lo + 1)) * 2 * (spec.qk_dim + spec.v_dim)
+            return run
+
+        _, t_rot, _ = _run_parallel([rotate(b, kv) for b in range(nb) for kv in range(spec.num_kv_heads)], threads)
+        f, t_att, _ = _run_parallel([attend(b, h, rows_per_head(b, h)) for b in range(nb) for h in range(Hq)],
+                                    threads)
+        full = prefill_flops(spec, B, S)
+        # key rotation: once per (batch, KV head), scaled to B sequences;
+        # attention: proportional to FLOPs (each row costs its visible keys)
+        return t_rot * B / nb + t_att * full / f, t_rot + t_att, f
+
+    def record(name, mode, est, meas, done, full):
+        res["configs"][name] = {"mode": mode, "oracle_s": est, "measured_s": meas, "flops_done": done,
+                                "flops_full": full, "gflops_per_s": full / est / 1e9}
+
+    # tiny fp32 pair, in full
+    est = meas = done = full = 0.0
+    for spec in synthetic.TINY_PAIR.layers:
+        e, m, d = time_layer(spec, 1, 64, lambda b, h: np.arange(64), dtype=torch.float32)
+        est, meas, done, full = est + e, meas + m, done + d, full + prefill_flops(spec, 1, 64)
+    record("c0 tiny fp32 pair", "full", est, meas, done, full)
+    # SWA layer B1 S4096, in full
+    spec = synthetic.SWA_PREFILL.layers[0]
+    e, m, d = time_layer(spec, 1, 4096, lambda b, h: np.arange(4096))
+    record("c1 SWA B1 S4096", "full", e, m, d, prefill_flops(spec, 1, 4096))
+    # global layer B2 S8192: 64 uniform rows per (batch, head), extrapolated by FLOPs
+    spec = synthetic.GLOBAL_PREFILL.layers[0]
+    rng = np.random.default_rng(1)
+    e, m, d = time_layer(spec, 2, 8192, lambda b, h: np.sort(rng.integers(0, 8192, 64)))
+    record("c2 global B2 S8192", "sampled, extrapolated", e, m, d, prefill_flops(spec, 2, 8192))
+    # hybrid stack B4 S32768: each layer kind timed on one sequence (the four
+    # are alike), 8 uniform rows per head, extrapolated to its layers of the
+    # stack (2 global, 6 sliding) over all 4 sequences
+    est = meas = done = 0.0
+    for lt in (0, 1):
+        spec = synthetic.mimo_layer(lt)
+        e, m, d = time_layer(spec, 4, 32768, lambda b, h: np.sort(rng.integers(0, 32768, 8)), batches=1)
+        n_layers = sum(1 for sp in synthetic.HYBRID_PREFILL.layers if sp.layer_type == lt)
+        est, meas, done = est + n_layers * e, meas + m, done + d
+    record("c3 hybrid stack B4 S32768", "sampled, extrapolated", est, meas, done,
+           sum(prefill_flops(sp, 4, 32768) for sp in synthetic.HYBRID_PREFILL.layers))
+    # hybrid decode B64, every layer and every KV group, in full
+    dw = synthetic.HYBRID_DECODE
+    lens = synthetic.decode_kv_lens(dw.batch, *dw.kv_len_range, seed=seed).tolist()
+    inp = _OracleInputs(seed)
+    tasks = [_decode_group_task(inp, spec, L, li, False, None) for li, spec in enumerate(dw.layers)
+             for L in lens for _ in range(spec.num_kv_heads)]
+    f, t, _ = _run_parallel(tasks, threads)
+    record("c4 hybrid decode B64", "full", t, t, f, sum(decode_flops(spec, lens) for spec in dw.layers))
+    return res
+
+
+def workload_config(args, reference=False, kind=None):
+    kind = kind or args.workload
     names = {"stack": f"{synthetic.HYBRID_PREFILL.name} + {synthetic.HYBRID_DECODE.name}",
              "swa": synthetic.SWA_PREFILL.name, "global": synthetic.GLOBAL_PREFILL.name,
              "decode": synthetic.HYBRID_DECODE.name,
@@ -644,64 +854,43 @@ def workload_config(args, reference=False):
                     "hidden 4096 pattern 0,1,1,1,1,1,0,1",
              "chunked": f"hybrid 8-layer stack, chunk of {CHUNK_SEQ} tokens after {CHUNK_PAST} cached, bf16 B4 "
                         f"pattern 0,1,1,1,1,1,0,1"}
-    cfg = {"workload": names[args.workload], "prefill_batch": synthetic.HYBRID_PREFILL.batch,
+    cfg = {"workload": names[kind], "prefill_batch": synthetic.HYBRID_PREFILL.batch,
            "prefill_seq": synthetic.HYBRID_PREFILL.seq, "decode_batch": synthetic.HYBRID_DECODE.batch,
            "kv_len_range": list(synthetic.HYBRID_DECODE.kv_len_range), "layers": "0,1,1,1,1,1,0,1",
            "parallelism": f"replicas x{args.gpus} (weak, no collective on the data path)",
            "l2": "no flush: each step streams ~60 GB of inputs, far above the 126 MB L2"}
-    if args.workload in ("stack", "decode", "decode_fp8"):
+    if kind in ("stack", "decode", "decode_fp8"):
         cfg["decode_launch"] = ("direct C-ABI calls, one per layer" if args.no_graph else
                                 "the 8 layers' C-ABI calls captured once in a CUDA graph, replayed each step")
-    if args.workload != "stack":
-        cfg["l2"] = "inputs larger than L2" if args.workload != "swa" else "L2 flushed between steps (256 MB write)"
+    if kind != "stack":
+        cfg["l2"] = "inputs larger than L2" if kind != "swa" else "L2 flushed between steps (256 MB write)"
+    if args.layers is not None and kind == args.workload:
+        cfg["layer_subset"] = args.layers
+    if (args.batch is not None or args.seq is not None) and kind == args.workload:
+        cfg["prefill_override"] = {"batch": args.batch, "seq": args.seq}
     return cfg
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
-    ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["stack", "swa", "global", "decode", "chunked", "decode_fp8", "qkv"], default="stack")
-    ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-graph", action="store_true", help="launch the decode layers one call at a time")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    args = ap.parse_args()
-    if args.workload in ("chunked", "decode_fp8", "qkv"):  # NEXT-row measurements: no host-buffer leg
-        args.no_e2e = True
-    if args.impl == "reference":
-        run_reference(args)
-        return
-
-    dist, rank, world, local = dist_setup(args.gpus)
-    torch.cuda.set_device(local)
-    import global_attention_partial_b200 as mimo
-    mimo.load()
-    peaks = measured_peaks()
-    w = StackWorkload(args.workload)
-    if not args.no_graph:
-        w.capture_decode()
-    stream = torch.cuda.current_stream()
-    flush = None
-    if args.workload == "swa":
-        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-
-    for _ in range(max(args.warmup, 0)):
+def time_workload(w, steps, warmup, stream, dist=None, local=0, sample_clocks=False):
+    """Warm-up, then `steps` timed steps bracketed by a barrier and a
+    synchronize on both sides, CUDA events on `stream`. The SWA layer alone
+    fits in L2, so its steps flush L2 first (a 256 MB write, outside the
+    events). Returns (ms per step, max over ranks; per-call-kind event times;
+    clocks or None)."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if w.kind == "swa" else None
+    for _ in range(max(warmup, 0)):
         w.step(stream)
     torch.cuda.synchronize()
-    if mimo.mimo_attn_get_device_error() != 0:
-        raise RuntimeError("device error word set during warm-up")
-
-    # ---- timed region (device-resident inputs)
-    sampler = ClockSampler(local)
-    sampler.start()
+    if w.mimo.mimo_attn_get_device_error() != 0:
+        raise RuntimeError(f"device error word set during the {w.kind} warm-up")
+    sampler = ClockSampler(local) if sample_clocks else None
+    if sampler:
+        sampler.start()
     events = {}
     barrier(dist, local)
     torch.cuda.synchronize()
     step_events = []
-    for _ in range(args.steps):
+    for _ in range(steps):
         if flush is not None:
             flush.zero_()
         e0 = torch.cuda.Event(enable_timing=True)
@@ -712,24 +901,30 @@ def main():
         step_events.append((e0, e1))
     torch.cuda.synchronize()
     barrier(dist, local)
-    clocks = sampler.stop()
-    ms_local = sum(a.elapsed_time(b) for a, b in step_events) / args.steps
+    clocks = sampler.stop() if sampler else None
+    ms_local = sum(a.elapsed_time(b) for a, b in step_events) / steps
     ms = max_over_ranks(dist, ms_local)
-
     kinds = {k: [a.elapsed_time(b) for a, b in v] for k, v in events.items()}
+    if w.mimo.mimo_attn_get_device_error() != 0:
+        raise RuntimeError(f"device error word set while timing {w.kind}")
+    return ms, kinds, clocks
+
+
+def summarize(w, ms, kinds, steps, peaks, stream):
+    """Step FLOPs, per-part rates and the roofline object of the workload's
+    dominant kernel, from the CUDA-event times of time_workload."""
     pflops = w.prefill_flops() if w.do_prefill else 0.0
     dflops = w.decode_flops() if w.do_decode else 0.0
     cflops = w.chunk_flops() if w.do_chunked else 0.0
     qflops = w.qkv_flops() if w.do_qkv else 0.0
     step_flops = pflops + dflops + cflops + qflops
-    value = job_value(world, step_flops, ms)
-
+    sustained = peaks["bf16_tflops_sustained"]
     parts = {}
     roofline = None
     if w.do_prefill:
-        ms_prefill = (sum(sum(v) for k, v in kinds.items() if k.startswith("prefill")) / args.steps)
+        ms_prefill = (sum(sum(v) for k, v in kinds.items() if k.startswith("prefill")) / steps)
         parts["prefill"] = {"ms": ms_prefill, "tflops": pflops / (ms_prefill * 1e-3) / 1e12,
-                            "frac_of_tensor_peak": pflops / (ms_prefill * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]}
+                            "frac_of_tensor_peak": pflops / (ms_prefill * 1e-3) / 1e12 / sustained}
         for kind, lt in (("prefill_global", 0), ("prefill_swa", 1)):
             if kind not in kinds:
                 continue
@@ -739,7 +934,7 @@ def main():
             byt = prefill_bytes(specs[0], w.pw.batch, w.pw.seq)
             parts[kind.replace("prefill_", "") + "_layer"] = {
                 "ms_per_launch": per, "tflops": f / (per * 1e-3) / 1e12,
-                "frac_of_tensor_peak": f / (per * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"],
+                "frac_of_tensor_peak": f / (per * 1e-3) / 1e12 / sustained,
                 "gbs_compulsory": byt / (per * 1e-3) / 1e9,
                 "frac_of_hbm_peak": byt / (per * 1e-3) / 1e9 / peaks["hbm_gbs"]}
         dom = "prefill_global" if "prefill_global" in kinds else "prefill_swa"
@@ -748,40 +943,47 @@ def main():
         per = statistics.mean(kinds[dom])
         if lt == 0:
             ach = prefill_flops(spec, w.pw.batch, w.pw.seq) / (per * 1e-3) / 1e12
-            roofline = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
-                        "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"],
-                        "traffic": committed_traffic("prefill_ga_global", "prefill_ga.cu"),
-                        "kernel": "prefill_ga_kernel (global layer, B4 S32768 causal)",
+            roofline = {"bound": "tensor", "achieved": ach, "peak": sustained,
+                        "unit": "TFLOP/s", "frac": ach / sustained,
+                        "traffic": committed_traffic("prefill_ga_global", "prefill_ga.cu", w.pw.batch * w.pw.seq),
+                        "kernel": f"prefill_ga_kernel (global layer, B{w.pw.batch} S{w.pw.seq} causal)",
                         "peak_kind": f"bf16 dense, sustained, {peaks['source']}"}
         else:
             ach = prefill_bytes(spec, w.pw.batch, w.pw.seq) / (per * 1e-3) / 1e9
             roofline = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                         "frac": ach / peaks["hbm_gbs"],
-                        "traffic": committed_traffic("prefill_swa_sliding", "prefill_swa.cu"),
-                        "kernel": "prefill_swa_kernel (sliding layer)", "peak_kind": f"HBM copy, {peaks['source']}"}
+                        "traffic": committed_traffic("prefill_swa_sliding", "prefill_swa.cu", w.pw.batch * w.pw.seq),
+                        "kernel": f"prefill_swa_kernel (sliding layer, B{w.pw.batch} S{w.pw.seq})",
+                        "peak_kind": f"HBM copy, {peaks['source']}"}
     if w.do_chunked:
         for kind, lt in (("chunk_global", 0), ("chunk_swa", 1)):
+            if kind not in kinds:
+                continue
             specs = [L["spec"] for L in w.chunk_layers if L["spec"].layer_type == lt]
             per = statistics.mean(kinds[kind])
             f = chunk_flops(specs[0], w.pw.batch, w.chunk_seq, w.chunk_past)
             parts[kind + "_layer"] = {"ms_per_launch": per, "tflops": f / (per * 1e-3) / 1e12,
-                                      "frac_of_tensor_peak": f / (per * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]}
-        ach = parts["chunk_global_layer"]["tflops"]
-        roofline = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                    "frac": ach / peaks["bf16_tflops_sustained"], "traffic": None,
-                    "kernel": "prefill_ga_kernel (global layer, chunk of 4096 after 28672 cached, B4)",
-                    "peak_kind": f"bf16 dense, sustained, {peaks['source']}"}
+                                      "frac_of_tensor_peak": f / (per * 1e-3) / 1e12 / sustained}
+        if "chunk_global_layer" in parts:
+            ach = parts["chunk_global_layer"]["tflops"]
+            roofline = {"bound": "tensor", "achieved": ach, "peak": sustained, "unit": "TFLOP/s",
+                        "frac": ach / sustained, "traffic": None,
+                        "kernel": "prefill_ga_kernel (global layer, chunk of 4096 after 28672 cached, B4)",
+                        "peak_kind": f"bf16 dense, sustained, {peaks['source']}"}
     if w.do_qkv:
         for kind, lt in (("qkv_global", 0), ("qkv_swa", 1)):
+            if kind not in kinds:
+                continue
             spec = [L["spec"] for L in w.qkv_layers if L["spec"].layer_type == lt][0]
             per = statistics.mean(kinds[kind])
             f = qkv_flops(spec, w.pw.batch, w.pw.seq)
             parts[kind + "_layer"] = {"ms_per_launch": per, "tflops": f / (per * 1e-3) / 1e12,
-                                      "frac_of_tensor_peak": f / (per * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]}
-        ach = parts["qkv_swa_layer"]["tflops"]
-        roofline = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                    "frac": ach / peaks["bf16_tflops_sustained"], "traffic": None,
-                    "kernel": "qkv_proj_kernel (sliding layer: 14848 features, B4 S32768, hidden 4096)",
+                                      "frac_of_tensor_peak": f / (per * 1e-3) / 1e12 / sustained}
+        key = "qkv_swa_layer" if "qkv_swa_layer" in parts else "qkv_global_layer"
+        ach = parts[key]["tflops"]
+        roofline = {"bound": "tensor", "achieved": ach, "peak": sustained, "unit": "TFLOP/s",
+                    "frac": ach / sustained, "traffic": None,
+                    "kernel": f"qkv_proj_kernel ({key[4:-6]} layer, B{w.pw.batch} S{w.pw.seq}, hidden 4096)",
                     "peak_kind": f"bf16 dense, sustained, {peaks['source']}"}
     if w.do_decode:
         per = statistics.mean(kinds["decode_stack"])
@@ -791,7 +993,7 @@ def main():
                            "bytes_per_stack": byt,
                            "launch": "direct calls" if getattr(w, "decode_graph", None) is None else "CUDA graph"}
         if getattr(w, "decode_graph", None) is not None:
-            # the same stack as 8 back-to-back direct calls, outside the timed region
+            # the same stack as back-to-back direct calls, outside the timed region
             d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             reps = 5
             d0.record(stream)
@@ -807,8 +1009,75 @@ def main():
             ach = byt / (per * 1e-3) / 1e9
             roofline = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                         "frac": ach / peaks["hbm_gbs"], "traffic": None,
-                        "kernel": "decode_mma_kernel (8-layer stack%s)" % (", fp8 KV cache" if w.fp8 else ""),
+                        "kernel": "decode_mma_kernel (%d-layer stack%s)" % (
+                            len(w.decode_layers), ", fp8 KV cache" if w.fp8 else ""),
                         "peak_kind": f"HBM copy, {peaks['source']}"}
+    return step_flops, parts, roofline
+
+
+# The configurations and NEXT-row workloads timed after the headline step
+# (outside its timed region), each reported under parts.configs.
+EXTRA_PARTS = ("swa", "global", "decode", "decode_fp8", "chunked", "qkv")
+
+
+def extra_parts(args, peaks, stream):
+    out = {}
+    for kind in EXTRA_PARTS:
+        w = StackWorkload(kind)
+        if not args.no_graph:
+            w.capture_decode()
+        steps = 20 if kind in ("swa", "global", "decode", "decode_fp8") else 3
+        ms, kinds, _ = time_workload(w, steps, 3, stream)
+        step_flops, parts, roofline = summarize(w, ms, kinds, steps, peaks, stream)
+        out[kind] = {"workload": workload_config(args, kind=kind)["workload"], "ms_per_step": ms, "steps": steps,
+                     "tflops": step_flops / (ms * 1e-3) / 1e12, "roofline": roofline, "parts": parts}
+        del w
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["stack", "swa", "global", "decode", "chunked", "decode_fp8", "qkv"],
+                    default="stack")
+    ap.add_argument("--layers", type=lambda x: [int(i) for i in x.split(",")], default=None,
+                    help="comma-separated layer indices of the workload to run (default: all), e.g. to profile one")
+    ap.add_argument("--batch", type=int, default=None, help="override the prefill batch (prefill / qkv workloads)")
+    ap.add_argument("--seq", type=int, default=None, help="override the prefill length (prefill / qkv workloads)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-parts", action="store_true",
+                    help="skip timing the other configurations after the stack step")
+    ap.add_argument("--no-graph", action="store_true", help="launch the decode layers one call at a time")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--oracle-table", action="store_true",
+                    help="with --impl reference: time the oracle over whole configurations (minutes)")
+    args = ap.parse_args()
+    if args.workload in ("chunked", "decode_fp8", "qkv") or args.layers is not None or args.seq or args.batch:
+        args.no_e2e = True  # NEXT-row and profiling runs: no host-buffer leg
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    dist, rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    import global_attention_partial_b200 as mimo
+    mimo.load()
+    peaks = measured_peaks()
+    w = StackWorkload(args.workload, layers=args.layers, batch=args.batch, seq=args.seq)
+    if not args.no_graph:
+        w.capture_decode()
+    stream = torch.cuda.current_stream()
+
+    # ---- timed region (device-resident inputs)
+    ms, kinds, clocks = time_workload(w, args.steps, args.warmup, stream, dist, local, sample_clocks=True)
+    step_flops, parts, roofline = summarize(w, ms, kinds, args.steps, peaks, stream)
+    value = job_value(world, step_flops, ms)
 
     # ---- e2e through the C ABI with host buffers
     e2e = None
@@ -835,21 +1104,29 @@ def main():
 
     if mimo.mimo_attn_get_device_error() != 0:
         raise RuntimeError("device error word set during the timed region")
+    launches = w.launches_per_step() * args.steps
+    del w
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    # ---- the other configurations, outside the timed region (rank-local, 1 GPU runs only)
+    if args.workload == "stack" and world == 1 and not args.no_parts and args.layers is None:
+        parts["configs"] = extra_parts(args, peaks, stream)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        f, t, desc = oracle_sample(args.cpu_seconds, kind=args.workload)
-        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": desc,
-               "seconds": t}
+        f, t, desc, threads = oracle_sample(args.cpu_seconds, kind=args.workload)
+        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": t, "cpu_model": cpu_model()}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None,
-                "dtype": "e4m3 KV cache, f16 mma, fp32 accumulate" if w.fp8 else "bf16", "data": "synthetic", "config": workload_config(args),
+                "dtype": "e4m3 KV cache, f16 mma, fp32 accumulate" if args.workload == "decode_fp8" else "bf16",
+                "data": "synthetic", "config": workload_config(args),
                 "roofline": roofline, "parts": parts, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": w.launches_per_step() * args.steps, "clocks": clocks,
-                "peaks": peaks}
+                "gpu_launches": launches, "clocks": clocks, "peaks": peaks}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()

@@ -45,6 +45,8 @@ EXPORTED = (
     "mimo_attn_get_device_error",
     "mimo_attn_status_string",
     "mimo_attn_debug_fail_launches",
+    "mimo_attn_debug_set_wait_limit",
+    "mimo_attn_debug_wait_probe",
     "mimo_attn_version",
 )
 
@@ -118,6 +120,10 @@ def load() -> ctypes.CDLL:
     lib.mimo_attn_status_string.restype = ctypes.c_char_p
     lib.mimo_attn_debug_fail_launches.argtypes = [i32]
     lib.mimo_attn_debug_fail_launches.restype = None
+    lib.mimo_attn_debug_set_wait_limit.argtypes = [ctypes.c_longlong]
+    lib.mimo_attn_debug_set_wait_limit.restype = i32
+    lib.mimo_attn_debug_wait_probe.argtypes = [vp]
+    lib.mimo_attn_debug_wait_probe.restype = i32
     lib.mimo_attn_version.argtypes = []
     lib.mimo_attn_version.restype = ctypes.c_char_p
     _lib = lib
@@ -281,6 +287,14 @@ def mimo_attn_get_device_error() -> int:
 
 def mimo_attn_debug_fail_launches(enable: bool) -> None:
     load().mimo_attn_debug_fail_launches(1 if enable else 0)
+
+
+def mimo_attn_debug_set_wait_limit(cycles: int) -> int:
+    return load().mimo_attn_debug_set_wait_limit(int(cycles))
+
+
+def mimo_attn_debug_wait_probe(stream=None) -> int:
+    return load().mimo_attn_debug_wait_probe(_stream(stream))
 
 
 def version() -> str:

@@ -14,13 +14,20 @@
 
 namespace {
 
-// Device error word: sticky bits set by kernels (kv_lens out of range, wait
-// timeouts). One copy per device, read by mimo_attn_get_device_error().
-__device__ unsigned g_device_error;
+// Device status block: the error word (sticky bits set by kernels: kv_lens
+// out of range, wait timeouts), read by mimo_attn_get_device_error(), and the
+// pipeline-wait limit the kernels read beside it. One copy per device.
+__device__ mimo::DeviceStatus g_device_status;
 
 int g_fail_launches = 0;
 
 constexpr int kMaxDevices = 64;
+
+// Device addresses looked up once per device and cached: the status block
+// here, the decode scratch array further down. One lock guards both caches,
+// so host threads that make their first call on a device at the same time
+// never race on them.
+std::mutex g_symbol_mutex;
 unsigned *g_err_ptr[kMaxDevices];
 
 unsigned *device_error_ptr()
@@ -28,11 +35,12 @@ unsigned *device_error_ptr()
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return nullptr;
+    std::lock_guard<std::mutex> lock(g_symbol_mutex);
     if (g_err_ptr[dev] == nullptr) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess)
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess)
             return nullptr;
-        g_err_ptr[dev] = static_cast<unsigned *>(p);
+        g_err_ptr[dev] = &static_cast<mimo::DeviceStatus *>(p)->error;
     }
     return g_err_ptr[dev];
 }
@@ -562,11 +570,34 @@ mimo_attn_status mimo_attn_get_device_error(uint32_t *bits)
     unsigned host = 0;
     const unsigned zero = 0;
     if (cudaDeviceSynchronize() != cudaSuccess ||
-        cudaMemcpyFromSymbol(&host, g_device_error, sizeof(host)) != cudaSuccess ||
-        cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+        cudaMemcpyFromSymbol(&host, g_device_status, sizeof(host), offsetof(mimo::DeviceStatus, error)) !=
+            cudaSuccess ||
+        cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero), offsetof(mimo::DeviceStatus, error)) !=
+            cudaSuccess)
         return MIMO_ATTN_ERR_CUDA;
     *bits = host;
     return MIMO_ATTN_OK;
+}
+
+mimo_attn_status mimo_attn_debug_set_wait_limit(long long cycles)
+{
+    const long long v = cycles > 0 ? cycles : 0;
+    if (cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpyToSymbol(g_device_status, &v, sizeof(v), offsetof(mimo::DeviceStatus, wait_limit)) !=
+            cudaSuccess)
+        return MIMO_ATTN_ERR_CUDA;
+    return MIMO_ATTN_OK;
+}
+
+mimo_attn_status mimo_attn_debug_wait_probe(void *stream)
+{
+    if (g_fail_launches)
+        return MIMO_ATTN_ERR_CUDA;
+    unsigned *err = device_error_ptr();
+    if (err == nullptr)
+        return MIMO_ATTN_ERR_CUDA;
+    return mimo::launch_wait_probe(err, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MIMO_ATTN_OK
+                                                                                           : MIMO_ATTN_ERR_CUDA;
 }
 
 const char *mimo_attn_status_string(mimo_attn_status status)
@@ -606,7 +637,6 @@ namespace {
 constexpr size_t kStaticScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) float g_decode_scratch[kStaticScratchBytes / sizeof(float)];
 
-std::mutex g_scratch_mutex;
 float *g_scratch_ptr[kMaxDevices];
 
 // Device address of g_decode_scratch on the current device. In host code the
@@ -617,7 +647,7 @@ float *static_scratch_ptr()
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return nullptr;
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    std::lock_guard<std::mutex> lock(g_symbol_mutex);
     if (g_scratch_ptr[dev] == nullptr) {
         float *ptr = nullptr;
         if (cudaGetSymbolAddress((void **)&ptr, g_decode_scratch) != cudaSuccess)

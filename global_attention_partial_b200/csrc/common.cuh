@@ -3,14 +3,16 @@
 // PTX wrappers for mbarriers, TMA tensor loads, tcgen05 (TMEM alloc, MMA,
 // commit, ld/st), cp.async, ldmatrix and mma.sync, plus the RoPE angle
 // routine shared by every kernel of the library. Every spin-wait is bounded:
-// after kWaitLimitCycles of waiting it sets the device error word and reports
-// a timeout so the caller can tear down instead of hanging.
+// after the device's wait limit (kWaitLimitCycles unless the test hook
+// shortened it) it sets the device error word and reports a timeout so the
+// caller can tear down instead of hanging.
 #pragma once
 
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
 
 namespace mimo {
@@ -18,8 +20,27 @@ namespace mimo {
 constexpr int kMaxHalfRotary = 128;          // rotary_dim <= 256
 constexpr unsigned kErrKvLen = 0x1u;         // = MIMO_ATTN_DEVERR_KV_LEN
 constexpr unsigned kErrTimeout = 0x2u;       // = MIMO_ATTN_DEVERR_TIMEOUT
-// Wait limit in SM clock cycles: ~4 s at 2 GHz, ~8 s at the lowest clocks.
+// Default wait limit in SM clock cycles: ~4 s at 2 GHz, ~8 s at the lowest
+// clocks. Teardown drains (mbar_drain) always use this one.
 constexpr long long kWaitLimitCycles = 8000000000ll;
+
+// Per-device status block. Kernels receive a pointer to `error` (the device
+// error word) and find the pipeline-wait limit beside it, so one pointer
+// serves both and no kernel needs another parameter. wait_limit <= 0 selects
+// kWaitLimitCycles; the host changes it only through the library's test hook.
+struct DeviceStatus {
+    unsigned error;
+    unsigned reserved;
+    long long wait_limit;
+};
+static_assert(offsetof(DeviceStatus, error) == 0, "the error word leads the status block");
+
+__device__ __forceinline__ long long wait_limit_of(const unsigned *err)
+{
+    const long long lim = reinterpret_cast<const volatile DeviceStatus *>(err)->wait_limit;
+    return lim > 0 ? lim : kWaitLimitCycles;
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Partial-RoPE parameters of one layer: pair j of the first rotary_dim dims
@@ -135,7 +156,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 
 // Waits for the phase of `bar` with the given parity to complete. Returns
 // false (without waiting further) once *abort is set by another thread of the
-// CTA, or after kWaitLimitCycles, in which case it sets *abort and the timeout
+// CTA, or after the device's wait limit (wait_limit_of(err), read once the
+// wait turns out to be slow), in which case it sets *abort and the timeout
 // bit of the device error word.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           unsigned *err)
@@ -143,12 +165,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity))
         return true;
     const long long t0 = cycles_now();
+    const long long limit = wait_limit_of(err);
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity))
             return true;
         if (*abort)
             return false;
-        if ((it & 255u) == 0 && cycles_now() - t0 > kWaitLimitCycles) {
+        if ((it & 255u) == 0 && cycles_now() - t0 > limit) {
             *abort = 1;
             atomicOr(err, kErrTimeout);
             return false;

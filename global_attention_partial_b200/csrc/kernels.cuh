@@ -196,4 +196,8 @@ int decode_chunk_keys(const LayerArgs &L, int dtype);
 int decode_max_splits(const LayerArgs &L, int dtype, int cap);
 cudaError_t launch_decode(const LayerArgs &L, const DecodeArgs &a, int dtype, cudaStream_t stream);
 
+// One CTA that waits on an mbarrier nothing arrives on, until the device's
+// wait limit ends the wait (timeout bit set in *err). Test probe only.
+cudaError_t launch_wait_probe(unsigned *err, cudaStream_t stream);
+
 } // namespace mimo

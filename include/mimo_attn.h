@@ -201,8 +201,9 @@ MIMO_ATTN_API mimo_attn_status mimo_attn_decode(const mimo_attn_layer *layer, in
  *     cache_capacity) must be at most 16 MiB (16777216 bytes), else the call
  *     returns MIMO_ATTN_ERR_WORKSPACE and launches nothing. (Example: 64
  *     query heads, cache 32768, up to 31 sequences per call.)
- *   - The array is device memory held by every GPU that loads the library,
- *     until the process exits.
+ *   - The 16 MiB are reserved on a device when the library's device code
+ *     first loads there (its first kernel launch or symbol lookup on that
+ *     device) and stay reserved until the process exits.
  *   - The first call on a device looks up the array's device address there
  *     (once per device, cached); make that first call before any stream
  *     capture.
@@ -307,6 +308,23 @@ MIMO_ATTN_API const char *mimo_attn_status_string(mimo_attn_status status);
  * MIMO_ATTN_ERR_CUDA after its argument checks, without launching. Lets the
  * host-side error path be tested without provoking a GPU fault. */
 MIMO_ATTN_API void mimo_attn_debug_fail_launches(int enable);
+
+/* Test hook: sets the pipeline-wait limit of the current device, in SM clock
+ * cycles; cycles <= 0 restores the default (8e9 cycles, ~4 s at 2 GHz). Every
+ * bounded wait of the library's pipelined kernels (an mbarrier that a copy or
+ * a tensor-core operation should complete) gives up after this many cycles,
+ * sets MIMO_ATTN_DEVERR_TIMEOUT and lets its kernel tear down. Synchronises
+ * the device. Returns MIMO_ATTN_OK or MIMO_ATTN_ERR_CUDA. Meant for tests of
+ * the timeout path together with mimo_attn_debug_wait_probe; a short limit
+ * during real work can end healthy kernels early. */
+MIMO_ATTN_API mimo_attn_status mimo_attn_debug_set_wait_limit(long long cycles);
+
+/* Test hook: launches one CTA on `stream` that waits, with the library's
+ * bounded wait, on an mbarrier nothing ever arrives on. The wait ends at the
+ * device's wait limit and sets MIMO_ATTN_DEVERR_TIMEOUT; no copy or
+ * tensor-core operation is in flight, so the context stays usable. With the
+ * default limit the kernel runs for ~4 s: shorten the limit first. */
+MIMO_ATTN_API mimo_attn_status mimo_attn_debug_wait_probe(void *stream);
 
 /* Version string of the library. */
 MIMO_ATTN_API const char *mimo_attn_version(void);

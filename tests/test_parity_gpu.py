@@ -124,6 +124,26 @@ def test_global_prefill_full_size_sampled_rows():
     _assert(c, BF, "global B2 S8192")
 
 
+@pytest.mark.parametrize("layer_idx", [0, 1])
+def test_hybrid_stack_full_size_sampled_rows(layer_idx):
+    """The hybrid 8-layer stack's prefill at its full size, B4 S32768 (Hq 64,
+    qk 192 / v 128, rotary 64), layer by layer as the benchmark runs it: layer
+    0 is global (4 KV heads, rope_theta) and layer 1 sliding (8 KV heads,
+    window 128, sinks), with the benchmark's seeds and launch path. Every
+    batch and all 64 heads on rows {0, 1, 126..129, 16383, 16384, 32766,
+    32767} plus 16 seeded random rows. Q alone is 3.2 GB here, so byte
+    offsets pass 2^31 and the global kernel's grid is (256, 32, 4)."""
+    wl = synthetic.HYBRID_PREFILL
+    spec = wl.layers[layer_idx]
+    assert spec.layer_type == (0 if layer_idx == 0 else 1)
+    c, out, inputs = check_prefill(spec, wl.batch, wl.seq, BF, seed=0, layer_idx=layer_idx, rows="sample",
+                                   n_random_rows=16)
+    del out, inputs
+    torch.cuda.empty_cache()
+    _assert(c, BF, f"hybrid stack layer {layer_idx} B{wl.batch} S{wl.seq}")
+    assert mimo.mimo_attn_get_device_error() == 0
+
+
 def test_prefill_is_deterministic():
     spec = synthetic.mimo_layer(0)
     q, k, v, _ = synthetic.prefill_inputs(spec, 1, 700, seed=3, layer=0, dtype=BF, device="cuda")

@@ -5,9 +5,11 @@ memory pool owns the whole GPU, a plugin without an allocator, a loop that
 must not pay cudaMalloc's implicit synchronisation. For them the library
 keeps the split-KV partials of decode in a 16 MiB array built into the
 library instead of a caller workspace. This test calls it through the C ABI
-and checks it against mimo_attn_decode (same tolerance as every bf16 parity
-test), on two calls in a row, since the shared array keeps the previous
-call's contents. The file name makes pytest collect it last.
+and checks it against mimo_attn_decode on calls in a row, since the shared
+array keeps the previous call's contents. Both entry points run the same
+kernels on the same inputs, so their outputs must be bit-identical (a
+tolerance would hide a stale partial that shifts a result slightly). The
+file name makes pytest collect it last.
 """
 import numpy as np
 import pytest
@@ -15,16 +17,30 @@ import torch
 
 import global_attention_partial_b200 as mimo
 from global_attention_partial_b200 import synthetic
-from tests.parity_util import BF16_MAX_ABS, BF16_MEAN_ABS
 
 pytestmark = pytest.mark.gpu
 
 
-def _inputs(spec, lens, cap, seed):
+def _inputs(spec, lens, cap, seed, nan=False):
     kv_lens = torch.tensor(lens, dtype=torch.int32)
     q, kn, vn, kc, vc, sinks = synthetic.decode_inputs(spec, len(lens), cap, kv_lens, seed=seed, layer=0,
                                                        device="cuda")
+    if nan:
+        for t in (q, kn, vn, kc, vc):
+            t.fill_(float("nan"))
     return q, kn, vn, kc, vc, (sinks if spec.layer_type == 1 else None), kv_lens.cuda()
+
+
+def _static(spec, lens, cap, seed, nan=False):
+    """One mimo_attn_decode_static call; returns its output."""
+    q, kn, vn, kc, vc, sinks, kv_lens = _inputs(spec, lens, cap, seed, nan)
+    lay = mimo.make_layer(spec.layer_type, spec.num_q_heads, spec.num_kv_heads, spec.qk_dim, spec.v_dim,
+                          spec.rotary_dim, spec.window, spec.theta, spec.hidden_size, sinks)
+    out = torch.empty((len(lens), spec.num_q_heads, spec.v_dim), dtype=torch.bfloat16, device="cuda")
+    st = mimo.mimo_attn_decode_static(lay, mimo.BF16, len(lens), q, kn, vn, kv_lens, kc, vc, kc.shape[1], out)
+    assert st == mimo.OK
+    torch.cuda.synchronize()
+    return out
 
 
 def _both(spec, lens, cap, seed):
@@ -49,10 +65,10 @@ def _both(spec, lens, cap, seed):
     return need, (out_a, kc_a, vc_a), (out_b, kc_b, vc_b)
 
 
-def _assert_close(a, b):
-    d = (a.double() - b.double()).abs()
+def _assert_same(a, b):
+    """Bit-identical outputs, all finite (same kernels, same inputs)."""
     assert torch.isfinite(b.double()).all()
-    assert d.max().item() <= BF16_MAX_ABS and d.mean().item() <= BF16_MEAN_ABS
+    assert torch.equal(a, b)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -69,7 +85,7 @@ def test_static_decode_matches_workspace_decode_two_calls_in_a_row():
     for lens, seed in calls:
         need, (out_a, kc_a, vc_a), (out_b, kc_b, vc_b) = _both(spec, lens, 8192, seed)
         assert 0 < need <= 16 << 20
-        _assert_close(out_a, out_b)
+        _assert_same(out_a, out_b)
         assert torch.equal(kc_a, kc_b) and torch.equal(vc_a, vc_b)
 
 
@@ -77,7 +93,30 @@ def test_static_decode_single_split_layer():
     spec = synthetic.mimo_layer(1)  # sliding ring: one split, no partials
     need, (out_a, _, _), (out_b, _, _) = _both(spec, [1, 50, 128, 129, 4000], 0, 13)
     assert need == 0
-    _assert_close(out_a, out_b)
+    _assert_same(out_a, out_b)
+
+
+def test_static_decode_ignores_stale_partials():
+    """A first call at the array's capacity on all-NaN inputs leaves NaN in
+    nearly every partial slot. Later calls of the same batch shape must read
+    only what they wrote themselves: one with every length <= 2048 (one
+    split per sequence, so no partial is read at all), then one with mixed
+    lengths (several splits). A stale read would show as NaN or as a
+    difference from mimo_attn_decode."""
+    spec = synthetic.mimo_layer(0)
+    B, cap = 120, 8192  # 120 x 64 heads x 4 splits x 130 floats = 15.97 MB of the 16 MiB
+    lay0 = mimo.make_layer(0, 64, 4, 192, 128, 64, 0, spec.theta, 4096, None)
+    assert 15 << 20 < mimo.mimo_attn_decode_workspace_size(lay0, mimo.BF16, B, cap) <= 16 << 20
+    stale = _static(spec, [cap] * B, cap, seed=31, nan=True)
+    assert torch.isnan(stale.double()).any()  # the array now holds non-finite partials
+    rng = np.random.default_rng(5)
+    short = rng.integers(1, 2049, B).tolist()
+    mixed = rng.integers(1, cap + 1, B).tolist()
+    for lens, seed in ((short, 32), (mixed, 33)):
+        need, (out_a, kc_a, vc_a), (out_b, kc_b, vc_b) = _both(spec, lens, cap, seed)
+        assert need > 15 << 20
+        _assert_same(out_a, out_b)
+        assert torch.equal(kc_a, kc_b) and torch.equal(vc_a, vc_b)
 
 
 def test_static_decode_rejects_sizes_beyond_the_array():
