@@ -35,6 +35,7 @@ def _worker(rank, world, port, out_dir):
 
         class Args:
             steps, warmup, gpus, workload = 1, 0, world, "swa"
+            oracle_table, no_graph, layers, batch, seq = False, False, None, None, None
         os.environ["MIMO_REF_STEP_SECONDS"] = "0.2"
         with contextlib.redirect_stdout(buf):
             bench.run_reference(Args())
