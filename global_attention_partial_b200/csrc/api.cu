@@ -120,6 +120,14 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // blocks of the tensor-core kernel aligned with the queries' spans.
 int cached_key_off(const mimo::LayerArgs &L) { return (int)round_up((size_t)(L.window - 1), 16); }
 
+// A sliding layer whose keys the tensor-core kernel rotates itself: no
+// rotated copy of K is written, the workspace holds only the RoPE table.
+bool swa_fused_keys(const mimo::LayerArgs &L, int dtype)
+{
+    return dtype == MIMO_ATTN_BF16 && mimo::prefill_swa_supported(L) &&
+           (L.rope.half == 0 || mimo::swa_rotates_keys(L));
+}
+
 } // namespace
 
 extern "C" {
@@ -138,8 +146,11 @@ size_t mimo_attn_prefill_workspace_size(const mimo_attn_layer *layer, int dtype,
     if (resolve_layer(layer, dtype, &L) != MIMO_ATTN_OK || batch < 0 || seq < 0)
         return 0;
     // the RoPE cos/sin table [S, r/2], then the rotated keys [B, S, Hkv, Dqk]
-    return round_up((size_t)seq * L.rope.half * sizeof(float2), 256) +
-           round_up((size_t)batch * seq * L.Hkv * L.Dqk * elem_size(dtype), 256);
+    // (none when the sliding-window kernel rotates the keys itself)
+    const size_t table = round_up((size_t)seq * L.rope.half * sizeof(float2), 256);
+    if (swa_fused_keys(L, dtype))
+        return table;
+    return table + round_up((size_t)batch * seq * L.Hkv * L.Dqk * elem_size(dtype), 256);
 }
 
 mimo_attn_status mimo_attn_prefill(const mimo_attn_layer *layer, int dtype, int batch, int seq,
@@ -185,6 +196,49 @@ mimo_attn_status mimo_attn_prefill(const mimo_attn_layer *layer, int dtype, int 
     if (err == nullptr)
         return MIMO_ATTN_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    if (swa_fused_keys(L, dtype)) {
+        // Sliding layer on the tensor-core kernel, which rotates K in shared
+        // memory: the RoPE table, the ring (when asked for), the attention.
+        float2 *table = L.rope.half > 0 ? reinterpret_cast<float2 *>(workspace) : nullptr;
+        if (mimo::launch_rope_table(L.rope, table, seq, s, positions) != cudaSuccess)
+            return MIMO_ATTN_ERR_CUDA;
+        if (has_cache) {
+            mimo::KprepArgs kr;
+            memset(&kr, 0, sizeof(kr));
+            kr.k = k;
+            kr.v = v;
+            kr.ring_k = k_cache;
+            kr.ring_v = v_cache;
+            kr.B = batch;
+            kr.S = seq;
+            kr.Hkv = L.Hkv;
+            kr.Dqk = L.Dqk;
+            kr.Dv = L.Dv;
+            kr.window = L.window;
+            kr.rope_table = table;
+            kr.rope = L.rope;
+            if (mimo::launch_kprep_ring(kr, dtype, s) != cudaSuccess)
+                return MIMO_ATTN_ERR_CUDA;
+        }
+        mimo::PrefillArgs pa;
+        memset(&pa, 0, sizeof(pa));
+        pa.q = q;
+        pa.krot = k;
+        pa.krot_rows = seq;
+        pa.key_rows_valid = seq;
+        pa.k_unrotated = L.rope.half > 0;
+        pa.v = v;
+        pa.v_rows = seq;
+        pa.positions = positions;
+        pa.rope_table = table;
+        pa.out = out;
+        pa.B = batch;
+        pa.S = seq;
+        pa.err = err;
+        return mimo::launch_prefill_swa(L, pa, table, num_sms(), s) == cudaSuccess ? MIMO_ATTN_OK
+                                                                                    : MIMO_ATTN_ERR_CUDA;
+    }
 
     mimo::KprepArgs kp;
     memset(&kp, 0, sizeof(kp));

@@ -74,8 +74,15 @@ struct KprepArgs {
 };
 cudaError_t launch_kprep(const KprepArgs &a, int dtype, cudaStream_t stream);
 
-// cos / sin of positions 0..n-1 for every rotary pair: table [n][rotary_dim/2].
-cudaError_t launch_rope_table(const RopeArgs &rope, float2 *table, long long n, cudaStream_t stream);
+// cos / sin of positions 0..n-1 (or positions[0..n-1] when positions is not
+// null) for every rotary pair: table [n][rotary_dim/2].
+cudaError_t launch_rope_table(const RopeArgs &rope, float2 *table, long long n, cudaStream_t stream,
+                              const int *positions = nullptr);
+
+// The sliding-window ring of a prefill: the last `window` tokens' rotated
+// keys and values into slots i mod window (a.ring_k / a.ring_v, a.rope_table
+// filled); nothing else.
+cudaError_t launch_kprep_ring(const KprepArgs &a, int dtype, cudaStream_t stream);
 
 // Prefill continuing a cache: writes the chunk's rotated keys and values
 // where the attention kernels read them. Global layers: cache rows
@@ -121,6 +128,7 @@ struct PrefillArgs {
     const int *past_lens;      // [B] tokens already in the cache, or nullptr
     int max_past;              // >= every past_lens[b]: the table has max_past + S rows
     int swa_key_off;           // sliding layers: key index of query 0 (a multiple of 16)
+    int k_unrotated;           // krot holds the input keys: the kernel rotates them (prefill_swa only)
     void *out;
     int B, S;
     unsigned *err;
@@ -138,8 +146,10 @@ bool prefill_ga_supported(const LayerArgs &L);
 cudaError_t launch_prefill_ga(const LayerArgs &L, const PrefillArgs &a, cudaStream_t stream);
 
 // Sliding-window prefill whose tiles need a single key span (persistent,
-// one CTA per SM); rope_table is the kprep table.
+// one CTA per SM); rope_table holds cos / sin per sequence index. With
+// a.k_unrotated the kernel rotates the keys itself (needs swa_rotates_keys).
 bool prefill_swa_supported(const LayerArgs &L);
+bool swa_rotates_keys(const LayerArgs &L);
 cudaError_t launch_prefill_swa(const LayerArgs &L, const PrefillArgs &a, const float2 *rope_table,
                                int num_sms, cudaStream_t stream);
 

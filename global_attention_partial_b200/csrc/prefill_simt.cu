@@ -93,6 +93,49 @@ __global__ void kprep_kernel(const __grid_constant__ KprepArgs a)
     }
 }
 
+// The sliding-window ring only: one warp per (b, token, kv) row of the last
+// min(S, window) tokens; rotates the key (table values) into ring slot
+// i mod window and copies the value. Used when the attention kernel rotates
+// the keys itself, so no other key copy is written.
+template <typename T>
+__global__ void kprep_ring_kernel(const __grid_constant__ KprepArgs a)
+{
+    const int warps = blockDim.x >> 5;
+    const long long row = (long long)blockIdx.x * warps + (threadIdx.x >> 5);
+    const int nring = a.S < a.window ? a.S : a.window;
+    const long long total = (long long)a.B * nring * a.Hkv;
+    if (row >= total)
+        return;
+    const int lane = threadIdx.x & 31;
+    const int kv = (int)(row % a.Hkv);
+    const long long br = row / a.Hkv;
+    const int i = a.S - nring + (int)(br % nring);
+    const int b = (int)(br / nring);
+    const int half = a.rope.half;
+    const float2 *cs = a.rope_table + (long long)i * half;
+    const long long src = ((long long)b * a.S + i) * a.Hkv + kv;
+    const long long dst = ((long long)b * a.window + i % a.window) * a.Hkv + kv;
+    const T *k = reinterpret_cast<const T *>(a.k) + src * a.Dqk;
+    T *rk = reinterpret_cast<T *>(a.ring_k) + dst * a.Dqk;
+    for (int e = lane; e < a.Dqk; e += 32) {
+        float y;
+        if (e < a.rope.rotary_dim) {
+            const int j = e < half ? e : e - half;
+            const float2 c = __ldg(cs + j);
+            const float xa = to_f32<T>(k[j]);
+            const float xb = to_f32<T>(k[j + half]);
+            y = e < half ? xa * c.x - xb * c.y : xb * c.x + xa * c.y;
+        } else {
+            y = to_f32<T>(k[e]);
+        }
+        rk[e] = from_f32<T>(y);
+    }
+    const T *v = reinterpret_cast<const T *>(a.v) + src * a.Dv;
+    T *rv = reinterpret_cast<T *>(a.ring_v) + dst * a.Dv;
+    for (int e = lane; e < a.Dv; e += 32)
+        rv[e] = v[e];
+}
+
 // bf16 rows in 16-byte units (8 elements): a lane takes either a pair of
 // rotary chunks (c, c + half/8), a pass-through K chunk, or a V chunk.
 // Needs rotary_dim % 16 == 0, Dqk % 8 == 0, Dv % 8 == 0.
@@ -337,13 +380,30 @@ cudaError_t launch_kprep(const KprepArgs &a, int dtype, cudaStream_t stream)
     return cudaGetLastError();
 }
 
-cudaError_t launch_rope_table(const RopeArgs &rope, float2 *table, long long n, cudaStream_t stream)
+cudaError_t launch_kprep_ring(const KprepArgs &a, int dtype, cudaStream_t stream)
+{
+    const int nring = a.S < a.window ? a.S : a.window;
+    const long long rows = (long long)a.B * nring * a.Hkv;
+    if (rows == 0)
+        return cudaSuccess;
+    const int threads = 256;
+    const long long blocks = (rows + (threads / 32) - 1) / (threads / 32);
+    if (dtype == kDtypeBf16)
+        kprep_ring_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, stream>>>(a);
+    else
+        kprep_ring_kernel<float><<<(unsigned)blocks, threads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rope_table(const RopeArgs &rope, float2 *table, long long n, cudaStream_t stream,
+                              const int *positions)
 {
     if (rope.half == 0 || n == 0)
         return cudaSuccess;
     KprepArgs a;
     memset(&a, 0, sizeof(a));
     a.S = (int)n;
+    a.positions = positions;
     a.rope_table = table;
     a.rope = rope;
     const long long tb = (n * rope.half + 255) / 256;

@@ -16,16 +16,18 @@
 // Two worker warpgroups take alternate tiles (tile n goes to warpgroup n % 2),
 // so one softmax overlaps the other tile's MMAs and epilogue. A worker
 // rotates its Q tile (partial RoPE, in place in swizzled shared memory, cos /
-// sin from the table kprep wrote), runs the softmax (thread r owns row r: the
+// sin from the per-call table), runs the softmax (thread r owns row r: the
 // row's 144 S values from TMEM, window mask, max, P as bf16 over the S
 // columns), then the epilogue (O from TMEM, sink fold, normalise, V scale,
 // store). Both workers run the same code, which keeps the instruction cache
-// warm.
+// warm. The keys arrive unrotated in a plain prefill: the Q-producer warp
+// rotates each 16-key block in the ring once it lands, before any QK^T reads
+// it. (A prefill continuing a cache reads a window of rotated keys.)
 //
 // Warp roles (384 threads = 3 warpgroups; setmaxnreg moves registers from the
 // control warpgroup to the workers):
 //   warps 0-3   worker for even tiles    warps 4-7   worker for odd tiles
-//   warp 8      TMA producer of the Q tiles
+//   warp 8      TMA producer of the Q tiles; rotates the new key blocks
 //   warp 9      MMA issuer of worker 0 (QK^T and PV of the even tiles)
 //   warp 10     MMA issuer of worker 1 (the odd tiles)
 //   warp 11     TMA producer of the K/V ring blocks
@@ -84,6 +86,7 @@ struct SwaParams {
     int max_past;
     int num_p_tiles, num_g_tiles, num_tiles, tiles_per_cta;
     int rope_half;
+    int rotate_k;              // K arrives unrotated: rotate each ring block in shared memory
     float scale_log2;
     float v_scale;
 };
@@ -91,6 +94,7 @@ struct SwaParams {
 struct Bars {
     uint64_t q_full[2], q_ready[2], q_empty[2];
     uint64_t kv_full[kRing], kv_empty[kRing];
+    uint64_t kv_ready[kRing];  // rotate_k: the block's keys are rotated in place
     uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
     uint64_t tab_full[2];  // the worker's 128 threads copied its RoPE table slice
     uint64_t drain[2];
@@ -186,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
         for (int i = 0; i < kRing; ++i) {
             mbar_init(&bars->kv_full[i], 1);
             mbar_init(&bars->kv_empty[i], 2);  // one commit from each issuer
+            mbar_init(&bars->kv_ready[i], 1);
         }
         mbar_init(&bars->drain[0], 1);
         mbar_init(&bars->drain[1], 1);
@@ -206,28 +211,122 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
         setmaxnreg_dec<kRegsControl>();
     }
     if (warp == 8) {
-        // ------------------------------------------------- TMA producer: Q
-        // Q tiles through their two buffers, each refilled once the QK^T of
-        // the tile two before has read it.
-        if (lane == 0 && n_local > 0) {
-            tma_prefetch_desc(&p.tm_q);
-            int last_q[2] = {-1, -1};
-            for (int n = 0; n < n_local; ++n) {
-                const int qb = n & 1;
-                if (!mbar_wait(&bars->q_empty[qb], ((uint32_t)(n >> 1) & 1u) ^ 1u, abort_flag, p.err))
-                    break;
-                const Tile c = tile_at(p, t_begin + n);
-                mbar_arrive_expect_tx(&bars->q_full[qb], kQBytes);
-                for (int a = 0; a < 3; ++a)
-                    tma_load_4d(sQ + qb * kQBytes + a * (kBlockM * 128), &p.tm_q, &bars->q_full[qb], a * 64,
-                                c.h0, c.p0, c.b);
-                last_q[qb] = n;
-            }
-            if (*abort_flag)
-                for (int qb = 0; qb < 2; ++qb)
-                    if (last_q[qb] >= 0)
-                        mbar_drain(&bars->q_full[qb], (uint32_t)(last_q[qb] >> 1) & 1u);
+        // --------------------------------- TMA producer of Q; key rotation
+        // An event loop that never blocks on one stream while the other can
+        // move: lane 0 issues each Q tile into its buffer once the QK^T of
+        // the tile two before has read it, and, when the keys arrive
+        // unrotated, the whole warp rotates (partial RoPE, in place in the
+        // ring) each key block as soon as it lands, in ring order. Each lane
+        // takes key rows x 16-byte chunk pairs (c, c + half / 8), i.e. 8
+        // rotary pairs, with cos / sin from the per-call table; the rotary
+        // dims all lie in the first 64-column block of the ring entry.
+        int last_q[2] = {-1, -1};
+        RingCursor cur;
+        const int nch = p.rope_half >> 3;
+        int nq = 0;                             // next Q tile to issue
+        int nr = p.rotate_k ? 0 : n_local;      // tile whose new blocks are being rotated
+        int blk = 0, blk_end = -1;              // its blocks still to rotate: [blk, blk_end]
+        if (nr < n_local) {
+            const Tile c0 = tile_at(p, t_begin);
+            blk = cur.advance(c0);
+            blk_end = c0.last_block;
         }
+        long long idle_since = cycles_now();
+        const long long limit = wait_limit_of(p.err);
+        bool ok = true;
+        if (lane == 0 && n_local > 0)
+            tma_prefetch_desc(&p.tm_q);
+        while (nq < n_local || nr < n_local) {
+            bool moved = false;
+            if (nq < n_local) {
+                int go = 0;
+                const int qb = nq & 1;
+                if (lane == 0 && mbar_try_wait(&bars->q_empty[qb], ((uint32_t)(nq >> 1) & 1u) ^ 1u)) {
+                    const Tile c = tile_at(p, t_begin + nq);
+                    mbar_arrive_expect_tx(&bars->q_full[qb], kQBytes);
+                    for (int a = 0; a < 3; ++a)
+                        tma_load_4d(sQ + qb * kQBytes + a * (kBlockM * 128), &p.tm_q, &bars->q_full[qb], a * 64,
+                                    c.h0, c.p0, c.b);
+                    last_q[qb] = nq;
+                    go = 1;
+                }
+                if (__shfl_sync(0xffffffffu, go, 0)) {
+                    ++nq;
+                    moved = true;
+                }
+            }
+            if (nr < n_local) {
+                const int e = cur.entry(blk);
+                const int slot = e % kRing;
+                int go = 0;
+                if (lane == 0)
+                    go = mbar_try_wait(&bars->kv_full[slot], (uint32_t)(e / kRing) & 1u) ? 1 : 0;
+                if (__shfl_sync(0xffffffffu, go, 0)) {
+                    for (int item = lane; item < kKeyBlock * nch; item += 32) {
+                        const int kr = item / nch;
+                        const int cp = item - kr * nch;
+                        const int u = blk * kKeyBlock + kr;  // key index = sequence index
+                        if (u >= p.S)
+                            continue;
+                        uint8_t *k_row = sK + slot * (kKeyBlock * 128) + kr * 128;
+                        uint4 *pa = reinterpret_cast<uint4 *>(k_row + ((cp ^ (kr & 7)) << 4));
+                        uint4 *pb = reinterpret_cast<uint4 *>(k_row + (((cp + nch) ^ (kr & 7)) << 4));
+                        const float4 *g =
+                            reinterpret_cast<const float4 *>(p.rope_table + (size_t)u * p.rope_half + cp * 8);
+                        float4 cs[4];
+#pragma unroll
+                        for (int w = 0; w < 4; ++w)
+                            cs[w] = __ldg(g + w);
+                        uint4 va = *pa, vb = *pb;
+                        uint32_t *xa_w = reinterpret_cast<uint32_t *>(&va);
+                        uint32_t *xb_w = reinterpret_cast<uint32_t *>(&vb);
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            const float2 xa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&xa_w[w]));
+                            const float2 xb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&xb_w[w]));
+                            const float4 cc = cs[w];  // (cos, sin) of pairs 8cp+2w, 8cp+2w+1
+                            xa_w[w] = pack_bf16x2(xa.x * cc.x - xb.x * cc.y, xa.y * cc.z - xb.y * cc.w);
+                            xb_w[w] = pack_bf16x2(xb.x * cc.x + xa.x * cc.y, xb.y * cc.z + xa.y * cc.w);
+                        }
+                        *pa = va;
+                        *pb = vb;
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&bars->kv_ready[slot]);
+                    moved = true;
+                    if (++blk > blk_end && ++nr < n_local) {
+                        const Tile c = tile_at(p, t_begin + nr);
+                        blk = cur.advance(c);
+                        blk_end = c.last_block;
+                    }
+                }
+            }
+            if (moved) {
+                idle_since = cycles_now();
+                continue;
+            }
+            // nothing ready: stop on another thread's abort or after the wait limit
+            int stop = 0;
+            if (lane == 0) {
+                if (*abort_flag) {
+                    stop = 1;
+                } else if (cycles_now() - idle_since > limit) {
+                    *abort_flag = 1;
+                    atomicOr(p.err, kErrTimeout);
+                    stop = 1;
+                }
+            }
+            if (__shfl_sync(0xffffffffu, stop, 0)) {
+                ok = false;
+                break;
+            }
+        }
+        if (lane == 0 && !ok)
+            for (int qb = 0; qb < 2; ++qb)
+                if (last_q[qb] >= 0)
+                    mbar_drain(&bars->q_full[qb], (uint32_t)(last_q[qb] >> 1) & 1u);
     } else if (warp == 11) {
         // ---------------------------------------------- TMA producer: K/V ring
         // Independent of the Q stream, so key blocks run ahead of the tiles
@@ -330,8 +429,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 wait(&bars->q_ready[t], ph);
                 // Only this tile's entries: those below e0 may already be
                 // released (and refilled) on behalf of the other worker.
-                for (known_full = max(known_full, e0); known_full < e0 + nb; ++known_full)
+                for (known_full = max(known_full, e0); known_full < e0 + nb; ++known_full) {
                     wait(&bars->kv_full[known_full % kRing], (uint32_t)(known_full / kRing) & 1u);
+                    if (p.rotate_k)
+                        wait(&bars->kv_ready[known_full % kRing], (uint32_t)(known_full / kRing) & 1u);
+                }
                 tc_fence_after();
                 const int s0 = e0 % kRing;
                 const int run1 = min(nb, kRing - s0);
@@ -571,6 +673,12 @@ int swa_heads_per_tile(const LayerArgs &L)
     return gp;
 }
 
+bool swa_rotates_keys(const LayerArgs &L)
+{
+    // every rotary dim in the first 64-column block, pairs in whole 16-byte chunks
+    return L.rope.half > 0 && L.rope.rotary_dim <= 64 && L.rope.half % 8 == 0;
+}
+
 bool prefill_swa_supported(const LayerArgs &L)
 {
     if (L.layer_type != 1 || L.Dqk != kDqk || L.Dv != kDv || L.rope.rotary_dim > kDqk)
@@ -615,6 +723,7 @@ cudaError_t launch_prefill_swa(const LayerArgs &L, const PrefillArgs &a, const f
     p.num_tiles = p.num_p_tiles * p.num_g_tiles * L.Hkv * a.B;
     p.tiles_per_cta = (p.num_tiles + num_sms - 1) / num_sms;
     p.rope_half = L.rope.half;
+    p.rotate_k = a.k_unrotated ? 1 : 0;
     p.scale_log2 = L.scale_log2;
     p.v_scale = L.v_scale;
 

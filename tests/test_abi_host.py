@@ -146,8 +146,11 @@ def test_decode_argument_checks(lib):
 
 def test_workspace_sizes(lib):
     l = layer()
-    # RoPE table [S, r/2] (cos, sin) then rotated keys [B, S, Hkv, Dqk], each rounded to 256 bytes
-    assert mimo.mimo_attn_prefill_workspace_size(l, mimo.BF16, 1, 4096) == 4096 * 32 * 8 + 4096 * 8 * 192 * 2
+    # RoPE table [S, r/2] (cos, sin); the sliding-window tensor-core kernel
+    # rotates K itself, so bf16 needs no rotated copy of K ...
+    assert mimo.mimo_attn_prefill_workspace_size(l, mimo.BF16, 1, 4096) == 4096 * 32 * 8
+    # ... while fp32 (CUDA-core path) also takes the rotated keys [B, S, Hkv, Dqk]
+    assert mimo.mimo_attn_prefill_workspace_size(l, mimo.FP32, 1, 4096) == 4096 * 32 * 8 + 4096 * 8 * 192 * 4
     assert mimo.mimo_attn_prefill_workspace_size(l, mimo.FP32, 1, 3) == 3 * 32 * 8 + 256 * math.ceil(3 * 8 * 192 * 4 / 256)
     # one split per sequence on the ring: no partials needed
     assert mimo.mimo_attn_decode_workspace_size(l, mimo.BF16, 64, 128) == 0

@@ -69,7 +69,7 @@ def test_tc_prefill_windows(window):
     _assert(c, BF, f"window {window}")
 
 
-@pytest.mark.parametrize("rotary", [0, 2, 64, 96, 192])
+@pytest.mark.parametrize("rotary", [0, 2, 16, 32, 48, 64, 96, 192])
 def test_tc_prefill_rotary_dims(rotary):
     for lt in (0, 1):
         spec = synthetic.mimo_layer(lt)
