@@ -13,29 +13,38 @@
 // and freed after the PV of the last tile that uses it. Q tiles stream through
 // two buffers.
 //
-// Two worker warpgroups take alternate tiles (tile n goes to warpgroup n % 2),
-// so one softmax overlaps the other tile's MMAs and epilogue. A worker
-// rotates its Q tile (partial RoPE, in place in swizzled shared memory, cos /
-// sin from the per-call table), runs the softmax (thread r owns row r: the
-// row's 144 S values from TMEM, window mask, max, P as bf16 over the S
-// columns), then the epilogue (O from TMEM, sink fold, normalise, V scale,
-// store). Both workers run the same code, which keeps the instruction cache
-// warm. The keys arrive unrotated in a plain prefill: the Q-producer warp
-// rotates each 16-key block in the ring once it lands, before any QK^T reads
-// it. (A prefill continuing a cache reads a window of rotated keys.)
+// Two workers take alternate tiles (tile n goes to worker n % 2), so one
+// worker's softmax overlaps the other tile's MMAs and epilogue. A worker is
+// two warpgroups, one per column half: the thread pair (row r, half 0) and
+// (row r, half 1) shares query row r. The pair moves the row's Q from shared
+// memory into TMEM, applying the partial RoPE on the way (cos / sin from the
+// per-call table; each half 16 of the 32 pairs), and releases the Q buffer
+// at once: QK^T reads A from TMEM, so the next Q tile's load starts a whole
+// tile earlier than if the buffer waited for the MMA, and the kernel, whose
+// limit is the bytes it keeps in flight, gets more loads going. The pair then
+// runs the softmax (each half 72 of the 144 S columns from TMEM: window mask,
+// max exchanged through shared memory, P as bf16 written back over the S
+// columns) and the epilogue (64 of the 128 O columns: sink fold, normalise,
+// V scale, store).
 //
-// Warp roles (384 threads = 3 warpgroups; setmaxnreg moves registers from the
+// The keys arrive unrotated in a plain prefill: the Q-producer warp rotates
+// each 16-key block in the ring once it lands, before any QK^T reads it. (A
+// prefill continuing a cache reads a window of rotated keys.)
+//
+// Warp roles (640 threads = 5 warpgroups; setmaxnreg moves registers from the
 // control warpgroup to the workers):
-//   warps 0-3   worker for even tiles    warps 4-7   worker for odd tiles
-//   warp 8      TMA producer of the Q tiles; rotates the new key blocks
-//   warp 9      MMA issuer of worker 0 (QK^T and PV of the even tiles)
-//   warp 10     MMA issuer of worker 1 (the odd tiles)
-//   warp 11     TMA producer of the K/V ring blocks
-
+//   warps 0-3 / 4-7     worker 0 (even tiles), column half 0 / half 1
+//   warps 8-11 / 12-15  worker 1 (odd tiles), column half 0 / half 1
+//   warp 16             TMA producer of the Q tiles; rotates the new key blocks
+//   warp 17             MMA issuer of worker 0 (QK^T and PV of the even tiles)
+//   warp 18             MMA issuer of worker 1 (the odd tiles)
+//   warp 19             TMA producer of the K/V ring blocks
 //
-// TMEM (512 columns), per worker t: S_t = [256t, 256t + 144) and
+// TMEM (512 columns), per worker t: S_t = [256t, 256t + 144),
+// Q_t = [256t + 144, 256t + 240) (192 bf16 as pairs) and
 // O_t = [256t + 72, 256t + 200). O overlaps the upper S columns, which are
-// dead once the softmax has read them; P (bf16) takes the first 72 columns.
+// dead once the softmax has read them, and Q, dead once QK^T has read it;
+// P (bf16) takes the first 72 columns.
 // Shared memory: Q 2 x 48 KB; K ring 12 x 16 keys x 384 B; V ring 12 x 16
 // keys x 256 B (128B-swizzled 64-column blocks, 1024-byte aligned).
 #include "kernels.cuh"
@@ -48,28 +57,32 @@ namespace {
 constexpr int kBlockM = 128;
 constexpr int kKeyBlock = 16;
 constexpr int kMaxSpanBlocks = 9;  // 144 keys
+constexpr int kHalfCols = kMaxSpanBlocks * kKeyBlock / 2;  // 72 S columns per thread
 constexpr int kRing = 12;          // ring entries of 16 keys
 constexpr int kDqk = 192;
 constexpr int kDv = 128;
-constexpr int kThreads = 384;
-// Register split across the three warpgroups. The block launches with
+constexpr int kThreads = 640;
+constexpr int kWorkerThreads = 256;  // one worker: two warpgroups
+// Register split across the five warpgroups. The block launches with
 // kThreads x kLaunchRegs registers (ptxas must report exactly kLaunchRegs);
-// the shares below add up to that pool: 128 * (208 + 208 + 88) = 384 * 168.
-constexpr int kLaunchRegs = 168;
-constexpr int kRegsWorker = 208;
-constexpr int kRegsControl = 88;
-static_assert(128 * (2 * kRegsWorker + kRegsControl) == kThreads * kLaunchRegs,
+// the shares below add up to that pool: 128 * (4 * 104 + 64) = 640 * 96.
+constexpr int kLaunchRegs = 96;
+constexpr int kRegsWorker = 104;
+constexpr int kRegsControl = 64;
+static_assert(128 * (4 * kRegsWorker + kRegsControl) == kThreads * kLaunchRegs,
               "warpgroup register shares must add up to the launch pool");
 constexpr int kQBytes = kBlockM * kDqk * 2;             // 49152
-constexpr int kKAtom = kRing * kKeyBlock * 128;         // 24576: one 64-column block of the K ring
-constexpr int kVAtom = kRing * kKeyBlock * 128;         // 24576
+constexpr int kKAtom = kRing * kKeyBlock * 128;         // one 64-column block of the K ring
+constexpr int kVAtom = kRing * kKeyBlock * 128;
 constexpr int kKBytes = 3 * kKAtom;
 constexpr int kVBytes = 2 * kVAtom;
 constexpr int kEntryBytes = kKeyBlock * (kDqk + kDv) * 2;  // 10240
 constexpr int kTmemCols = 512;
+constexpr int kWarpQ = 16, kWarpMma0 = 17, kWarpKV = 19;
 
 __device__ __forceinline__ uint32_t col_s(int t) { return t ? 256u : 0u; }
 __device__ __forceinline__ uint32_t col_o(int t) { return col_s(t) + 72u; }
+__device__ __forceinline__ uint32_t col_q(int t) { return col_s(t) + 144u; }
 
 struct SwaParams {
     CUtensorMap tm_q;  // [B, S, Hq, Dqk]    box {64, gp, P, 1}
@@ -94,17 +107,18 @@ struct SwaParams {
 struct Bars {
     uint64_t q_full[2], q_ready[2], q_empty[2];
     uint64_t kv_full[kRing], kv_empty[kRing];
-    uint64_t kv_ready[kRing];  // rotate_k: the block's keys are rotated in place
+    uint64_t kv_ready[kRing];  // the block's keys are rotated in place (or need no rotation)
     uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
-    uint64_t tab_full[2];  // the worker's 128 threads copied its RoPE table slice
+    uint64_t xchg[2];      // both halves of worker t published their row maxima
+    uint64_t qrot[2];      // (generic RoPE only) both halves rotated Q in shared memory
     uint64_t drain[2];
     uint32_t tmem_base;
     int abort;
 };
 
-// RoPE table slice of one tile per worker: 16 positions x 32 (cos, sin) pairs.
-constexpr int kTabBytes = 16 * 32 * 8;
-constexpr int kSmemBytes = 1024 + 2 * kQBytes + kKBytes + kVBytes + 2 * kTabBytes + (int)sizeof(Bars) + 64;
+// Per worker: a row maximum and a row sum per half and query row.
+constexpr int kRedBytes = 2 * 2 * kBlockM * 4;
+constexpr int kSmemBytes = 1024 + 2 * kQBytes + kKBytes + kVBytes + 2 * kRedBytes + (int)sizeof(Bars) + 64;
 static_assert(kSmemBytes <= 232448, "shared memory");
 
 struct Tile {
@@ -131,8 +145,8 @@ __device__ __forceinline__ Tile tile_at(const SwaParams &p, int t)
     return c;
 }
 
-// Ring bookkeeping shared (and replayed identically) by the producer and
-// the MMA issuer: entries are numbered in load order; a run's blocks get
+// Ring bookkeeping shared (and replayed identically) by the producers and
+// the MMA issuers: entries are numbered in load order; a run's blocks get
 // consecutive entries.
 struct RingCursor {
     int run = -1;
@@ -158,6 +172,23 @@ struct RingCursor {
     __device__ __forceinline__ int entry(int block) const { return base + block; }
 };
 
+// Partial RoPE of the 16-byte chunk pair (a, b) = dims (8c .. 8c+7,
+// 8c+half .. 8c+half+7) of one row: pair 8c + 2w turns by the angle whose
+// (cos, sin) cs[w] holds in (x, y), pair 8c + 2w + 1 by (z, w).
+__device__ __forceinline__ void rope_chunk_pair(uint4 &va, uint4 &vb, const float4 (&cs)[4])
+{
+    uint32_t *a = reinterpret_cast<uint32_t *>(&va);
+    uint32_t *b = reinterpret_cast<uint32_t *>(&vb);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const float2 xa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&a[w]));
+        const float2 xb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&b[w]));
+        const float4 cc = cs[w];
+        a[w] = pack_bf16x2(xa.x * cc.x - xb.x * cc.y, xa.y * cc.z - xb.y * cc.w);
+        b[w] = pack_bf16x2(xb.x * cc.x + xa.x * cc.y, xb.y * cc.z + xa.y * cc.w);
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_constant__ SwaParams p)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -166,8 +197,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
     uint8_t *sQ = smem;                  // 2 buffers
     uint8_t *sK = sQ + 2 * kQBytes;      // 3 atoms of the ring
     uint8_t *sV = sK + kKBytes;          // 2 atoms of the ring
-    uint8_t *sTab = sV + kVBytes;        // 2 RoPE table slices
-    Bars *bars = reinterpret_cast<Bars *>(sTab + 2 * kTabBytes);
+    float *sRed = reinterpret_cast<float *>(sV + kVBytes);  // [worker][max | sum][half][row]
+    Bars *bars = reinterpret_cast<Bars *>(sV + kVBytes + 2 * kRedBytes);
     volatile int *abort_flag = &bars->abort;
 
     const int warp = threadIdx.x >> 5;
@@ -179,13 +210,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->q_full[i], 1);
-            mbar_init(&bars->q_ready[i], 128);
-            mbar_init(&bars->q_empty[i], 1);
+            mbar_init(&bars->q_ready[i], kWorkerThreads);
+            mbar_init(&bars->q_empty[i], kWorkerThreads);  // the workers copied Q into TMEM
             mbar_init(&bars->s_full[i], 1);
-            mbar_init(&bars->p_full[i], 128);
+            mbar_init(&bars->p_full[i], kWorkerThreads);
             mbar_init(&bars->o_full[i], 1);
-            mbar_init(&bars->o_free[i], 128);
-            mbar_init(&bars->tab_full[i], 128);
+            mbar_init(&bars->o_free[i], kWorkerThreads);
+            mbar_init(&bars->xchg[i], kWorkerThreads);
+            mbar_init(&bars->qrot[i], kWorkerThreads);
         }
         for (int i = 0; i < kRing; ++i) {
             mbar_init(&bars->kv_full[i], 1);
@@ -198,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
         fence_barrier_init();
         fence_proxy_async_smem();
     }
-    if (warp == 9) {
+    if (warp == kWarpMma0) {
         tmem_alloc(&bars->tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -207,26 +239,27 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-    if (warp >= 8) {
+    if (warp >= kWarpQ)
         setmaxnreg_dec<kRegsControl>();
-    }
-    if (warp == 8) {
+    if (warp == kWarpQ) {
         // --------------------------------- TMA producer of Q; key rotation
         // An event loop that never blocks on one stream while the other can
-        // move: lane 0 issues each Q tile into its buffer once the QK^T of
-        // the tile two before has read it, and, when the keys arrive
-        // unrotated, the whole warp rotates (partial RoPE, in place in the
-        // ring) each key block as soon as it lands, in ring order. Each lane
-        // takes key rows x 16-byte chunk pairs (c, c + half / 8), i.e. 8
-        // rotary pairs, with cos / sin from the per-call table; the rotary
-        // dims all lie in the first 64-column block of the ring entry.
+        // move (non-blocking barrier tests, a short sleep when idle): lane 0
+        // issues each Q tile into its buffer once the QK^T of the tile two
+        // before has read it, and the whole warp rotates (partial RoPE, in
+        // place in the ring) each key block as soon as it lands, in ring
+        // order, then marks it ready. Each lane takes key rows x 16-byte chunk
+        // pairs (c, c + half / 8), i.e. 8 rotary pairs, with cos / sin from
+        // the per-call table; the rotary dims all lie in the first 64-column
+        // block of the ring entry. Keys that arrive rotated are only marked
+        // ready.
         int last_q[2] = {-1, -1};
         RingCursor cur;
         const int nch = p.rope_half >> 3;
-        int nq = 0;                             // next Q tile to issue
-        int nr = p.rotate_k ? 0 : n_local;      // tile whose new blocks are being rotated
-        int blk = 0, blk_end = -1;              // its blocks still to rotate: [blk, blk_end]
-        if (nr < n_local) {
+        int nq = 0;                     // next Q tile to issue
+        int nr = 0;                     // tile whose new key blocks are being processed
+        int blk = 0, blk_end = -1;      // its blocks still to process: [blk, blk_end]
+        if (n_local > 0) {
             const Tile c0 = tile_at(p, t_begin);
             blk = cur.advance(c0);
             blk_end = c0.last_block;
@@ -241,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
             if (nq < n_local) {
                 int go = 0;
                 const int qb = nq & 1;
-                if (lane == 0 && mbar_try_wait(&bars->q_empty[qb], ((uint32_t)(nq >> 1) & 1u) ^ 1u)) {
+                if (lane == 0 && mbar_test_wait(&bars->q_empty[qb], ((uint32_t)(nq >> 1) & 1u) ^ 1u)) {
                     const Tile c = tile_at(p, t_begin + nq);
                     mbar_arrive_expect_tx(&bars->q_full[qb], kQBytes);
                     for (int a = 0; a < 3; ++a)
@@ -260,9 +293,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 const int slot = e % kRing;
                 int go = 0;
                 if (lane == 0)
-                    go = mbar_try_wait(&bars->kv_full[slot], (uint32_t)(e / kRing) & 1u) ? 1 : 0;
+                    go = mbar_test_wait(&bars->kv_full[slot], (uint32_t)(e / kRing) & 1u) ? 1 : 0;
                 if (__shfl_sync(0xffffffffu, go, 0)) {
-                    for (int item = lane; item < kKeyBlock * nch; item += 32) {
+                    for (int item = lane; p.rotate_k && item < kKeyBlock * nch; item += 32) {
                         const int kr = item / nch;
                         const int cp = item - kr * nch;
                         const int u = blk * kKeyBlock + kr;  // key index = sequence index
@@ -278,16 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                         for (int w = 0; w < 4; ++w)
                             cs[w] = __ldg(g + w);
                         uint4 va = *pa, vb = *pb;
-                        uint32_t *xa_w = reinterpret_cast<uint32_t *>(&va);
-                        uint32_t *xb_w = reinterpret_cast<uint32_t *>(&vb);
-#pragma unroll
-                        for (int w = 0; w < 4; ++w) {
-                            const float2 xa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&xa_w[w]));
-                            const float2 xb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&xb_w[w]));
-                            const float4 cc = cs[w];  // (cos, sin) of pairs 8cp+2w, 8cp+2w+1
-                            xa_w[w] = pack_bf16x2(xa.x * cc.x - xb.x * cc.y, xa.y * cc.z - xb.y * cc.w);
-                            xb_w[w] = pack_bf16x2(xb.x * cc.x + xa.x * cc.y, xb.y * cc.z + xa.y * cc.w);
-                        }
+                        rope_chunk_pair(va, vb, cs);
                         *pa = va;
                         *pb = vb;
                     }
@@ -322,12 +346,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 ok = false;
                 break;
             }
+            __nanosleep(64);
         }
         if (lane == 0 && !ok)
             for (int qb = 0; qb < 2; ++qb)
                 if (last_q[qb] >= 0)
                     mbar_drain(&bars->q_full[qb], (uint32_t)(last_q[qb] >> 1) & 1u);
-    } else if (warp == 11) {
+    } else if (warp == kWarpKV) {
         // ---------------------------------------------- TMA producer: K/V ring
         // Independent of the Q stream, so key blocks run ahead of the tiles
         // as far as the ring's free entries allow.
@@ -362,9 +387,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 for (int e = max(0, loaded - kRing); e < loaded; ++e)
                     mbar_drain(&bars->kv_full[e % kRing], (uint32_t)(e / kRing) & 1u);
         }
-    } else if (warp == 9 || warp == 10) {
+    } else if (warp >= kWarpQ) {
         // ------------------------------------------------------ MMA issuers
-        // Issuer t (warp 9 + t) serves worker t: the tiles n with n % 2 == t,
+        // Issuer t (warp 17 + t) serves worker t: the tiles n with n % 2 == t,
         // in order, each with blocking waits, so it reacts as soon as an input
         // is ready. Both walk every tile with the producer's ring cursor to
         // number the entries. An entry is free (its kv_empty barrier counts
@@ -374,16 +399,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
         // remaining entry after its last tile. As a tile spans at most 9 of
         // the 12 entries, every entry the producer waits on is then committed
         // by an issuer that is not waiting on that producer.
-        const int t = warp - 9;
+        const int t = warp - kWarpMma0;
         if (lane == 0 && t < n_local) {
             const uint32_t idesc_pv = idesc_bf16_f32(kBlockM, kDv, false, true);
-            const uint32_t q_lo = sdesc_lo(smem_u32(sQ + t * kQBytes), 16);
             const uint32_t k_lo = sdesc_lo(smem_u32(sK), 16);
             const uint32_t v_lo = sdesc_lo(smem_u32(sV), kVAtom);
-            constexpr uint32_t kQAtomStep = (kBlockM * 128) >> 4;
             constexpr uint32_t kKAtomStep = kKAtom >> 4;
             constexpr uint32_t kSlotStep = (kKeyBlock * 128) >> 4;
-            const uint32_t s_col = tmem + col_s(t), o_col = tmem + col_o(t);
+            const uint32_t s_col = tmem + col_s(t), o_col = tmem + col_o(t), q_col = tmem + col_q(t);
             bool ok = true;
             auto wait = [&](uint64_t *bar, uint32_t parity) {
                 if (!mbar_try_wait(bar, parity) && !mbar_wait(bar, parity, abort_flag, p.err))
@@ -402,7 +425,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 }
             };
             // S_t = Q_t K^T over the entries [e0, e0 + nb): one group of 12
-            // MMAs (N = 16 keys per entry), two when the span wraps the ring.
+            // MMAs (N = 16 keys per entry, A = 16 dims of Q_t = 8 TMEM
+            // columns), two groups when the span wraps the ring.
             auto qk_part = [&](uint32_t d, int slot, int blocks) {
                 const uint32_t idesc = idesc_bf16_f32(kBlockM, blocks * kKeyBlock, false, false);
                 const uint32_t kb = k_lo + (uint32_t)slot * kSlotStep;
@@ -410,10 +434,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 for (int atom = 0; atom < 3; ++atom)
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4)
-                        umma_ss_lo(d, q_lo + atom * kQAtomStep + 2 * k4, kb + atom * kKAtomStep + 2 * k4, idesc,
+                        umma_ts_lo(d, q_col + (uint32_t)(8 * (4 * atom + k4)), kb + atom * kKAtomStep + 2 * k4, idesc,
                                    (atom | k4) ? 1u : 0u);
             };
-            int known_full = 0;  // entries [0, known_full) have landed
+            int known_full = 0;  // entries [0, known_full) have landed (and are rotated)
             int freed = 0;       // entries [0, freed) committed by this issuer
             walk_to(t);
             for (int n = t; ok && n < n_local; n += 2) {
@@ -422,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 // again: commit them before waiting, so that the ring can refill
                 // while this tile's blocks are still missing (otherwise two
                 // tiles of 9 blocks from different runs, one per issuer, could
-                // wait on each other's 12-entry ring).
+                // wait on each other's ring).
                 for (; freed < e0; ++freed)
                     umma_commit(&bars->kv_empty[freed % kRing]);
                 wait(&bars->o_free[t], ph ^ 1u);  // epilogue of tile n - 2 has read O
@@ -431,8 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 // released (and refilled) on behalf of the other worker.
                 for (known_full = max(known_full, e0); known_full < e0 + nb; ++known_full) {
                     wait(&bars->kv_full[known_full % kRing], (uint32_t)(known_full / kRing) & 1u);
-                    if (p.rotate_k)
-                        wait(&bars->kv_ready[known_full % kRing], (uint32_t)(known_full / kRing) & 1u);
+                    wait(&bars->kv_ready[known_full % kRing], (uint32_t)(known_full / kRing) & 1u);
                 }
                 tc_fence_after();
                 const int s0 = e0 % kRing;
@@ -441,7 +464,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 if (nb > run1)
                     qk_part(s_col + (uint32_t)(run1 * kKeyBlock), 0, nb - run1);
                 umma_commit(&bars->s_full[t]);
-                umma_commit(&bars->q_empty[t]);
                 // O_t = P_t V over the same entries, one N = 128 MMA per entry.
                 wait(&bars->p_full[t], ph);
                 tc_fence_after();
@@ -469,16 +491,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 mbar_drain(&bars->drain[t], 0);
             }
         }
-    } else if (warp < 8) {
+    } else {
         // ------------------------------------------------------------ workers
         setmaxnreg_inc<kRegsWorker>();
-        const int t = warp >> 2;             // this worker takes tiles n with n % 2 == t
-        const int row = threadIdx.x & 127;
+        const int t = warp >> 3;             // this worker takes tiles n with n % 2 == t
+        const int hf = (warp >> 2) & 1;      // column half
+        const int row = threadIdx.x & 127;   // = the TMEM lane this warp may access
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        const uint32_t s_addr = lane_base + col_s(t);
-        const uint32_t o_addr = lane_base + col_o(t);
+        const uint32_t s_addr = lane_base + col_s(t) + (uint32_t)(kHalfCols * hf);
+        const uint32_t p_addr = lane_base + col_s(t) + (uint32_t)(kHalfCols / 2 * hf);
+        const uint32_t o_addr = lane_base + col_o(t) + (uint32_t)(64 * hf);
+        const uint32_t q_addr = lane_base + col_q(t);
+        float *red_max = sRed + t * (4 * kBlockM);  // [half][row]
+        float *red_sum = red_max + 2 * kBlockM;
         const int half = p.rope_half;
         const float sc = p.scale_log2;
+        const bool fast_rope = half == 32 && p.P == 16;
         bool ok = true;
         for (int n = t; ok && n < n_local; n += 2) {
             const uint32_t ph = (uint32_t)(n >> 1) & 1u;
@@ -489,73 +517,95 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
             // has position past + i; key rows below key_off - past precede
             // position 0 and are never visible
             const int past = p.past_lens != nullptr ? min(max(__ldg(p.past_lens + c.b), 0), p.max_past) : 0;
-            // ---- partial RoPE of this row of Q_n (buffer t)
-            // With 16 positions per tile and 32 pairs (the MiMo layer), the
-            // tile's 4 KB slice of the RoPE table is copied into shared memory
-            // before waiting for Q, so its latency overlaps the Q load without
-            // holding registers across the wait.
-            const bool fast_rope = half == 32 && p.P == 16;
-            const float4 *tab_row = reinterpret_cast<const float4 *>(sTab + t * kTabBytes) + (row >> 3) * 16;
-            if (fast_rope) {
-                const int qi = c.p0 + (row >> 3);
-                const bool in = qi < p.S;
-                const float2 *src = p.rope_table + (size_t)(past + (in ? qi : 0)) * 32 + (row & 7) * 4;
-                uint8_t *dst = sTab + t * kTabBytes + (row >> 3) * 256 + (row & 7) * 32;
-                cp_async16(dst, src, in ? 16u : 0u);
-                cp_async16(dst + 16, src + 2, in ? 16u : 0u);
-                cp_async_mbar_arrive(&bars->tab_full[t]);  // arrives once this thread's copies landed
-            }
-            if (!mbar_wait(&bars->q_full[t], ph, abort_flag, p.err) ||
-                (fast_rope && !mbar_wait(&bars->tab_full[t], ph, abort_flag, p.err))) {
+            const bool rot = i < p.S && half > 0;
+            if (!mbar_wait(&bars->q_full[t], ph, abort_flag, p.err)) {
                 ok = false;
                 break;
             }
-            if (i < p.S && half > 0) {
-                uint8_t *q_row = sQ + t * kQBytes + row * 128;
+            // ---- this row's Q_n into TMEM (the A operand of QK^T), partial
+            // RoPE on the way. Half hf takes rotary pairs 16hf .. 16hf + 15
+            // (16-byte chunks 2hf, 2hf + 1 of the first 64-column block and
+            // their partners 4 chunks up) and the pass-through dims of block
+            // 1 + hf. Dims (2c, 2c + 1) form TMEM column c of Q_t.
+            uint8_t *q_row = sQ + t * kQBytes + row * 128;
+            if (half > 0 && !fast_rope) {
+                // other rotary widths: rotate in place in shared memory first
+                // (pairs j = hf, hf + 2, ...), then copy like the fast path;
+                // every thread arrives, rows past the sequence end included
                 const float2 *cs = p.rope_table + (size_t)(past + i) * half;
-                if (fast_rope && i < p.S) {
-                    // One 128-byte swizzled row: chunks 0-3 hold dims 0-31, 4-7 dims 32-63.
-                    uint4 v[8];
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch)
-                        v[ch] = *reinterpret_cast<const uint4 *>(q_row + ((ch ^ (row & 7)) << 4));
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint32_t *a = reinterpret_cast<uint32_t *>(&v[ch]);
-                        uint32_t *bb = reinterpret_cast<uint32_t *>(&v[ch + 4]);
-#pragma unroll
-                        for (int w = 0; w < 4; ++w) {
-                            const float2 xa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&a[w]));
-                            const float2 xb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&bb[w]));
-                            const float4 cc = tab_row[ch * 4 + w];  // (cos, sin) of pairs 8ch+2w, 8ch+2w+1
-                            a[w] = pack_bf16x2(xa.x * cc.x - xb.x * cc.y, xa.y * cc.z - xb.y * cc.w);
-                            bb[w] = pack_bf16x2(xb.x * cc.x + xa.x * cc.y, xb.y * cc.z + xa.y * cc.w);
-                        }
-                    }
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch)
-                        *reinterpret_cast<uint4 *>(q_row + ((ch ^ (row & 7)) << 4)) = v[ch];
-                } else {
-                    for (int j = 0; j < half; ++j) {
-                        const int ea = j, eb = j + half;
-                        __nv_bfloat16 *pa = reinterpret_cast<__nv_bfloat16 *>(
-                            sQ + t * kQBytes + (ea >> 6) * (kBlockM * 128) + row * 128 +
-                            ((((ea & 63) >> 3) ^ (row & 7)) << 4) + ((ea & 7) << 1));
-                        __nv_bfloat16 *pb = reinterpret_cast<__nv_bfloat16 *>(
-                            sQ + t * kQBytes + (eb >> 6) * (kBlockM * 128) + row * 128 +
-                            ((((eb & 63) >> 3) ^ (row & 7)) << 4) + ((eb & 7) << 1));
-                        const float xa = __bfloat162float(*pa);
-                        const float xb = __bfloat162float(*pb);
-                        const float2 cj = __ldg(cs + j);
-                        *pa = __float2bfloat16_rn(xa * cj.x - xb * cj.y);
-                        *pb = __float2bfloat16_rn(xb * cj.x + xa * cj.y);
-                    }
+                for (int j = hf; rot && j < half; j += 2) {
+                    const int ea = j, eb = j + half;
+                    __nv_bfloat16 *pa = reinterpret_cast<__nv_bfloat16 *>(
+                        q_row + (ea >> 6) * (kBlockM * 128) + ((((ea & 63) >> 3) ^ (row & 7)) << 4) + ((ea & 7) << 1));
+                    __nv_bfloat16 *pb = reinterpret_cast<__nv_bfloat16 *>(
+                        q_row + (eb >> 6) * (kBlockM * 128) + ((((eb & 63) >> 3) ^ (row & 7)) << 4) + ((eb & 7) << 1));
+                    const float xa = __bfloat162float(*pa);
+                    const float xb = __bfloat162float(*pb);
+                    const float2 cj = __ldg(cs + j);
+                    *pa = __float2bfloat16_rn(xa * cj.x - xb * cj.y);
+                    *pb = __float2bfloat16_rn(xb * cj.x + xa * cj.y);
+                }
+                mbar_arrive(&bars->qrot[t]);
+                if (!mbar_wait(&bars->qrot[t], ph, abort_flag, p.err)) {
+                    ok = false;
+                    break;
                 }
             }
-            fence_proxy_async_smem();
+            // Q_t's columns hold O of tile n - 2 until both halves have read it
+            if (n >= 2 && !mbar_wait(&bars->o_free[t], ph ^ 1u, abort_flag, p.err)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            {
+                // rotary chunks 2hf, 2hf + 1 and their partners 2hf + 4, 2hf + 5
+                uint4 ca[2], cb[2];
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const int ch = 2 * hf + k;
+                    ca[k] = *reinterpret_cast<const uint4 *>(q_row + ((ch ^ (row & 7)) << 4));
+                    cb[k] = *reinterpret_cast<const uint4 *>(q_row + (((ch + 4) ^ (row & 7)) << 4));
+                }
+                if (rot && fast_rope) {
+                    // this half's 16 (cos, sin) pairs from the table (the
+                    // producer warp read the same rows for the keys: L1 hits)
+                    const float4 *g = reinterpret_cast<const float4 *>(p.rope_table + (size_t)(past + i) * 32) + 8 * hf;
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        float4 cs[4];
+#pragma unroll
+                        for (int w = 0; w < 4; ++w)
+                            cs[w] = __ldg(g + 4 * k + w);  // pairs 8 (2hf + k) + 2w, + 1
+                        rope_chunk_pair(ca[k], cb[k], cs);
+                    }
+                }
+                const uint32_t lo8[8] = {ca[0].x, ca[0].y, ca[0].z, ca[0].w, ca[1].x, ca[1].y, ca[1].z, ca[1].w};
+                const uint32_t hi8[8] = {cb[0].x, cb[0].y, cb[0].z, cb[0].w, cb[1].x, cb[1].y, cb[1].z, cb[1].w};
+                tmem_st8(q_addr + 8 * hf, lo8);       // dims 16hf .. 16hf + 15
+                tmem_st8(q_addr + 16 + 8 * hf, hi8);  // dims 32 + 16hf .. 32 + 16hf + 15
+            }
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {  // block 1 + hf: dims 64 (1 + hf) .. 64 (1 + hf) + 63
+                uint32_t w16[16];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(q_row + (1 + hf) * (kBlockM * 128) +
+                                                                      (((4 * part + k) ^ (row & 7)) << 4));
+                    w16[4 * k] = v.x;
+                    w16[4 * k + 1] = v.y;
+                    w16[4 * k + 2] = v.z;
+                    w16[4 * k + 3] = v.w;
+                }
+                tmem_st16(q_addr + 32 + 32 * hf + 16 * part, w16);
+            }
+            if (half > 0 && !fast_rope)
+                fence_proxy_async_smem();  // the in-place rotation's writes, before the next TMA fill
+            mbar_arrive(&bars->q_empty[t]);  // this thread's reads of the Q buffer are done
+            tmem_wait_st();
+            tc_fence_before();
             mbar_arrive(&bars->q_ready[t]);
 
-            // ---- softmax over the tile's key span
+            // ---- softmax over the tile's key span, this half's 72 columns
             const int k0 = c.first_block * kKeyBlock;
             const int hi = i + p.key_off - k0;  // the row's own key column
             const int lo = max(hi - p.window + 1, max(p.key_off - past, 0) - k0);  // first visible column
@@ -565,49 +615,94 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 break;
             }
             tc_fence_after();
-            float x[kMaxSpanBlocks * kKeyBlock];
+            float x[kHalfCols];
             {
-                uint32_t r[kMaxSpanBlocks][16];
+                uint32_t r[4][16], r8[8];
 #pragma unroll
-                for (int q = 0; q < kMaxSpanBlocks; ++q)
+                for (int q = 0; q < 4; ++q)
                     tmem_ld16(s_addr + 16 * q, r[q]);
+                tmem_ld8(s_addr + 64, r8);
                 tmem_wait_ld_only();
 #pragma unroll
-                for (int q = 0; q < kMaxSpanBlocks; ++q) {
+                for (int q = 0; q < 4; ++q) {
                     tmem_tie(r[q]);
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
                         x[16 * q + e] = __uint_as_float(r[q][e]);
                 }
+                tmem_tie(r8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    x[64 + e] = __uint_as_float(r8[e]);
+            }
+            // Window mask. On interior tiles every row sees columns 16 .. 127
+            // (its window starts at most 16 columns in, ends at least at 127),
+            // so only the 16 edge columns of each half need the test.
+            const int c0 = kHalfCols * hf;  // global column of x[0]
+            if (__all_sync(0xffffffffu, lo <= 16 && hi >= 127)) {
+                if (hf == 0) {  // (static indices keep x in registers)
+#pragma unroll
+                    for (int col = 0; col < 16; ++col)
+                        x[col] = ((unsigned)(col - lo) <= span) ? x[col] : -INFINITY;
+                } else {
+#pragma unroll
+                    for (int col = kHalfCols - 16; col < kHalfCols; ++col)
+                        x[col] = ((unsigned)(kHalfCols + col - lo) <= span) ? x[col] : -INFINITY;
+                }
+            } else {
+#pragma unroll
+                for (int col = 0; col < kHalfCols; ++col)
+                    x[col] = ((unsigned)(c0 + col - lo) <= span) ? x[col] : -INFINITY;
             }
             float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int col = 0; col < kMaxSpanBlocks * kKeyBlock; ++col) {
-                x[col] = ((unsigned)(col - lo) <= span) ? x[col] : -INFINITY;
-                mxv[col & 3] = fmaxf(mxv[col & 3], x[col]);
+            for (int col = 0; col < kHalfCols; col += 8)
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mxv[k] = fmax3(mxv[k], x[col + 2 * k], x[col + 2 * k + 1]);
+            float mx = fmax3(mxv[0], mxv[1], fmaxf(mxv[2], mxv[3]));
+            // the row's maximum over both halves
+            red_max[hf * kBlockM + row] = mx;
+            mbar_arrive(&bars->xchg[t]);
+            if (!mbar_wait(&bars->xchg[t], ph, abort_flag, p.err)) {
+                ok = false;
+                break;
             }
-            const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3]));
+            mx = fmaxf(mx, red_max[(hf ^ 1) * kBlockM + row]);
             const float m2 = mx * sc;   // base-2 units
             const float mu = (mx == -INFINITY) ? 0.f : m2;
-            float rsv[4] = {0.f, 0.f, 0.f, 0.f};
+            const f32x2 sc2 = {sc, sc}, nmu2 = {-mu, -mu};
+            f32x2 rsv[2] = {{0.f, 0.f}, {0.f, 0.f}};
+            // P over this half's columns: bf16 pairs into TMEM columns
+            // [36 hf, 36 hf + 36) of S. Both halves have read their S columns
+            // (the exchange above), so no write lands on unread scores.
 #pragma unroll
-            for (int q = 0; q < kMaxSpanBlocks; ++q) {
-                uint32_t pk[8];
+            for (int q = 0; q < kHalfCols / 8; ++q) {
+                uint32_t pk[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float e0 = fast_exp2(fmaf(x[16 * q + 2 * e], sc, -mu));
-                    const float e1 = fast_exp2(fmaf(x[16 * q + 2 * e + 1], sc, -mu));
-                    rsv[e & 3] += e0 + e1;
-                    pk[e] = pack_bf16x2(e0, e1);
+                for (int e = 0; e < 4; ++e) {
+                    const f32x2 z = fma2(f32x2{x[8 * q + 2 * e], x[8 * q + 2 * e + 1]}, sc2, nmu2);
+                    const f32x2 ez = {fast_exp2(z.x), fast_exp2(z.y)};
+                    rsv[e & 1] = add2(rsv[e & 1], ez);
+                    pk[e] = pack_bf16x2(ez.x, ez.y);
                 }
-                tmem_st8(s_addr + 8 * q, pk);
+                tmem_st4(p_addr + 4 * q, pk);
             }
-            const float rs = (rsv[0] + rsv[1]) + (rsv[2] + rsv[3]);
+            const float rs_half = (rsv[0].x + rsv[0].y) + (rsv[1].x + rsv[1].y);
+            red_sum[hf * kBlockM + row] = rs_half;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars->p_full[t]);
 
-            // ---- epilogue
+            // ---- epilogue: this half's 64 output columns. The p_full wait
+            // returns at once (the PV behind o_full needed it) and orders the
+            // partner's row sum, read before o_free lets the next tile reuse it.
+            if (!mbar_wait(&bars->o_full[t], ph, abort_flag, p.err) ||
+                !mbar_wait(&bars->p_full[t], ph, abort_flag, p.err)) {
+                ok = false;
+                break;
+            }
+            const float rs = rs_half + red_sum[(hf ^ 1) * kBlockM + row];
             float o_scale;
             if (p.sinks != nullptr) {
                 const float s2 = __ldg(p.sinks + h) * kLog2e;
@@ -617,43 +712,41 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
             } else {
                 o_scale = p.v_scale / rs;
             }
-            if (!mbar_wait(&bars->o_full[t], ph, abort_flag, p.err)) {
-                ok = false;
-                break;
-            }
             tc_fence_after();
-            uint32_t o[4][32];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                tmem_ld32(o_addr + 32 * q, o[q]);
+            uint32_t o[2][32];
+            tmem_ld32(o_addr, o[0]);
+            tmem_ld32(o_addr + 32, o[1]);
             tmem_wait_ld_only();
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                tmem_tie(o[q]);
+            tmem_tie(o[0]);
+            tmem_tie(o[1]);
             tc_fence_before();
             mbar_arrive(&bars->o_free[t]);
             if (i < p.S) {
-                uint8_t *dst = reinterpret_cast<uint8_t *>(p.out + (((size_t)c.b * p.S + i) * p.Hq + h) * kDv);
+                uint8_t *dst =
+                    reinterpret_cast<uint8_t *>(p.out + (((size_t)c.b * p.S + i) * p.Hq + h) * kDv + 64 * hf);
+                const f32x2 os2 = {o_scale, o_scale};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < 2; ++q) {
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         uint32_t w[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            w[e] = pack_bf16x2(__uint_as_float(o[q][hh * 16 + 2 * e]) * o_scale,
-                                               __uint_as_float(o[q][hh * 16 + 2 * e + 1]) * o_scale);
+                        for (int e = 0; e < 8; ++e) {
+                            const f32x2 v = mul2(f32x2{__uint_as_float(o[q][hh * 16 + 2 * e]),
+                                                       __uint_as_float(o[q][hh * 16 + 2 * e + 1])},
+                                                 os2);
+                            w[e] = pack_bf16x2(v.x, v.y);
+                        }
                         st_global_32B(dst + (q * 2 + hh) * 32, w, p.out_v8 != 0);
                     }
                 }
             }
         }
-        cp_async_wait<0>();  // no table copy may land after an abort ended the loop
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == kWarpMma0) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
