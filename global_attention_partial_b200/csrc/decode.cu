@@ -406,7 +406,10 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
     for (int t = 0; t < n_tiles; ++t) {
         const int base_key = key_begin + t * kTileKeys;
         const int kb = warp * 16;  // this warp's 16 keys within the tile
+        // Two accumulators per n-tile (even and odd k-steps), so the 12
+        // dependent MMAs of a score tile form two chains of 6.
         float s_acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float s_odd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         const uint8_t *land = nullptr;       // fp8: this warp's landed rows of tile t
         const __nv_bfloat16 *st = nullptr;   // bf16: the CTA's stage of tile t
         if constexpr (kFp8) {
@@ -437,7 +440,8 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
                 const uint32_t kw[12] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w, w2.x, w2.y, w2.z, w2.w};
 #pragma unroll
                 for (int ks = 0; ks < 12; ++ks)
-                    mma_f16_16816(s_acc[nt], qa[ks], e4m3x2_to_f16x2((uint16_t)(kw[ks] & 0xFFFFu)),
+                    mma_f16_16816((ks & 1) ? s_odd[nt] : s_acc[nt], qa[ks],
+                                  e4m3x2_to_f16x2((uint16_t)(kw[ks] & 0xFFFFu)),
                                   e4m3x2_to_f16x2((uint16_t)(kw[ks] >> 16)));
             }
         } else {
@@ -472,10 +476,15 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
             for (int ks = 0; ks < 12; ++ks) {
                 uint32_t b0, b1, b2, b3;
                 ldmatrix_x4(base + ks * 32, b0, b1, b2, b3);
-                mma_bf16_16816(s_acc[0], qa[ks], b0, b1);
-                mma_bf16_16816(s_acc[1], qa[ks], b2, b3);
+                mma_bf16_16816((ks & 1) ? s_odd[0] : s_acc[0], qa[ks], b0, b1);
+                mma_bf16_16816((ks & 1) ? s_odd[1] : s_acc[1], qa[ks], b2, b3);
             }
         }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                s_acc[nt][e] += s_odd[nt][e];
         // Scale, mask keys past the end of the range (only the range's last
         // tile has any), online softmax.
         float mx0 = -INFINITY, mx1 = -INFINITY;
@@ -514,10 +523,10 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
         float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-            p[nt][0] = exp2f(s_acc[nt][0] - u0);
-            p[nt][1] = exp2f(s_acc[nt][1] - u0);
-            p[nt][2] = exp2f(s_acc[nt][2] - u1);
-            p[nt][3] = exp2f(s_acc[nt][3] - u1);
+            p[nt][0] = fast_exp2(s_acc[nt][0] - u0);
+            p[nt][1] = fast_exp2(s_acc[nt][1] - u0);
+            p[nt][2] = fast_exp2(s_acc[nt][2] - u1);
+            p[nt][3] = fast_exp2(s_acc[nt][3] - u1);
             rs0 += p[nt][0] + p[nt][1];
             rs1 += p[nt][2] + p[nt][3];
         }
