@@ -323,7 +323,9 @@ class StackWorkload:
         return sum(decode_bytes(L["spec"], self.lens, 1 if self.fp8 else 2) for L in self.decode_layers)
 
     def launches_per_step(self):
-        n = 3 * len(self.prefill_layers)  # RoPE table + K-prep + attention
+        # prefill: RoPE table + attention, plus the key pre-pass on global
+        # layers (sliding layers rotate K inside the attention kernel)
+        n = sum(3 if L["spec"].layer_type == 0 else 2 for L in self.prefill_layers)
         for L in self.chunk_layers:  # RoPE table + cache prep (1 global, 2 sliding) + attention
             n += 3 if L["spec"].layer_type == 0 else 4
         for L in self.decode_layers:
@@ -750,11 +752,11 @@ def run_reference(args):
 
 def oracle_table(args):
     """Wall time of the fp64 oracle over whole configurations, threaded over
-    the host cores: the tiny fp32 pair, the SWA layer (B1 S4096) and the
-    hybrid decode (B64, every layer) in full; the global layer (B2 S8192)
-    and the hybrid prefill stack (B4 S32768) on a sample of query rows,
-    extrapolated by unmasked FLOPs (each row's cost is proportional to its
-    visible keys). The inputs are the synthetic ones (CPU draws, bf16)."""
+    the host cores: the tiny fp32 pair, the SWA layer (B1 S4096), the global
+    layer (B2 S8192) and the hybrid decode (B64, every layer) in full; the
+    hybrid prefill stack (B4 S32768) on a sample of query rows, extrapolated
+    by unmasked FLOPs (each row's cost is proportional to its visible keys).
+    The inputs are the synthetic ones (CPU draws, bf16)."""
     import oracle
     oracle.build()
     threads = host_cores()
@@ -817,11 +819,11 @@ def oracle_table(args):
     spec = synthetic.SWA_PREFILL.layers[0]
     e, m, d = time_layer(spec, 1, 4096, lambda b, h: np.arange(4096))
     record("c1 SWA B1 S4096", "full", e, m, d, prefill_flops(spec, 1, 4096))
-    # global layer B2 S8192: 64 uniform rows per (batch, head), extrapolated by FLOPs
+    # global layer B2 S8192, in full (under a minute on 16 cores)
     spec = synthetic.GLOBAL_PREFILL.layers[0]
     rng = np.random.default_rng(1)
-    e, m, d = time_layer(spec, 2, 8192, lambda b, h: np.sort(rng.integers(0, 8192, 64)))
-    record("c2 global B2 S8192", "sampled, extrapolated", e, m, d, prefill_flops(spec, 2, 8192))
+    e, m, d = time_layer(spec, 2, 8192, lambda b, h: np.arange(8192))
+    record("c2 global B2 S8192", "full", e, m, d, prefill_flops(spec, 2, 8192))
     # hybrid stack B4 S32768: each layer kind timed on one sequence (the four
     # are alike), 8 uniform rows per head, extrapolated to its layers of the
     # stack (2 global, 6 sliding) over all 4 sequences
@@ -854,9 +856,11 @@ def workload_config(args, reference=False, kind=None):
                     "hidden 4096 pattern 0,1,1,1,1,1,0,1",
              "chunked": f"hybrid 8-layer stack, chunk of {CHUNK_SEQ} tokens after {CHUNK_PAST} cached, bf16 B4 "
                         f"pattern 0,1,1,1,1,1,0,1"}
-    cfg = {"workload": names[kind], "prefill_batch": synthetic.HYBRID_PREFILL.batch,
-           "prefill_seq": synthetic.HYBRID_PREFILL.seq, "decode_batch": synthetic.HYBRID_DECODE.batch,
-           "kv_len_range": list(synthetic.HYBRID_DECODE.kv_len_range), "layers": "0,1,1,1,1,1,0,1",
+    pw = {"swa": synthetic.SWA_PREFILL, "global": synthetic.GLOBAL_PREFILL}.get(kind, synthetic.HYBRID_PREFILL)
+    cfg = {"workload": names[kind], "prefill_batch": pw.batch, "prefill_seq": pw.seq,
+           "decode_batch": synthetic.HYBRID_DECODE.batch,
+           "kv_len_range": list(synthetic.HYBRID_DECODE.kv_len_range),
+           "layers": ",".join(str(t) for t in pw.pattern),
            "parallelism": f"replicas x{args.gpus} (weak, no collective on the data path)",
            "l2": "no flush: each step streams ~60 GB of inputs, far above the 126 MB L2"}
     if kind in ("stack", "decode", "decode_fp8"):
