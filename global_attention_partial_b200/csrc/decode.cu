@@ -7,17 +7,21 @@
 //   writes key and value into the cache slot (L-1 for a global cache,
 //   (L-1) mod window for a sliding-window ring) and uses its own copy.
 //   K/V tiles of 64 keys stream through a multi-stage cp.async pipeline with
-//   16-byte coalesced loads; each warp takes 16 keys of a tile and runs
-//   S = Q K^T and O += P V on mma.sync m16n8k16 (query heads on M, keys on
-//   N), with the row max / sum reduced by warp shuffles. Warps are merged
+//   16-byte coalesced loads (all stages go out as soon as kv_lens, the first
+//   load of the kernel, has arrived); each warp takes 16 keys of a tile and
+//   runs S = Q K^T and O += P V on mma.sync m16n8k16 (query heads on M, keys
+//   on N), with the row max / sum reduced by warp shuffles. Warps are merged
 //   through shared memory; a sequence with one split is finished in place
 //   (sink folded, V scale applied), otherwise the (m, l, O) partials go to the
-//   workspace and a combine kernel merges them.
+//   workspace and a combine kernel merges them, one warp per query head.
 // fp8 (E4M3) caches, same kernel with kFp8: each warp streams its own 16 keys
 //   of every tile through a private cp.async ring and builds its f16 mma
 //   operands from the landed bytes in registers (QK over a permuted order of
 //   the 192 dims, PV with permuted output dims, undone at the merge); the new
-//   token is quantized into its slot and read back as codes.
+//   token is quantized into its slot and read back as codes. Sliding layers
+//   with a ring of at most two tiles take a slim form (query fragments read
+//   from shared memory per k-step, 2 stages, 4 CTAs per SM), so one wave
+//   holds every (sequence, KV head) of a B64 batch.
 // Other dtypes / dims: a CUDA-core path (one warp per query head) after a
 // separate new-token write.
 #include "kernels.cuh"
@@ -45,10 +49,13 @@ constexpr int kStageElems = kTileKeys * (kKStride + kVStride);
 constexpr int kLandRow = kDqk + kDv;             // bytes per key
 constexpr int kWarpLand = 16 * kLandRow;         // one warp's 16 keys: 5120
 constexpr int kLandBytes = kTileKeys * kLandRow;  // one stage of the CTA: 20480
-template <int ST, bool F8 = false> struct DecodeCfg {
+// SLIM (fp8 only): the query fragments stay in shared memory and are read per
+// k-step instead of held in 48 registers, so 4 CTAs fit per SM (128 registers,
+// 2 stages): the 512 CTAs of a 128-slot sliding layer at B64 run in one wave.
+template <int ST, bool F8 = false, bool SLIM = false> struct DecodeCfg {
     static constexpr int kSmemBytes = F8 ? (16 * kQStride + kDqk + kDv) * 2 + kLandRow + ST * kLandBytes
                                          : (16 * kQStride + ST * kStageElems + kDqk + kDv) * 2;
-    static constexpr int kCtasPerSm = F8 ? (ST <= 3 ? 3 : 2) : (ST <= 2 ? 2 : 1);
+    static constexpr int kCtasPerSm = SLIM ? 4 : F8 ? (ST <= 3 ? 3 : 2) : (ST <= 2 ? 2 : 1);
 };
 
 // 16-bit operand type of the tensor-core path: bf16 for bf16 caches, f16 for
@@ -72,6 +79,8 @@ constexpr int kDecodeStages = 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kDecodeStagesFp8 = 3;  // 5 KB per warp and stage; 69 KB per CTA: 3 CTAs (12 warps) per SM
 static_assert(DecodeCfg<kDecodeStagesFp8, true>::kSmemBytes <= 72 * 1024, "3 CTAs per SM");
+constexpr int kDecodeStagesSlim = 2;  // 48 KB per CTA: 4 CTAs per SM
+static_assert(DecodeCfg<kDecodeStagesSlim, true, true>::kSmemBytes <= 55 * 1024, "4 CTAs per SM");
 
 struct DecodeSmem {
     float wm[4][16];
@@ -81,7 +90,7 @@ struct DecodeSmem {
 // reuse the stage buffers: 4 x 16 rows x 136 floats = 34 KB.
 constexpr int kMergeStride = kDv + 8;
 static_assert(4 * 16 * kMergeStride * 4 <= kStageElems * 2, "merge slices fit in one stage buffer");
-static_assert(4 * 16 * kMergeStride * 4 <= kDecodeStagesFp8 * kLandBytes, "merge slices fit in the fp8 rings");
+static_assert(4 * 16 * kMergeStride * 4 <= kDecodeStagesSlim * kLandBytes, "merge slices fit in the fp8 rings");
 
 __device__ __forceinline__ int visible_count(int layer_type, int Lb, int window)
 {
@@ -93,10 +102,11 @@ __device__ __forceinline__ bool kv_len_ok(int layer_type, int Lb, int cap)
     return Lb >= 1 && (layer_type == 1 || Lb <= cap);
 }
 
-template <int kStages, bool kFp8 = false>
-__global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm)
+template <int kStages, bool kFp8 = false, bool kSlim = false>
+__global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8, kSlim>::kCtasPerSm)
     decode_mma_kernel(const __grid_constant__ LayerArgs L, const __grid_constant__ DecodeArgs a)
 {
+    static_assert(!kSlim || kFp8, "the slim form is the fp8 one");
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // Query rows: bf16, or f16 with fp8 caches. bf16: then the K/V stage
     // ring and the raw new k/v. fp8: the raw new k/v, the new token's codes
@@ -118,10 +128,13 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
     const int b = blockIdx.z;
     const int G = L.G;
     const int half = L.rope.half;
+    // kv_lens goes out first: every later step waits for it, and loads issued
+    // after the K/V tile copies would queue behind them.
+    const int Lb = __ldg(a.kv_lens + b);
 
     // The query rows of this KV group and the new token's k/v do not depend
-    // on kv_lens: their loads go out first, beside the kv_lens load, instead
-    // of one dependent round trip after another.
+    // on kv_lens: their loads go out beside it, instead of one dependent
+    // round trip after another.
     const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(a.q) +
                               ((size_t)b * L.Hq + (size_t)kvh * G) * kDqk;
     const bool vec_rope = L.rope.rotary_dim % 16 == 0;
@@ -154,8 +167,17 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
         nv = __ldg(reinterpret_cast<const uint4 *>(kn) + tid);
     else if (tid < 40)
         nv = __ldg(reinterpret_cast<const uint4 *>(vn) + (tid - 24));
+    // The sink logits of the group's heads are read now, not in the epilogue.
+    const float sink_in = (L.sinks != nullptr && tid < G) ? __ldg(L.sinks + kvh * G + tid) : 0.f;
 
-    const int Lb = __ldg(a.kv_lens + b);
+    const size_t kv_row = (size_t)L.Hkv;  // rows of the cache are [slot][Hkv][D]
+    const uint8_t *kc8 = reinterpret_cast<const uint8_t *>(a.k_cache) + ((size_t)b * a.cap * kv_row + kvh) * kDqk;
+    const uint8_t *vc8 = reinterpret_cast<const uint8_t *>(a.v_cache) + ((size_t)b * a.cap * kv_row + kvh) * kDv;
+    const __nv_bfloat16 *kc = reinterpret_cast<const __nv_bfloat16 *>(a.k_cache) +
+                              ((size_t)b * a.cap * kv_row + kvh) * kDqk;
+    const __nv_bfloat16 *vc = reinterpret_cast<const __nv_bfloat16 *>(a.v_cache) +
+                              ((size_t)b * a.cap * kv_row + kvh) * kDv;
+
     if (!kv_len_ok(L.layer_type, Lb, a.cap)) {
         if (split == 0 && kvh == 0 && tid == 0)
             atomicOr(a.err, kErrKvLen);
@@ -171,24 +193,18 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
     const bool owns_new = slot_new >= key_begin && slot_new < key_end;
     const double pos = (double)(Lb - 1);
 
-    const size_t kv_row = (size_t)L.Hkv;  // rows of the cache are [slot][Hkv][D]
-    const __nv_bfloat16 *kc = reinterpret_cast<const __nv_bfloat16 *>(a.k_cache) +
-                              ((size_t)b * a.cap * kv_row + kvh) * kDqk;
-    const __nv_bfloat16 *vc = reinterpret_cast<const __nv_bfloat16 *>(a.v_cache) +
-                              ((size_t)b * a.cap * kv_row + kvh) * kDv;
-
-    // The first K/V tiles go out before the query preparation below.
+    // The K/V tiles go out before the query preparation below: the whole
+    // ring of kStages tiles. Rows past the range and the new token's slot are
+    // zero-filled (the new token comes from its own copy; a slot past the
+    // range may hold any bits).
     const int n_tiles = (key_end - key_begin + kTileKeys - 1) / kTileKeys;
-    const uint8_t *kc8 = reinterpret_cast<const uint8_t *>(a.k_cache) + ((size_t)b * a.cap * kv_row + kvh) * kDqk;
-    const uint8_t *vc8 = reinterpret_cast<const uint8_t *>(a.v_cache) + ((size_t)b * a.cap * kv_row + kvh) * kDv;
     // Each thread copies a fixed pattern of 16-byte chunks in every tile, so
     // the shared-memory offsets are compile-time steps from one base and only
-    // the key rows change per tile. Rows past the range and the new token's
-    // slot are zero-filled (the new token comes from its own copy).
-    // bf16: K rows are 24 chunks: thread (key kr + 16i, chunk kch + 8j); V rows
-    // are 16 chunks: thread (key vr + 8i, chunk vch).
-    // fp8, per warp and its 16 keys: K rows are 12 chunks: lane (key fr + 8i,
-    // chunk fch + 4j); V rows are 8 chunks: lane (key gr + 4i, chunk gch).
+    // the key rows change per tile. bf16: K rows are 24 chunks: thread (key
+    // kr + 16i, chunk kch + 8j); V rows are 16 chunks: thread (key vr + 8i,
+    // chunk vch). fp8, per warp and its 16 keys: K rows are 12 chunks: lane
+    // (key fr + 8i, chunk fch + 4j); V rows are 8 chunks: lane (key gr + 4i,
+    // chunk gch).
     const int kr = tid >> 3, kch = tid & 7;
     const int vr = tid >> 4, vch = tid & 15;
     const int fr = lane >> 2, fch = lane & 3;
@@ -237,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
         }
     };
 #pragma unroll
-    for (int s = 0; s < kStages - 1; ++s) {
+    for (int s = 0; s < kStages; ++s) {
         if (s < n_tiles)
             issue(s);
         cp_async_commit();
@@ -246,11 +262,14 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
     // cos/sin of the new token's position for every rotary pair, once per CTA;
     // the raw new k/v chunks go to shared memory.
     __shared__ float2 s_cs[kMaxHalfRotary];
+    __shared__ float s_sink[16];
     for (int j = tid; j < half; j += kThreads) {
         float c, s;
         rope_cos_sin(pos, L.rope.inv_freq[j], c, s);
         s_cs[j] = make_float2(c, s);
     }
+    if (tid < 16)
+        s_sink[tid] = sink_in;
     if (tid < 24)
         reinterpret_cast<uint4 *>(sKnew)[tid] = nv;
     else if (tid < 40)
@@ -377,10 +396,14 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
     // lane read its key operands as whole words: in k-step ks, lane (g, tq)
     // holds dims tq*48 + 4*ks + {0, 1} (fragment k = 2tq, 2tq+1) and
     // tq*48 + 4*ks + {2, 3} (k = 2tq+8, 2tq+9), for the query as for the key.
-    uint32_t qa[12][4];
-    if constexpr (kFp8) {
-        const uint32_t *q0 = reinterpret_cast<const uint32_t *>(sQ + g * kQStride + tq * 48);
-        const uint32_t *q1 = reinterpret_cast<const uint32_t *>(sQ + (g + 8) * kQStride + tq * 48);
+    uint32_t qa[kSlim ? 1 : 12][4];
+    // fp8: the two words of k-step ks in rows g and g + 8 (64-bit reads)
+    const uint2 *q0w = reinterpret_cast<const uint2 *>(sQ + g * kQStride + tq * 48);
+    const uint2 *q1w = reinterpret_cast<const uint2 *>(sQ + (g + 8) * kQStride + tq * 48);
+    if constexpr (kSlim) {
+    } else if constexpr (kFp8) {
+        const uint32_t *q0 = reinterpret_cast<const uint32_t *>(q0w);
+        const uint32_t *q1 = reinterpret_cast<const uint32_t *>(q1w);
 #pragma unroll
         for (int ks = 0; ks < 12; ++ks) {
             qa[ks][0] = q0[2 * ks];
@@ -414,11 +437,15 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
         const __nv_bfloat16 *st = nullptr;   // bf16: the CTA's stage of tile t
         if constexpr (kFp8) {
             // The warp refills the ring entry of tile t - 1 once all its lanes
-            // are done with it, then waits for its own copies of tile t.
+            // are done with it, then waits for its own copies of tile t. The
+            // first kStages tiles went out before the loop, so tile t is
+            // always commit group t.
             __syncwarp();
-            if (t + kStages - 1 < n_tiles)
-                issue(t + kStages - 1);
-            cp_async_commit();
+            if (t > 0) {
+                if (t + kStages - 1 < n_tiles)
+                    issue(t + kStages - 1);
+                cp_async_commit();
+            }
             cp_async_wait<kStages - 1>();
             __syncwarp();
             if (base_key + kb >= key_end)
@@ -439,19 +466,38 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
                 const uint4 w0 = kr4[0], w1 = kr4[1], w2 = kr4[2];
                 const uint32_t kw[12] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w, w2.x, w2.y, w2.z, w2.w};
 #pragma unroll
-                for (int ks = 0; ks < 12; ++ks)
-                    mma_f16_16816((ks & 1) ? s_odd[nt] : s_acc[nt], qa[ks],
+                for (int ks = 0; ks < 12; ++ks) {
+                    uint32_t qf[4];
+                    if constexpr (kSlim) {
+                        const uint2 x0 = q0w[ks], x1 = q1w[ks];
+                        qf[0] = x0.x;
+                        qf[1] = x1.x;
+                        qf[2] = x0.y;
+                        qf[3] = x1.y;
+                    } else {
+                        qf[0] = qa[ks][0];
+                        qf[1] = qa[ks][1];
+                        qf[2] = qa[ks][2];
+                        qf[3] = qa[ks][3];
+                    }
+                    // (the slim form keeps one chain per n-tile: registers)
+                    mma_f16_16816((ks & 1) && !kSlim ? s_odd[nt] : s_acc[nt], qf,
                                   e4m3x2_to_f16x2((uint16_t)(kw[ks] & 0xFFFFu)),
                                   e4m3x2_to_f16x2((uint16_t)(kw[ks] >> 16)));
+                }
             }
         } else {
             // Tile t + kStages - 1 goes out before the wait for tile t, so
             // kStages tiles are in flight during it; the barrier first makes
             // sure every warp is done with the buffer it refills (tile t - 1's).
-            __syncthreads();
-            if (t + kStages - 1 < n_tiles)
-                issue(t + kStages - 1);
-            cp_async_commit();
+            // The first kStages tiles went out before the loop, so tile t is
+            // always commit group t.
+            if (t > 0) {
+                __syncthreads();
+                if (t + kStages - 1 < n_tiles)
+                    issue(t + kStages - 1);
+                cp_async_commit();
+            }
             cp_async_wait<kStages - 1>();
             __syncthreads();
             __nv_bfloat16 *stw = sStage + (t % kStages) * kStageElems;
@@ -484,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-                s_acc[nt][e] += s_odd[nt][e];
+                s_acc[nt][e] += kSlim ? 0.f : s_odd[nt][e];
         // Scale, mask keys past the end of the range (only the range's last
         // tile has any), online softmax.
         float mx0 = -INFINITY, mx1 = -INFINITY;
@@ -608,27 +654,19 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
     }
     const float f0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M0);
     const float f1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M1);
-    // Each warp writes its rescaled partial O into its own slice (rows padded
-    // to kMergeStride floats: the 8 rows of a warp's access fall in different
-    // banks), then one pass sums the four slices.
+    // Each warp writes its rescaled partial O into its own slice in fragment
+    // order (column 8d + n holds n-tile d, column n; rows padded to
+    // kMergeStride floats so the 8 rows of a warp's access fall in different
+    // banks), then one pass sums the four slices. With fp8 caches n-tile d,
+    // column n is output dim 16n + d: the summing pass undoes that.
     float *slices = reinterpret_cast<float *>(kFp8 ? sLand : reinterpret_cast<uint8_t *>(sStage));
     {
         float *sl = slices + warp * 16 * kMergeStride;
 #pragma unroll
         for (int d = 0; d < 16; ++d) {
-            if constexpr (kFp8) {
-                // undo the output-dim permutation: n-tile d, column n is dim n*16 + d
-                const int c0 = (2 * tq) * 16 + d, c1 = (2 * tq + 1) * 16 + d;
-                sl[g * kMergeStride + c0] = o[d][0] * f0;
-                sl[g * kMergeStride + c1] = o[d][1] * f0;
-                sl[(g + 8) * kMergeStride + c0] = o[d][2] * f1;
-                sl[(g + 8) * kMergeStride + c1] = o[d][3] * f1;
-            } else {
-                const int col = d * 8 + 2 * tq;
-                *reinterpret_cast<float2 *>(sl + g * kMergeStride + col) = make_float2(o[d][0] * f0, o[d][1] * f0);
-                *reinterpret_cast<float2 *>(sl + (g + 8) * kMergeStride + col) =
-                    make_float2(o[d][2] * f1, o[d][3] * f1);
-            }
+            const int col = d * 8 + 2 * tq;
+            *reinterpret_cast<float2 *>(sl + g * kMergeStride + col) = make_float2(o[d][0] * f0, o[d][1] * f0);
+            *reinterpret_cast<float2 *>(sl + (g + 8) * kMergeStride + col) = make_float2(o[d][2] * f1, o[d][3] * f1);
         }
     }
     __syncthreads();
@@ -647,27 +685,40 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
             Ls += (red.wm[w][r] == -INFINITY) ? 0.f : red.wl[w][r] * exp2f(red.wm[w][r] - M);
         // this row's 16 columns, summed over the four warps' slices
         float v[16];
+        if constexpr (kFp8) {
+            // output dims c0 + j = 16n + d with n = c0 / 16, d = j: column 8j + n
+            const int n = c0 >> 4;
 #pragma unroll
-        for (int c = 0; c < 16; c += 4) {
-            float4 acc = *reinterpret_cast<const float4 *>(slices + r * kMergeStride + c0 + c);
+            for (int j = 0; j < 16; ++j) {
+                float acc = slices[r * kMergeStride + 8 * j + n];
 #pragma unroll
-            for (int w = 1; w < 4; ++w) {
-                const float4 x = *reinterpret_cast<const float4 *>(slices + (w * 16 + r) * kMergeStride + c0 + c);
-                acc.x += x.x;
-                acc.y += x.y;
-                acc.z += x.z;
-                acc.w += x.w;
+                for (int w = 1; w < 4; ++w)
+                    acc += slices[(w * 16 + r) * kMergeStride + 8 * j + n];
+                v[j] = acc;
             }
-            v[c] = acc.x;
-            v[c + 1] = acc.y;
-            v[c + 2] = acc.z;
-            v[c + 3] = acc.w;
+        } else {
+#pragma unroll
+            for (int c = 0; c < 16; c += 4) {
+                float4 acc = *reinterpret_cast<const float4 *>(slices + r * kMergeStride + c0 + c);
+#pragma unroll
+                for (int w = 1; w < 4; ++w) {
+                    const float4 x = *reinterpret_cast<const float4 *>(slices + (w * 16 + r) * kMergeStride + c0 + c);
+                    acc.x += x.x;
+                    acc.y += x.y;
+                    acc.z += x.z;
+                    acc.w += x.w;
+                }
+                v[c] = acc.x;
+                v[c + 1] = acc.y;
+                v[c + 2] = acc.z;
+                v[c + 3] = acc.w;
+            }
         }
         const int h = kvh * G + r;
         if (nsplit == 1) {
             float scale;
             if (L.sinks != nullptr) {
-                const float s2 = __ldg(L.sinks + h) * kLog2e;
+                const float s2 = s_sink[r] * kLog2e;
                 const float mf = fmaxf(M, s2);
                 const float al = exp2f(M - mf);
                 scale = al * L.v_scale / (Ls * al + exp2f(s2 - mf));
@@ -699,13 +750,21 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8>::kCtasPerSm
     }
 }
 
-// Merges the split partials of one (batch, query head): log-sum-exp merge,
-// sink folded into the denominator, V scale applied.
+// Merges the split partials of one (batch, query head) per warp (Dv 128):
+// log-sum-exp merge, sink folded into the denominator, V scale applied. grid
+// (Hq / 4, batch), 4 warps. Lane s holds split s's (m, l) (more splits:
+// strided loops); each lane takes four output dims as two float2 reads of
+// every split's partial O (8-byte aligned: rows of Dv + 2 floats).
 template <typename T>
-__global__ void decode_combine_kernel(const __grid_constant__ LayerArgs L, const __grid_constant__ DecodeArgs a)
+__global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_constant__ LayerArgs L,
+                                                             const __grid_constant__ DecodeArgs a)
 {
-    const int h = blockIdx.x;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int h = blockIdx.x * 4 + warp;
     const int b = blockIdx.y;
+    if (h >= L.Hq)
+        return;
     const int Lb = __ldg(a.kv_lens + b);
     if (!kv_len_ok(L.layer_type, Lb, a.cap))
         return;
@@ -713,29 +772,63 @@ __global__ void decode_combine_kernel(const __grid_constant__ LayerArgs L, const
     const int nsplit = (n_vis + a.chunk - 1) / a.chunk;
     if (nsplit <= 1)
         return;
-    const float *part = a.partial + ((size_t)b * L.Hq + h) * a.max_splits * (L.Dv + 2);
-    float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s)
-        M = fmaxf(M, part[(size_t)s * (L.Dv + 2) + L.Dv]);
-    float s2 = -INFINITY;
-    if (L.sinks != nullptr) {
-        s2 = __ldg(L.sinks + h) * kLog2e;
-        M = fmaxf(M, s2);
+    const int stride = L.Dv + 2;
+    const float *part = a.partial + ((size_t)b * L.Hq + h) * a.max_splits * stride;
+    const float s2 = L.sinks != nullptr ? __ldg(L.sinks + h) * kLog2e : -INFINITY;
+    // every split holds at least one key, so its m is finite
+    float m_l = -INFINITY, l_l = 0.f;
+    if (lane < nsplit) {
+        m_l = part[(size_t)lane * stride + L.Dv];
+        l_l = part[(size_t)lane * stride + L.Dv + 1];
     }
-    float Ls = (L.sinks != nullptr) ? exp2f(s2 - M) : 0.f;
-    for (int s = 0; s < nsplit; ++s) {
-        const float *ps = part + (size_t)s * (L.Dv + 2);
+    float M = fmaxf(m_l, s2);
+    for (int s = lane + 32; s < nsplit; s += 32)
+        M = fmaxf(M, part[(size_t)s * stride + L.Dv]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float w_l = lane < nsplit ? exp2f(m_l - M) : 0.f;  // weight of split `lane`
+    float Ls = w_l * l_l;
+    for (int s = lane + 32; s < nsplit; s += 32) {
+        const float *ps = part + (size_t)s * stride;
         Ls += ps[L.Dv + 1] * exp2f(ps[L.Dv] - M);
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+    if (L.sinks != nullptr)
+        Ls += exp2f(s2 - M);
     const float scale = L.v_scale / Ls;
-    for (int e = threadIdx.x; e < L.Dv; e += blockDim.x) {
-        float acc = 0.f;
-        for (int s = 0; s < nsplit; ++s) {
-            const float *ps = part + (size_t)s * (L.Dv + 2);
-            acc += ps[e] * exp2f(ps[L.Dv] - M);
+    // dims 2 lane, 2 lane + 1 and 64 + 2 lane, 65 + 2 lane (Dv 128), splits
+    // in batches of 8 whose loads all go out before the sums
+    T *out = reinterpret_cast<T *>(a.out) + ((size_t)b * L.Hq + h) * kDv;
+    float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+    for (int s0 = 0; s0 < nsplit; s0 += 8) {
+        float2 o0[8], o1[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float *ps = part + (size_t)(s0 + j) * stride + 2 * lane;
+            o0[j] = s0 + j < nsplit ? *reinterpret_cast<const float2 *>(ps) : make_float2(0.f, 0.f);
+            o1[j] = s0 + j < nsplit ? *reinterpret_cast<const float2 *>(ps + 64) : make_float2(0.f, 0.f);
         }
-        reinterpret_cast<T *>(a.out)[((size_t)b * L.Hq + h) * L.Dv + e] = from_f32<T>(acc * scale);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int s = s0 + j;
+            float w;
+            if (s < 32)
+                w = __shfl_sync(0xffffffffu, w_l, s);
+            else
+                w = s < nsplit ? exp2f(part[(size_t)s * stride + kDv] - M) : 0.f;
+            acc0.x += w * o0[j].x;
+            acc0.y += w * o0[j].y;
+            acc1.x += w * o1[j].x;
+            acc1.y += w * o1[j].y;
+        }
     }
+    out[2 * lane] = from_f32<T>(acc0.x * scale);
+    out[2 * lane + 1] = from_f32<T>(acc0.y * scale);
+    out[64 + 2 * lane] = from_f32<T>(acc1.x * scale);
+    out[65 + 2 * lane] = from_f32<T>(acc1.y * scale);
 }
 
 // ------------------------------------------------------- CUDA-core path
@@ -917,18 +1010,25 @@ cudaError_t launch_decode(const LayerArgs &L, const DecodeArgs &a, int dtype, cu
     if (a.fp8_cache && !decode_mma_supported(L, dtype))
         return cudaErrorInvalidValue;
     if (decode_mma_supported(L, dtype)) {
-        static std::atomic<unsigned long long> prepared[2] = {{0}, {0}};
-        const int f = a.fp8_cache ? 1 : 0;
+        static std::atomic<unsigned long long> prepared[3] = {{0}, {0}, {0}};
+        // fp8 sliding layers whose ring is at most two tiles take the slim form
+        const int f = a.fp8_cache ? (L.layer_type == 1 && L.window <= 2 * kTileKeys ? 2 : 1) : 0;
         {
-            cudaError_t e = f ? prepare_kernel_once(decode_mma_kernel<kDecodeStagesFp8, true>,
-                                                    DecodeCfg<kDecodeStagesFp8, true>::kSmemBytes, prepared[1])
-                              : prepare_kernel_once(decode_mma_kernel<kDecodeStages, false>,
-                                                    DecodeCfg<kDecodeStages, false>::kSmemBytes, prepared[0]);
+            cudaError_t e =
+                f == 2 ? prepare_kernel_once(decode_mma_kernel<kDecodeStagesSlim, true, true>,
+                                             DecodeCfg<kDecodeStagesSlim, true, true>::kSmemBytes, prepared[2])
+                : f == 1 ? prepare_kernel_once(decode_mma_kernel<kDecodeStagesFp8, true>,
+                                               DecodeCfg<kDecodeStagesFp8, true>::kSmemBytes, prepared[1])
+                         : prepare_kernel_once(decode_mma_kernel<kDecodeStages, false>,
+                                               DecodeCfg<kDecodeStages, false>::kSmemBytes, prepared[0]);
             if (e != cudaSuccess)
                 return e;
         }
         dim3 grid(a.max_splits, L.Hkv, a.B);
-        if (f)
+        if (f == 2)
+            decode_mma_kernel<kDecodeStagesSlim, true, true>
+                <<<grid, kThreads, DecodeCfg<kDecodeStagesSlim, true, true>::kSmemBytes, stream>>>(L, a);
+        else if (f == 1)
             decode_mma_kernel<kDecodeStagesFp8, true>
                 <<<grid, kThreads, DecodeCfg<kDecodeStagesFp8, true>::kSmemBytes, stream>>>(L, a);
         else
@@ -937,7 +1037,7 @@ cudaError_t launch_decode(const LayerArgs &L, const DecodeArgs &a, int dtype, cu
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess || a.max_splits <= 1)
             return e;
-        decode_combine_kernel<__nv_bfloat16><<<dim3(L.Hq, a.B), 128, 0, stream>>>(L, a);
+        decode_combine_kernel<__nv_bfloat16><<<dim3((L.Hq + 3) / 4, a.B), 128, 0, stream>>>(L, a);
         return cudaGetLastError();
     }
     dim3 g1(L.Hkv, a.B);

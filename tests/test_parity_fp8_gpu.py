@@ -155,6 +155,38 @@ def test_decode_fp8_small_every_output(layer_type):
     _check_fp8(spec, out, q, kn, vn, kc0, vc0, kc, vc, sinks, range(len(lens)), lens)
 
 
+@pytest.mark.parametrize("layer_type", [0, 1])
+def test_decode_fp8_stale_slots_hold_nan(layer_type):
+    """E4M3 NaN codes (0x7F, 0xFF) in every slot a sequence has not written
+    yet leave the output equal to the one from finite caches."""
+    spec = synthetic.mimo_layer(layer_type)
+    lens = [1, 2, 63, 64, 65, 100, 127, 128, 129, 191, 192, 300]
+    kv_lens, q, kn, vn, kc, vc, sinks = _fp8_inputs(spec, len(lens), 512, lens, seed=6)
+    kc0, vc0 = kc.clone(), vc.clone()
+    for b, L in enumerate(lens):
+        kc[b, L:] = 0x7F
+        vc[b, L:] = 0xFF
+    lay = lib_layer(spec, sinks)
+    out = mimo.decode_fp8kv(lay, q, kn, vn, kv_lens.cuda(), kc, vc, K_SCALE, V_SCALE)
+    torch.cuda.synchronize()
+    assert mimo.mimo_attn_get_device_error() == 0
+    assert bool(torch.isfinite(out).all())
+    G = spec.num_q_heads // spec.num_kv_heads
+    vscale = oracle.v_scale(spec.hidden_size, spec.num_q_heads, spec.v_dim)
+    gpu, ref = [], []
+    for b, L in enumerate(lens):
+        for kv in range(spec.num_kv_heads):
+            hs = slice(kv * G, (kv + 1) * G)
+            o, _, _ = oracle.decode_fp8kv(
+                f64(q[b, hs]), f64(kn[b, kv]), f64(vn[b, kv]), kc0[b, :, kv].cpu().numpy(),
+                vc0[b, :, kv].cpu().numpy(), L, spec.rotary_dim, spec.theta, spec.layer_type, spec.window,
+                1 / math.sqrt(spec.qk_dim), None if sinks is None else f64(sinks[hs]), vscale, K_SCALE, V_SCALE)
+            gpu.append(f64(out[b, hs]))
+            ref.append(o)
+    c = compare(np.concatenate(gpu), np.concatenate(ref))
+    assert c.max_abs <= 2e-2 and c.mean_abs <= 2e-3, f"fp8 decode, NaN codes: max {c.max_abs:.3e} mean {c.mean_abs:.3e}"
+
+
 def test_decode_fp8_full_size_sampled_batches():
     """Decode workload shape (B64, L ~ U[1024, 32768], cache 32768) with fp8
     caches: one global and one SWA layer, every head of 6 sampled sequences."""

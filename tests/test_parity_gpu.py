@@ -246,6 +246,38 @@ def test_decode_small_every_output(layer_type):
 
 
 @pytest.mark.parametrize("layer_type", [0, 1])
+def test_decode_stale_slots_hold_nan(layer_type):
+    """Cache slots past a sequence's length may hold any bits: with NaN in
+    every slot a sequence has not written yet (global: slots >= L; ring:
+    slots >= L while L < window), the output equals the one from finite
+    caches. Lengths cover the first tiles, which the kernel loads before it
+    reads kv_lens."""
+    spec = synthetic.mimo_layer(layer_type)
+    lens = [1, 2, 63, 64, 65, 100, 127, 128, 129, 191, 192, 300]
+    B, cap = len(lens), 512
+    kv_lens = torch.tensor(lens, dtype=torch.int32)
+    q, kn, vn, kc, vc, sinks = synthetic.decode_inputs(spec, B, cap, kv_lens, seed=5, layer=0, dtype=BF,
+                                                       device="cuda")
+    sinks = sinks if layer_type == 1 else None
+    kc0, vc0 = kc.clone(), vc.clone()
+    for b, L in enumerate(lens):
+        kc[b, L:] = float("nan")
+        vc[b, L:] = float("nan")
+    lay = lib_layer(spec, sinks)
+    out = mimo.decode(lay, q, kn, vn, kv_lens.cuda(), kc, vc)
+    torch.cuda.synchronize()
+    assert mimo.mimo_attn_get_device_error() == 0
+    assert bool(torch.isfinite(out).all())
+    G = spec.num_q_heads // spec.num_kv_heads
+    gpu, ref = [], []
+    for b, L in enumerate(lens):
+        for kv, (o, _, _) in enumerate(_oracle_decode(spec, b, L, q, kn, vn, kc0, vc0, sinks)):
+            gpu.append(f64(out[b, kv * G:(kv + 1) * G]))
+            ref.append(o)
+    _assert(compare(np.concatenate(gpu), np.concatenate(ref)), BF, "decode, NaN in unwritten slots")
+
+
+@pytest.mark.parametrize("layer_type", [0, 1])
 def test_decode_fp32_cuda_core_path(layer_type):
     spec = synthetic.LayerSpec(layer_type, 4, 2 if layer_type else 1, 48, 32, 16, 16,
                                1e4 if layer_type else 1e6, 256, layer_type == 1)
