@@ -16,16 +16,17 @@
 // Two workers take alternate tiles (tile n goes to worker n % 2), so one
 // worker's softmax overlaps the other tile's MMAs and epilogue. A worker is
 // two warpgroups, one per column half: the thread pair (row r, half 0) and
-// (row r, half 1) shares query row r. The pair moves the row's Q from shared
-// memory into TMEM, applying the partial RoPE on the way (cos / sin from the
-// per-call table; each half 16 of the 32 pairs), and releases the Q buffer
-// at once: QK^T reads A from TMEM, so the next Q tile's load starts a whole
-// tile earlier than if the buffer waited for the MMA, and the kernel, whose
-// limit is the bytes it keeps in flight, gets more loads going. The pair then
-// runs the softmax (each half 72 of the 144 S columns from TMEM: window mask,
-// max exchanged through shared memory, P as bf16 written back over the S
-// columns) and the epilogue (64 of the 128 O columns: sink fold, normalise,
-// V scale, store).
+// (row r, half 1) shares query row r. The pair runs the softmax (each half 72
+// of the 144 S columns from TMEM: window mask, max exchanged through shared
+// memory, P as bf16 written back over the S columns) and the epilogue (64 of
+// the 128 O columns: sink fold, normalise, V scale, store). Between the two,
+// while PV runs, it moves the first 64 dims of the row's next Q tile from
+// shared memory into TMEM, applying the partial RoPE on the way (cos / sin
+// from the per-call table; each half 16 of the 32 pairs): QK^T takes those
+// four k-steps' A operand from TMEM and the other eight straight from the Q
+// buffer, which its commit then frees. So a tile's QK^T can start as soon as
+// the epilogue of the worker's previous tile has read O, and it runs while
+// that epilogue's stores drain.
 //
 // The keys arrive unrotated in a plain prefill: the Q-producer warp rotates
 // each 16-key block in the ring once it lands, before any QK^T reads it. (A
@@ -41,10 +42,9 @@
 //   warp 19             TMA producer of the K/V ring blocks
 //
 // TMEM (512 columns), per worker t: S_t = [256t, 256t + 144),
-// Q_t = [256t + 144, 256t + 240) (192 bf16 as pairs) and
-// O_t = [256t + 72, 256t + 200). O overlaps the upper S columns, which are
-// dead once the softmax has read them, and Q, dead once QK^T has read it;
-// P (bf16) takes the first 72 columns.
+// O_t = [256t + 72, 256t + 200) and Q_t = [256t + 200, 256t + 232) (dims
+// 0 .. 63 as bf16 pairs). O overlaps the upper S columns, which are dead once
+// the softmax has read them; P (bf16) takes the first 72 columns.
 // Shared memory: Q 2 x 48 KB; K ring 12 x 16 keys x 384 B; V ring 12 x 16
 // keys x 256 B (128B-swizzled 64-column blocks, 1024-byte aligned).
 #include "kernels.cuh"
@@ -82,7 +82,7 @@ constexpr int kWarpQ = 16, kWarpMma0 = 17, kWarpKV = 19;
 
 __device__ __forceinline__ uint32_t col_s(int t) { return t ? 256u : 0u; }
 __device__ __forceinline__ uint32_t col_o(int t) { return col_s(t) + 72u; }
-__device__ __forceinline__ uint32_t col_q(int t) { return col_s(t) + 144u; }
+__device__ __forceinline__ uint32_t col_q(int t) { return col_s(t) + 200u; }
 
 struct SwaParams {
     CUtensorMap tm_q;  // [B, S, Hq, Dqk]    box {64, gp, P, 1}
@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->q_full[i], 1);
             mbar_init(&bars->q_ready[i], kWorkerThreads);
-            mbar_init(&bars->q_empty[i], kWorkerThreads);  // the workers copied Q into TMEM
+            mbar_init(&bars->q_empty[i], 1);  // QK^T of the tile has read the buffer
             mbar_init(&bars->s_full[i], 1);
             mbar_init(&bars->p_full[i], kWorkerThreads);
             mbar_init(&bars->o_full[i], 1);
@@ -404,6 +404,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
             const uint32_t idesc_pv = idesc_bf16_f32(kBlockM, kDv, false, true);
             const uint32_t k_lo = sdesc_lo(smem_u32(sK), 16);
             const uint32_t v_lo = sdesc_lo(smem_u32(sV), kVAtom);
+            const uint32_t q_lo = sdesc_lo(smem_u32(sQ + t * kQBytes), 16);  // this worker's Q buffer
+            constexpr uint32_t kQBoxStep = (kBlockM * 128) >> 4;
             constexpr uint32_t kKAtomStep = kKAtom >> 4;
             constexpr uint32_t kSlotStep = (kKeyBlock * 128) >> 4;
             const uint32_t s_col = tmem + col_s(t), o_col = tmem + col_o(t), q_col = tmem + col_q(t);
@@ -424,18 +426,29 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                     nb = c.last_block - c.first_block + 1;
                 }
             };
-            // S_t = Q_t K^T over the entries [e0, e0 + nb): one group of 12
-            // MMAs (N = 16 keys per entry, A = 16 dims of Q_t = 8 TMEM
-            // columns), two groups when the span wraps the ring.
-            auto qk_part = [&](uint32_t d, int slot, int blocks) {
-                const uint32_t idesc = idesc_bf16_f32(kBlockM, blocks * kKeyBlock, false, false);
-                const uint32_t kb = k_lo + (uint32_t)slot * kSlotStep;
-#pragma unroll
-                for (int atom = 0; atom < 3; ++atom)
+            // S_t = Q_t K^T over the entries [e0, e0 + nb): groups of 12
+            // MMAs (K = 16 dims each) over at most 8 entries (N <= 128 keys:
+            // with A in shared memory, N = 144 ran at about half the rate of
+            // 128 + 16), split again where the span wraps the ring. The first
+            // four k-steps take A from TMEM (dims 0 .. 63, rotated by the
+            // workers: 8 columns per k-step), the other eight from the Q
+            // buffer's 64-column blocks 1 and 2.
+            auto qk_part = [&](uint32_t d0, int slot0, int blocks0) {
+                for (int b0 = 0; b0 < blocks0; b0 += 8) {
+                    const int blocks = min(8, blocks0 - b0);
+                    const uint32_t d = d0 + (uint32_t)(b0 * kKeyBlock);
+                    const uint32_t idesc = idesc_bf16_f32(kBlockM, blocks * kKeyBlock, false, false);
+                    const uint32_t kb = k_lo + (uint32_t)(slot0 + b0) * kSlotStep;
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4)
-                        umma_ts_lo(d, q_col + (uint32_t)(8 * (4 * atom + k4)), kb + atom * kKAtomStep + 2 * k4, idesc,
-                                   (atom | k4) ? 1u : 0u);
+                        umma_ts_lo(d, q_col + (uint32_t)(8 * k4), kb + 2 * k4, idesc, k4 ? 1u : 0u);
+#pragma unroll
+                    for (int atom = 1; atom < 3; ++atom)
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4)
+                            umma_ss_lo(d, q_lo + atom * kQBoxStep + 2 * k4, kb + atom * kKAtomStep + 2 * k4, idesc,
+                                       1u);
+                }
             };
             int known_full = 0;  // entries [0, known_full) have landed (and are rotated)
             int freed = 0;       // entries [0, freed) committed by this issuer
@@ -464,6 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 if (nb > run1)
                     qk_part(s_col + (uint32_t)(run1 * kKeyBlock), 0, nb - run1);
                 umma_commit(&bars->s_full[t]);
+                umma_commit(&bars->q_empty[t]);  // the Q buffer may take the worker's next tile
                 // O_t = P_t V over the same entries, one N = 128 MMA per entry.
                 wait(&bars->p_full[t], ph);
                 tc_fence_after();
@@ -507,30 +521,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
         const int half = p.rope_half;
         const float sc = p.scale_log2;
         const bool fast_rope = half == 32 && p.P == 16;
-        bool ok = true;
-        for (int n = t; ok && n < n_local; n += 2) {
-            const uint32_t ph = (uint32_t)(n >> 1) & 1u;
-            const Tile c = tile_at(p, t_begin + n);
+        // Q tile nn's first 64 dims into TMEM (the A operand of the first four
+        // k-steps of QK^T; the other eight read the Q buffer), partial RoPE on
+        // the way. Half hf takes rotary pairs 16hf .. 16hf + 15: 16-byte
+        // chunks 2hf, 2hf + 1 and their partners 4 chunks up. Dims (2c, 2c + 1)
+        // form TMEM column c of Q_t. Other rotary widths rotate every rotary
+        // dim in place in the buffer first (both halves, then a barrier).
+        auto load_q = [&](int nn) -> bool {
+            const uint32_t ph = (uint32_t)(nn >> 1) & 1u;
+            const Tile c = tile_at(p, t_begin + nn);
             const int i = c.p0 + row / p.gp;
-            const int h = c.h0 + row % p.gp;
-            // cached tokens before this chunk (0 for a plain prefill): query i
-            // has position past + i; key rows below key_off - past precede
-            // position 0 and are never visible
             const int past = p.past_lens != nullptr ? min(max(__ldg(p.past_lens + c.b), 0), p.max_past) : 0;
             const bool rot = i < p.S && half > 0;
-            if (!mbar_wait(&bars->q_full[t], ph, abort_flag, p.err)) {
-                ok = false;
-                break;
-            }
-            // ---- this row's Q_n into TMEM (the A operand of QK^T), partial
-            // RoPE on the way. Half hf takes rotary pairs 16hf .. 16hf + 15
-            // (16-byte chunks 2hf, 2hf + 1 of the first 64-column block and
-            // their partners 4 chunks up) and the pass-through dims of block
-            // 1 + hf. Dims (2c, 2c + 1) form TMEM column c of Q_t.
+            if (!mbar_wait(&bars->q_full[t], ph, abort_flag, p.err))
+                return false;
             uint8_t *q_row = sQ + t * kQBytes + row * 128;
             if (half > 0 && !fast_rope) {
-                // other rotary widths: rotate in place in shared memory first
-                // (pairs j = hf, hf + 2, ...), then copy like the fast path;
                 // every thread arrives, rows past the sequence end included
                 const float2 *cs = p.rope_table + (size_t)(past + i) * half;
                 for (int j = hf; rot && j < half; j += 2) {
@@ -546,64 +552,51 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                     *pb = __float2bfloat16_rn(xb * cj.x + xa * cj.y);
                 }
                 mbar_arrive(&bars->qrot[t]);
-                if (!mbar_wait(&bars->qrot[t], ph, abort_flag, p.err)) {
-                    ok = false;
-                    break;
-                }
+                if (!mbar_wait(&bars->qrot[t], ph, abort_flag, p.err))
+                    return false;
             }
-            // Q_t's columns hold O of tile n - 2 until both halves have read it
-            if (n >= 2 && !mbar_wait(&bars->o_free[t], ph ^ 1u, abort_flag, p.err)) {
-                ok = false;
-                break;
+            uint4 ca[2], cb[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int ch = 2 * hf + k;
+                ca[k] = *reinterpret_cast<const uint4 *>(q_row + ((ch ^ (row & 7)) << 4));
+                cb[k] = *reinterpret_cast<const uint4 *>(q_row + (((ch + 4) ^ (row & 7)) << 4));
             }
-            tc_fence_after();
-            {
-                // rotary chunks 2hf, 2hf + 1 and their partners 2hf + 4, 2hf + 5
-                uint4 ca[2], cb[2];
+            if (rot && fast_rope) {
+                // this half's 16 (cos, sin) pairs from the table (the
+                // producer warp read the same rows for the keys: L1 hits)
+                const float4 *g = reinterpret_cast<const float4 *>(p.rope_table + (size_t)(past + i) * 32) + 8 * hf;
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
-                    const int ch = 2 * hf + k;
-                    ca[k] = *reinterpret_cast<const uint4 *>(q_row + ((ch ^ (row & 7)) << 4));
-                    cb[k] = *reinterpret_cast<const uint4 *>(q_row + (((ch + 4) ^ (row & 7)) << 4));
-                }
-                if (rot && fast_rope) {
-                    // this half's 16 (cos, sin) pairs from the table (the
-                    // producer warp read the same rows for the keys: L1 hits)
-                    const float4 *g = reinterpret_cast<const float4 *>(p.rope_table + (size_t)(past + i) * 32) + 8 * hf;
+                    float4 cs[4];
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        float4 cs[4];
-#pragma unroll
-                        for (int w = 0; w < 4; ++w)
-                            cs[w] = __ldg(g + 4 * k + w);  // pairs 8 (2hf + k) + 2w, + 1
-                        rope_chunk_pair(ca[k], cb[k], cs);
-                    }
+                    for (int w = 0; w < 4; ++w)
+                        cs[w] = __ldg(g + 4 * k + w);  // pairs 8 (2hf + k) + 2w, + 1
+                    rope_chunk_pair(ca[k], cb[k], cs);
                 }
-                const uint32_t lo8[8] = {ca[0].x, ca[0].y, ca[0].z, ca[0].w, ca[1].x, ca[1].y, ca[1].z, ca[1].w};
-                const uint32_t hi8[8] = {cb[0].x, cb[0].y, cb[0].z, cb[0].w, cb[1].x, cb[1].y, cb[1].z, cb[1].w};
-                tmem_st8(q_addr + 8 * hf, lo8);       // dims 16hf .. 16hf + 15
-                tmem_st8(q_addr + 16 + 8 * hf, hi8);  // dims 32 + 16hf .. 32 + 16hf + 15
             }
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {  // block 1 + hf: dims 64 (1 + hf) .. 64 (1 + hf) + 63
-                uint32_t w16[16];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(q_row + (1 + hf) * (kBlockM * 128) +
-                                                                      (((4 * part + k) ^ (row & 7)) << 4));
-                    w16[4 * k] = v.x;
-                    w16[4 * k + 1] = v.y;
-                    w16[4 * k + 2] = v.z;
-                    w16[4 * k + 3] = v.w;
-                }
-                tmem_st16(q_addr + 32 + 32 * hf + 16 * part, w16);
-            }
+            const uint32_t lo8[8] = {ca[0].x, ca[0].y, ca[0].z, ca[0].w, ca[1].x, ca[1].y, ca[1].z, ca[1].w};
+            const uint32_t hi8[8] = {cb[0].x, cb[0].y, cb[0].z, cb[0].w, cb[1].x, cb[1].y, cb[1].z, cb[1].w};
+            tmem_st8(q_addr + 8 * hf, lo8);       // dims 16hf .. 16hf + 15
+            tmem_st8(q_addr + 16 + 8 * hf, hi8);  // dims 32 + 16hf .. 32 + 16hf + 15
             if (half > 0 && !fast_rope)
-                fence_proxy_async_smem();  // the in-place rotation's writes, before the next TMA fill
-            mbar_arrive(&bars->q_empty[t]);  // this thread's reads of the Q buffer are done
+                fence_proxy_async_smem();  // the in-place rotation, before QK^T reads the buffer
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars->q_ready[t]);
+            return true;
+        };
+        bool ok = t >= n_local || load_q(t);
+        for (int n = t; ok && n < n_local; n += 2) {
+            const uint32_t ph = (uint32_t)(n >> 1) & 1u;
+            const Tile c = tile_at(p, t_begin + n);
+            const int i = c.p0 + row / p.gp;
+            const int h = c.h0 + row % p.gp;
+            // cached tokens before this chunk (0 for a plain prefill): query i
+            // has position past + i; key rows below key_off - past precede
+            // position 0 and are never visible
+            const int past = p.past_lens != nullptr ? min(max(__ldg(p.past_lens + c.b), 0), p.max_past) : 0;
+            const float sink = p.sinks != nullptr ? __ldg(p.sinks + h) : 0.f;  // read now, used in the epilogue
 
             // ---- softmax over the tile's key span, this half's 72 columns
             const int k0 = c.first_block * kKeyBlock;
@@ -694,6 +687,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
             tc_fence_before();
             mbar_arrive(&bars->p_full[t]);
 
+            // ---- while PV runs: the rotary block of this worker's next Q
+            // tile into TMEM (QK^T of this tile, complete at s_full, has read
+            // Q_t), so that tile's QK^T can start as soon as O is read below.
+            if (n + 2 < n_local && !load_q(n + 2)) {
+                ok = false;
+                break;
+            }
+
             // ---- epilogue: this half's 64 output columns. The p_full wait
             // returns at once (the PV behind o_full needed it) and orders the
             // partner's row sum, read before o_free lets the next tile reuse it.
@@ -703,14 +704,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 break;
             }
             const float rs = rs_half + red_sum[(hf ^ 1) * kBlockM + row];
+            // (rs >= 1: the row maximum's own term; approximate exp2 and
+            // division, well inside bf16 output rounding)
             float o_scale;
             if (p.sinks != nullptr) {
-                const float s2 = __ldg(p.sinks + h) * kLog2e;
+                const float s2 = sink * kLog2e;
                 const float mf = fmaxf(m2, s2);
-                const float a = exp2f(m2 - mf);
-                o_scale = a * p.v_scale / (rs * a + exp2f(s2 - mf));
+                const float a = fast_exp2(m2 - mf);
+                o_scale = __fdividef(a * p.v_scale, rs * a + fast_exp2(s2 - mf));
             } else {
-                o_scale = p.v_scale / rs;
+                o_scale = __fdividef(p.v_scale, rs);
             }
             tc_fence_after();
             uint32_t o[2][32];
