@@ -155,6 +155,18 @@ def test_decode_fp8_small_every_output(layer_type):
     _check_fp8(spec, out, q, kn, vn, kc0, vc0, kc, vc, sinks, range(len(lens)), lens)
 
 
+@pytest.mark.parametrize("window", [16, 64, 100, 128, 192, 256])
+def test_decode_fp8_sliding_windows(window):
+    """Sliding layers with rings of one to four 64-key tiles: up to two tiles
+    take the slim kernel form (4 CTAs per SM), longer rings the 3-stage one.
+    Lengths below, at and past the window; every output."""
+    spec = synthetic.mimo_layer(1, window=window)
+    lens = sorted({1, 2, window - 1, window, window + 1, 2 * window + 3, 700})
+    lens = [L for L in lens if L >= 1]
+    out, (q, kn, vn, kc0, vc0, kc, vc, sinks) = _run_fp8(spec, len(lens), window, lens, seed=window)
+    _check_fp8(spec, out, q, kn, vn, kc0, vc0, kc, vc, sinks, range(len(lens)), lens)
+
+
 @pytest.mark.parametrize("layer_type", [0, 1])
 def test_decode_fp8_stale_slots_hold_nan(layer_type):
     """E4M3 NaN codes (0x7F, 0xFF) in every slot a sequence has not written
