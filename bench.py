@@ -433,12 +433,19 @@ class StackWorkload:
 class HostInputs:
     """Pinned host buffers of every step input and result. Layers of the same
     shape share one pinned set (bounded host memory); each step still copies
-    every layer's full inputs host->device and its full result back."""
+    every layer's full inputs host->device and its full result back.
+
+    The copies are pipelined with the compute, as a serving loop would: per
+    prefill layer, its inputs go host->device on one copy stream, the layer
+    runs on the compute stream once they have landed, and its output goes
+    device->host on a second copy stream (the two directions use separate
+    copy engines). The decode stack's inputs follow the prefill inputs, and
+    its outputs are read back after it. Per-layer events keep the next step's
+    copies off buffers still in use: a layer's inputs are overwritten only
+    after its compute has read them, its output only after it was read back."""
 
     def __init__(self, w: StackWorkload):
         self.w = w
-        self.items_in = []
-        self.items_out = []
         shared = {}
 
         def pinned_like(t, key, fill_from=None):
@@ -450,25 +457,58 @@ class HostInputs:
                 shared[k] = h
             return shared[k]
 
+        # one unit per prefill layer, then one for the whole decode stack
+        self.units = []
         for L in w.prefill_layers:
-            for key in ("q", "k", "v"):
-                self.items_in.append((L[key], pinned_like(L[key], key, L[key])))
-            self.items_out.append((L["out"], pinned_like(L["out"], "out")))
-        for L in w.decode_layers:
-            for key in ("q", "kn", "vn"):
-                self.items_in.append((L[key], pinned_like(L[key], "dec_" + key, L[key])))
-            self.items_out.append((L["out"], pinned_like(L["out"], "dec_out")))
-        self.h2d = sum(h.numel() * h.element_size() for _, h in self.items_in)
-        self.d2h = sum(h.numel() * h.element_size() for _, h in self.items_out)
+            ins = [(L[key], pinned_like(L[key], key, L[key])) for key in ("q", "k", "v")]
+            outs = [(L["out"], pinned_like(L["out"], "out"))]
+            self.units.append((L, ins, outs))
+        if w.decode_layers:
+            ins, outs = [], []
+            for L in w.decode_layers:
+                ins += [(L[key], pinned_like(L[key], "dec_" + key, L[key])) for key in ("q", "kn", "vn")]
+                outs.append((L["out"], pinned_like(L["out"], "dec_out")))
+            self.units.append((None, ins, outs))
+        self.h2d = sum(h.numel() * h.element_size() for _, ins, _ in self.units for _, h in ins)
+        self.d2h = sum(h.numel() * h.element_size() for _, _, outs in self.units for _, h in outs)
         self.pinned_bytes = sum(h.numel() * h.element_size() for h in shared.values())
+        self.s_in = torch.cuda.Stream()
+        self.s_out = torch.cuda.Stream()
+        n = len(self.units)
+        self.landed = [torch.cuda.Event() for _ in range(n)]
+        self.computed = [torch.cuda.Event() for _ in range(n)]
+        self.read_back = [torch.cuda.Event() for _ in range(n)]
+        self.primed = False
 
     def step(self, stream):
-        with torch.cuda.stream(stream):
-            for d, h in self.items_in:
-                d.copy_(h, non_blocking=True)
-            self.w.step(stream)
-            for d, h in self.items_out:
-                h.copy_(d, non_blocking=True)
+        """One step; its copies start after the work already queued on
+        `stream`, and `stream` ends after the step's last read-back."""
+        start = torch.cuda.Event()
+        start.record(stream)
+        self.s_in.wait_event(start)
+        for u, (L, ins, outs) in enumerate(self.units):
+            with torch.cuda.stream(self.s_in):
+                if self.primed:
+                    self.s_in.wait_event(self.computed[u])
+                for d, h in ins:
+                    d.copy_(h, non_blocking=True)
+                self.landed[u].record(self.s_in)
+            with torch.cuda.stream(stream):  # (the decode graph replays on the current stream)
+                stream.wait_event(self.landed[u])
+                if self.primed:
+                    stream.wait_event(self.read_back[u])
+                if L is not None:
+                    self.w.run_prefill_layer(L, stream)
+                else:
+                    self.w.run_decode_stack(stream)
+                self.computed[u].record(stream)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(self.computed[u])
+                for d, h in outs:
+                    h.copy_(d, non_blocking=True)
+                self.read_back[u].record(self.s_out)
+        stream.wait_event(self.read_back[-1])
+        self.primed = True
 
 
 # ------------------------------------------------------------------ oracle
@@ -1103,7 +1143,8 @@ def main():
         ms_e2e = max_over_ranks(dist, e0.elapsed_time(e1) / e2e_steps)
         e2e = {"value": job_value(world, step_flops, ms_e2e), "unit": "TFLOP/s",
                "h2d_bytes_per_step": host.h2d, "d2h_bytes_per_step": host.d2h, "ms_per_step": ms_e2e,
-               "steps": e2e_steps}
+               "steps": e2e_steps,
+               "overlap": "per layer: host->device copy, compute and device->host copy on three streams"}
         del host
 
     if mimo.mimo_attn_get_device_error() != 0:
