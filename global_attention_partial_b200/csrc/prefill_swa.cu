@@ -43,10 +43,21 @@
 //
 // TMEM (512 columns), per worker t: S_t = [256t, 256t + 144),
 // O_t = [256t + 72, 256t + 200) and Q_t = [256t + 200, 256t + 232) (dims
-// 0 .. 63 as bf16 pairs). O overlaps the upper S columns, which are dead once
-// the softmax has read them; P (bf16) takes the first 72 columns.
-// Shared memory: Q 2 x 48 KB; K ring 12 x 16 keys x 384 B; V ring 12 x 16
-// keys x 256 B (128B-swizzled 64-column blocks, 1024-byte aligned).
+// 0 .. 63 as bf16 pairs), X_t = [256t + 232, 256t + 234) (the halves' row
+// sums). O overlaps the upper S columns, which are dead once the
+// softmax has read them; P (bf16) takes the first 72 columns.
+// Shared memory: Q 2 x 48 KB; K ring 11 x 16 keys x 384 B; V ring 11 x 16
+// keys x 256 B (128B-swizzled 64-column blocks, 1024-byte aligned); 16 KB of
+// O staging.
+//
+// Epilogue: each warp writes its 32 rows x 64 output columns (scaled, bf16)
+// into a 4 KB staging slot and one lane issues a TMA store of them, so the
+// warp goes on at once; the slot is released a tile later, once the store
+// has read it. Half 0 stages in the first 64-column block of its worker's Q
+// buffer (dead once copied into TMEM, refilled only after the release); half
+// 1 in a 16 KB region the two workers take in turn. The two halves of a row
+// exchange their row maxima through shared memory and their row sums through
+// two TMEM columns.
 #include "kernels.cuh"
 
 #include <math.h>
@@ -58,7 +69,7 @@ constexpr int kBlockM = 128;
 constexpr int kKeyBlock = 16;
 constexpr int kMaxSpanBlocks = 9;  // 144 keys
 constexpr int kHalfCols = kMaxSpanBlocks * kKeyBlock / 2;  // 72 S columns per thread
-constexpr int kRing = 12;          // ring entries of 16 keys
+constexpr int kRing = 11;          // ring entries of 16 keys
 constexpr int kDqk = 192;
 constexpr int kDv = 128;
 constexpr int kThreads = 640;
@@ -83,13 +94,18 @@ constexpr int kWarpQ = 16, kWarpMma0 = 17, kWarpKV = 19;
 __device__ __forceinline__ uint32_t col_s(int t) { return t ? 256u : 0u; }
 __device__ __forceinline__ uint32_t col_o(int t) { return col_s(t) + 72u; }
 __device__ __forceinline__ uint32_t col_q(int t) { return col_s(t) + 200u; }
+// Two columns per worker through which the two halves of a row exchange
+// their row sums (read together with O).
+__device__ __forceinline__ uint32_t col_x(int t) { return col_s(t) + 232u; }
 
 struct SwaParams {
     CUtensorMap tm_q;  // [B, S, Hq, Dqk]    box {64, gp, P, 1}
     CUtensorMap tm_k;  // [B, S, Hkv, Dqk]   box {64, 1, 16, 1}
     CUtensorMap tm_v;  // [B, S, Hkv, Dv]    box {64, 1, 16, 1}
+    CUtensorMap tm_o;  // [B, S, Hq, Dv]     box {64, gp, 32 / gp, 1}: one warp's 32 rows, one half
     __nv_bfloat16 *out;
-    int out_v8;                // out is 32-byte aligned: 256-bit stores
+    int o_tma;                 // O through the staging slots and TMA stores, else direct stores
+    int out_v8;                // (direct stores) out is 32-byte aligned: 256-bit stores
     const float2 *rope_table;  // row (past + i): (cos, sin) of the pairs at query i's position
     const float *sinks;
     const int *past_lens;      // [B] cached tokens before the chunk, or nullptr
@@ -109,6 +125,7 @@ struct Bars {
     uint64_t kv_full[kRing], kv_empty[kRing];
     uint64_t kv_ready[kRing];  // the block's keys are rotated in place (or need no rotation)
     uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
+    uint64_t ost_free[4];  // half 1's staging slot of warp quarter q: the previous tile's store has read it
     uint64_t xchg[2];      // both halves of worker t published their row maxima
     uint64_t qrot[2];      // (generic RoPE only) both halves rotated Q in shared memory
     uint64_t drain[2];
@@ -116,9 +133,15 @@ struct Bars {
     int abort;
 };
 
-// Per worker: a row maximum and a row sum per half and query row.
+// O staging: a warp's 32 rows x 64 columns (4 KB, 128-byte swizzled rows).
+// Half 0 of worker t stages in the first 64-column block of its own Q
+// buffer (dead once copied into TMEM); half 1 of both workers shares one
+// region, a slot per warp quarter, handed from one tile to the next.
+constexpr int kOSlotBytes = 32 * 128;
+constexpr int kOStageBytes = 4 * kOSlotBytes;
+// Per worker: each half's row maximum per query row.
 constexpr int kRedBytes = 2 * 2 * kBlockM * 4;
-constexpr int kSmemBytes = 1024 + 2 * kQBytes + kKBytes + kVBytes + 2 * kRedBytes + (int)sizeof(Bars) + 64;
+constexpr int kSmemBytes = 1024 + 2 * kQBytes + kKBytes + kVBytes + kOStageBytes + kRedBytes + (int)sizeof(Bars) + 64;
 static_assert(kSmemBytes <= 232448, "shared memory");
 
 struct Tile {
@@ -197,8 +220,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
     uint8_t *sQ = smem;                  // 2 buffers
     uint8_t *sK = sQ + 2 * kQBytes;      // 3 atoms of the ring
     uint8_t *sV = sK + kKBytes;          // 2 atoms of the ring
-    float *sRed = reinterpret_cast<float *>(sV + kVBytes);  // [worker][max | sum][half][row]
-    Bars *bars = reinterpret_cast<Bars *>(sV + kVBytes + 2 * kRedBytes);
+    uint8_t *sOst = sV + kVBytes;        // half 1's O staging (1024-byte aligned)
+    float *sRedMax = reinterpret_cast<float *>(sOst + kOStageBytes);  // [worker][half][row]
+    Bars *bars = reinterpret_cast<Bars *>(sOst + kOStageBytes + kRedBytes);
     volatile int *abort_flag = &bars->abort;
 
     const int warp = threadIdx.x >> 5;
@@ -211,7 +235,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->q_full[i], 1);
             mbar_init(&bars->q_ready[i], kWorkerThreads);
-            mbar_init(&bars->q_empty[i], 1);  // QK^T of the tile has read the buffer
+            // QK^T of the tile has read the buffer, and the four half-0 warps
+            // have released their O staging in its first block
+            mbar_init(&bars->q_empty[i], 1 + 4);
             mbar_init(&bars->s_full[i], 1);
             mbar_init(&bars->p_full[i], kWorkerThreads);
             mbar_init(&bars->o_full[i], 1);
@@ -224,6 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
             mbar_init(&bars->kv_empty[i], 2);  // one commit from each issuer
             mbar_init(&bars->kv_ready[i], 1);
         }
+        for (int i = 0; i < 4; ++i)
+            mbar_init(&bars->ost_free[i], 1);
         mbar_init(&bars->drain[0], 1);
         mbar_init(&bars->drain[1], 1);
         bars->abort = 0;
@@ -397,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
         // entries below the span of a tile before waiting for it and below the
         // span of its next tile after the PV of its current one, and every
         // remaining entry after its last tile. As a tile spans at most 9 of
-        // the 12 entries, every entry the producer waits on is then committed
+        // the 11 entries, every entry the producer waits on is then committed
         // by an issuer that is not waiting on that producer.
         const int t = warp - kWarpMma0;
         if (lane == 0 && t < n_local) {
@@ -516,8 +544,26 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
         const uint32_t p_addr = lane_base + col_s(t) + (uint32_t)(kHalfCols / 2 * hf);
         const uint32_t o_addr = lane_base + col_o(t) + (uint32_t)(64 * hf);
         const uint32_t q_addr = lane_base + col_q(t);
-        float *red_max = sRed + t * (4 * kBlockM);  // [half][row]
-        float *red_sum = red_max + 2 * kBlockM;
+        const uint32_t x_addr = lane_base + col_x(t);  // row sum exchange with the other half
+        float *red_max = sRedMax + t * (2 * kBlockM);   // [half][row]
+        const int wq = warp & 3;                        // this warp's 32 rows of the tile
+        uint8_t *const o_stage = hf == 0 ? sQ + t * kQBytes + wq * kOSlotBytes : sOst + wq * kOSlotBytes;
+        bool o_used = false;     // (lane 0) this warp wrote o_stage in its last epilogue
+        bool o_pending = false;  // (lane 0) ... and a store from it may still be reading it
+        // Lane 0 lets the staging slot go once its store has read it: half 0's
+        // slot back to the Q buffer's next fill (one of the five arrivals of
+        // q_empty, made every tile), half 1's to the other worker's next tile
+        // (one arrival per use, a store issued or not).
+        auto release_stage = [&](bool every_tile) {
+            if (lane == 0) {
+                if (o_pending)
+                    bulk_wait_read_all();
+                if (hf == 0 ? every_tile : o_used)
+                    mbar_arrive(hf == 0 ? &bars->q_empty[t] : &bars->ost_free[wq]);
+                o_pending = false;
+                o_used = false;
+            }
+        };
         const int half = p.rope_half;
         const float sc = p.scale_log2;
         const bool fast_rope = half == 32 && p.P == 16;
@@ -607,6 +653,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 ok = false;
                 break;
             }
+            // The O staging of this worker's previous tile (its store was
+            // issued a tile ago), released before this tile's epilogue reuses
+            // it; half 0 arrives every tile (QK^T of this tile has read the
+            // Q buffer's other blocks by now).
+            release_stage(true);
             tc_fence_after();
             float x[kHalfCols];
             {
@@ -682,7 +733,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 tmem_st4(p_addr + 4 * q, pk);
             }
             const float rs_half = (rsv[0].x + rsv[0].y) + (rsv[1].x + rsv[1].y);
-            red_sum[hf * kBlockM + row] = rs_half;
+            {
+                const uint32_t v[1] = {__float_as_uint(rs_half)};
+                tmem_st1(x_addr + hf, v);
+            }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars->p_full[t]);
@@ -703,7 +757,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
                 ok = false;
                 break;
             }
-            const float rs = rs_half + red_sum[(hf ^ 1) * kBlockM + row];
+            tc_fence_after();
+            uint32_t o[2][32], rsp[1];
+            tmem_ld1(x_addr + (hf ^ 1), rsp);
+            tmem_ld32(o_addr, o[0]);
+            tmem_ld32(o_addr + 32, o[1]);
+            tmem_wait_ld_only();
+            tmem_tie(rsp);
+            tmem_tie(o[0]);
+            tmem_tie(o[1]);
+            tc_fence_before();
+            mbar_arrive(&bars->o_free[t]);
+            const float rs = rs_half + __uint_as_float(rsp[0]);
             // (rs >= 1: the row maximum's own term; approximate exp2 and
             // division, well inside bf16 output rounding)
             float o_scale;
@@ -715,36 +780,81 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_swa_kernel(const __grid_c
             } else {
                 o_scale = __fdividef(p.v_scale, rs);
             }
-            tc_fence_after();
-            uint32_t o[2][32];
-            tmem_ld32(o_addr, o[0]);
-            tmem_ld32(o_addr + 32, o[1]);
-            tmem_wait_ld_only();
-            tmem_tie(o[0]);
-            tmem_tie(o[1]);
-            tc_fence_before();
-            mbar_arrive(&bars->o_free[t]);
-            if (i < p.S) {
-                uint8_t *dst =
-                    reinterpret_cast<uint8_t *>(p.out + (((size_t)c.b * p.S + i) * p.Hq + h) * kDv + 64 * hf);
-                const f32x2 os2 = {o_scale, o_scale};
+            if (!p.o_tma) {
+                // direct stores: this row's 64 columns as four 32-byte pieces
+                if (i < p.S) {
+                    uint8_t *dst =
+                        reinterpret_cast<uint8_t *>(p.out + (((size_t)c.b * p.S + i) * p.Hq + h) * kDv + 64 * hf);
+                    const f32x2 os2 = {o_scale, o_scale};
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
+                    for (int q = 0; q < 4; ++q) {
                         uint32_t w[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
-                            const f32x2 v = mul2(f32x2{__uint_as_float(o[q][hh * 16 + 2 * e]),
-                                                       __uint_as_float(o[q][hh * 16 + 2 * e + 1])},
+                            const int col = 16 * q + 2 * e;
+                            const f32x2 v = mul2(f32x2{__uint_as_float(o[col >> 5][col & 31]),
+                                                       __uint_as_float(o[col >> 5][(col & 31) + 1])},
                                                  os2);
                             w[e] = pack_bf16x2(v.x, v.y);
                         }
-                        st_global_32B(dst + (q * 2 + hh) * 32, w, p.out_v8 != 0);
+                        st_global_32B(dst + q * 32, w, p.out_v8 != 0);
                     }
+                }
+                continue;
+            }
+            // The slot must be free: half 0's block of the Q buffer holds the
+            // next tile's rotary dims until both halves have copied them
+            // (q_ready); half 1's slot until the other worker's previous
+            // store has read it. (The parity wait is exact: this worker
+            // released its own use of two tiles ago before this point.)
+            {
+                const bool waited = hf == 0 ? (n + 2 >= n_local ||
+                                               mbar_wait(&bars->q_ready[t], (uint32_t)((n + 2) >> 1) & 1u, abort_flag,
+                                                         p.err))
+                                            : mbar_wait(&bars->ost_free[wq], ((uint32_t)n & 1u) ^ 1u, abort_flag, p.err);
+                if (!waited) {
+                    ok = false;
+                    break;
+                }
+            }
+            // Row = lane, 128 bytes; 16-byte chunk j at j ^ (lane & 7), the
+            // 128-byte swizzle of the store's tensor map.
+            {
+                const f32x2 os2 = {o_scale, o_scale};
+                uint8_t *srow = o_stage + lane * 128;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int col = 8 * j + 2 * e;
+                        const f32x2 v = mul2(f32x2{__uint_as_float(o[col >> 5][col & 31]),
+                                                   __uint_as_float(o[col >> 5][(col & 31) + 1])},
+                                             os2);
+                        w[e] = pack_bf16x2(v.x, v.y);
+                    }
+                    *reinterpret_cast<uint4 *>(srow + ((j ^ (lane & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            // (a warp whose rows all lie past the sequence end stores nothing;
+            // a partly past box is clipped by the tensor map)
+            const int w_pos = c.p0 + wq * (32 / p.gp);
+            if (lane == 0) {
+                o_used = true;
+                if (w_pos < p.S) {
+                    tma_store_4d(&p.tm_o, o_stage, 64 * hf, c.h0, w_pos, c.b);
+                    bulk_commit_group();
+                    o_pending = true;
                 }
             }
         }
+        // the last tile's staging: released for the other worker, and every
+        // store complete before the CTA ends
+        release_stage(false);
+        if (lane == 0)
+            bulk_wait_all();
     }
 
     tc_fence_before();
@@ -797,7 +907,8 @@ cudaError_t launch_prefill_swa(const LayerArgs &L, const PrefillArgs &a, const f
     const int P = kBlockM / gp;
     if (!make_bf16_map_4d(&p.tm_q, a.q, kDqk, L.Hq, a.S, a.S, a.B, 64, gp, P) ||
         !make_bf16_map_4d(&p.tm_k, a.krot, kDqk, L.Hkv, a.key_rows_valid, a.krot_rows, a.B, 64, 1, kKeyBlock) ||
-        !make_bf16_map_4d(&p.tm_v, a.v, kDv, L.Hkv, a.key_rows_valid, a.v_rows, a.B, 64, 1, kKeyBlock))
+        !make_bf16_map_4d(&p.tm_v, a.v, kDv, L.Hkv, a.key_rows_valid, a.v_rows, a.B, 64, 1, kKeyBlock) ||
+        !make_bf16_map_4d(&p.tm_o, a.out, kDv, L.Hq, a.S, a.S, a.B, 64, gp, 32 / gp))
         return cudaErrorInvalidValue;
     p.out = reinterpret_cast<__nv_bfloat16 *>(a.out);
     p.out_v8 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
@@ -818,6 +929,11 @@ cudaError_t launch_prefill_swa(const LayerArgs &L, const PrefillArgs &a, const f
     p.num_g_tiles = L.G / gp;
     p.num_tiles = p.num_p_tiles * p.num_g_tiles * L.Hkv * a.B;
     p.tiles_per_cta = (p.num_tiles + num_sms - 1) / num_sms;
+    // The staged TMA-store epilogue pays off once a CTA runs many tiles
+    // (B4 S32768: ~440 per CTA, 1.85 -> 1.77 ms per layer); with two or three
+    // per CTA the final drain of its stores costs more (B1 S4096: 0.085 ->
+    // 0.091 ms), so short runs store directly.
+    p.o_tma = p.tiles_per_cta >= 8 ? 1 : 0;
     p.rope_half = L.rope.half;
     p.rotate_k = a.k_unrotated ? 1 : 0;
     p.scale_log2 = L.scale_log2;
