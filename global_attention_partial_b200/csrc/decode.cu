@@ -49,9 +49,10 @@ constexpr int kStageElems = kTileKeys * (kKStride + kVStride);
 constexpr int kLandRow = kDqk + kDv;             // bytes per key
 constexpr int kWarpLand = 16 * kLandRow;         // one warp's 16 keys: 5120
 constexpr int kLandBytes = kTileKeys * kLandRow;  // one stage of the CTA: 20480
-// SLIM (fp8 only): the query fragments stay in shared memory and are read per
-// k-step instead of held in 48 registers, so 4 CTAs fit per SM (128 registers,
-// 2 stages): the 512 CTAs of a 128-slot sliding layer at B64 run in one wave.
+// SLIM: the query fragments stay in shared memory and are read per k-step
+// instead of held in 48 registers, so 4 CTAs fit per SM (128 registers; fp8:
+// 2 stages of 20 KB, bf16: 1 stage of 43 KB): the 512 CTAs of a 128-slot
+// sliding layer at B64 run in one wave.
 template <int ST, bool F8 = false, bool SLIM = false> struct DecodeCfg {
     static constexpr int kSmemBytes = F8 ? (16 * kQStride + kDqk + kDv) * 2 + kLandRow + ST * kLandBytes
                                          : (16 * kQStride + ST * kStageElems + kDqk + kDv) * 2;
@@ -79,8 +80,10 @@ constexpr int kDecodeStages = 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kDecodeStagesFp8 = 3;  // 5 KB per warp and stage; 69 KB per CTA: 3 CTAs (12 warps) per SM
 static_assert(DecodeCfg<kDecodeStagesFp8, true>::kSmemBytes <= 72 * 1024, "3 CTAs per SM");
-constexpr int kDecodeStagesSlim = 2;  // 48 KB per CTA: 4 CTAs per SM
+constexpr int kDecodeStagesSlim = 2;  // fp8: 48 KB per CTA: 4 CTAs per SM
 static_assert(DecodeCfg<kDecodeStagesSlim, true, true>::kSmemBytes <= 55 * 1024, "4 CTAs per SM");
+constexpr int kDecodeStagesSlimBf16 = 1;  // bf16: 49 KB per CTA: 4 CTAs per SM
+static_assert(DecodeCfg<kDecodeStagesSlimBf16, false, true>::kSmemBytes <= 55 * 1024, "4 CTAs per SM");
 
 struct DecodeSmem {
     float wm[4][16];
@@ -106,7 +109,6 @@ template <int kStages, bool kFp8 = false, bool kSlim = false>
 __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8, kSlim>::kCtasPerSm)
     decode_mma_kernel(const __grid_constant__ LayerArgs L, const __grid_constant__ DecodeArgs a)
 {
-    static_assert(!kSlim || kFp8, "the slim form is the fp8 one");
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // Query rows: bf16, or f16 with fp8 caches. bf16: then the K/V stage
     // ring and the raw new k/v. fp8: the raw new k/v, the new token's codes
@@ -400,6 +402,9 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8, kSlim>::kCt
     // fp8: the two words of k-step ks in rows g and g + 8 (64-bit reads)
     const uint2 *q0w = reinterpret_cast<const uint2 *>(sQ + g * kQStride + tq * 48);
     const uint2 *q1w = reinterpret_cast<const uint2 *>(sQ + (g + 8) * kQStride + tq * 48);
+    // bf16: ldmatrix base of the query fragments (rows and 8-column halves by lane)
+    const uint32_t q_ldm = smem_u32(sQ) + (uint32_t)((((lane & 7) + ((lane >> 3) & 1) * 8) * kQStride +
+                                                     (lane >> 4) * 8) * 2u);
     if constexpr (kSlim) {
     } else if constexpr (kFp8) {
         const uint32_t *q0 = reinterpret_cast<const uint32_t *>(q0w);
@@ -412,12 +417,9 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8, kSlim>::kCt
             qa[ks][3] = q1[2 * ks + 1];
         }
     } else {
-        const int mi = lane >> 3;
-        const int r = (lane & 7) + (mi & 1) * 8;
-        const uint32_t base = smem_u32(sQ) + (uint32_t)(r * kQStride + (mi >> 1) * 8) * 2u;
 #pragma unroll
         for (int ks = 0; ks < 12; ++ks)
-            ldmatrix_x4(base + ks * 32, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
+            ldmatrix_x4(q_ldm + ks * 32, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
     }
     float m0 = -INFINITY, m1 = -INFINITY;  // running max of rows g, g+8 (base 2)
     float l0 = 0.f, l1 = 0.f;              // this thread's partial sums
@@ -522,8 +524,17 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<kStages, kFp8, kSlim>::kCt
             for (int ks = 0; ks < 12; ++ks) {
                 uint32_t b0, b1, b2, b3;
                 ldmatrix_x4(base + ks * 32, b0, b1, b2, b3);
-                mma_bf16_16816((ks & 1) ? s_odd[0] : s_acc[0], qa[ks], b0, b1);
-                mma_bf16_16816((ks & 1) ? s_odd[1] : s_acc[1], qa[ks], b2, b3);
+                uint32_t qf[4];
+                if constexpr (kSlim) {
+                    ldmatrix_x4(q_ldm + ks * 32, qf[0], qf[1], qf[2], qf[3]);
+                } else {
+                    qf[0] = qa[ks][0];
+                    qf[1] = qa[ks][1];
+                    qf[2] = qa[ks][2];
+                    qf[3] = qa[ks][3];
+                }
+                mma_bf16_16816((ks & 1) && !kSlim ? s_odd[0] : s_acc[0], qf, b0, b1);
+                mma_bf16_16816((ks & 1) && !kSlim ? s_odd[1] : s_acc[1], qf, b2, b3);
             }
         }
 #pragma unroll
@@ -1010,13 +1021,16 @@ cudaError_t launch_decode(const LayerArgs &L, const DecodeArgs &a, int dtype, cu
     if (a.fp8_cache && !decode_mma_supported(L, dtype))
         return cudaErrorInvalidValue;
     if (decode_mma_supported(L, dtype)) {
-        static std::atomic<unsigned long long> prepared[3] = {{0}, {0}, {0}};
-        // fp8 sliding layers whose ring is at most two tiles take the slim form
-        const int f = a.fp8_cache ? (L.layer_type == 1 && L.window <= 2 * kTileKeys ? 2 : 1) : 0;
+        static std::atomic<unsigned long long> prepared[4] = {{0}, {0}, {0}, {0}};
+        // sliding layers whose ring is at most two tiles take the slim forms
+        const bool slim = L.layer_type == 1 && L.window <= 2 * kTileKeys;
+        const int f = a.fp8_cache ? (slim ? 2 : 1) : (slim ? 3 : 0);
         {
             cudaError_t e =
-                f == 2 ? prepare_kernel_once(decode_mma_kernel<kDecodeStagesSlim, true, true>,
-                                             DecodeCfg<kDecodeStagesSlim, true, true>::kSmemBytes, prepared[2])
+                f == 3 ? prepare_kernel_once(decode_mma_kernel<kDecodeStagesSlimBf16, false, true>,
+                                             DecodeCfg<kDecodeStagesSlimBf16, false, true>::kSmemBytes, prepared[3])
+                : f == 2 ? prepare_kernel_once(decode_mma_kernel<kDecodeStagesSlim, true, true>,
+                                               DecodeCfg<kDecodeStagesSlim, true, true>::kSmemBytes, prepared[2])
                 : f == 1 ? prepare_kernel_once(decode_mma_kernel<kDecodeStagesFp8, true>,
                                                DecodeCfg<kDecodeStagesFp8, true>::kSmemBytes, prepared[1])
                          : prepare_kernel_once(decode_mma_kernel<kDecodeStages, false>,
@@ -1025,7 +1039,10 @@ cudaError_t launch_decode(const LayerArgs &L, const DecodeArgs &a, int dtype, cu
                 return e;
         }
         dim3 grid(a.max_splits, L.Hkv, a.B);
-        if (f == 2)
+        if (f == 3)
+            decode_mma_kernel<kDecodeStagesSlimBf16, false, true>
+                <<<grid, kThreads, DecodeCfg<kDecodeStagesSlimBf16, false, true>::kSmemBytes, stream>>>(L, a);
+        else if (f == 2)
             decode_mma_kernel<kDecodeStagesSlim, true, true>
                 <<<grid, kThreads, DecodeCfg<kDecodeStagesSlim, true, true>::kSmemBytes, stream>>>(L, a);
         else if (f == 1)
