@@ -245,6 +245,17 @@ def test_decode_small_every_output(layer_type):
     _check_decode(spec, out, inputs, caches, range(len(lens)), lens)
 
 
+@pytest.mark.parametrize("window", [16, 64, 100, 128, 192, 256])
+def test_decode_sliding_windows(window):
+    """Sliding layers with rings of one to four 64-key tiles: up to two tiles
+    take the slim kernel form (one stage, 4 CTAs per SM), longer rings the
+    2-stage one. Lengths below, at and past the window; every output."""
+    spec = synthetic.mimo_layer(1, window=window)
+    lens = sorted({1, 2, window - 1, window, window + 1, 2 * window + 3, 700} - {0})
+    out, inputs, caches = _run_decode(spec, len(lens), window, lens, seed=window)
+    _check_decode(spec, out, inputs, caches, range(len(lens)), lens)
+
+
 @pytest.mark.parametrize("layer_type", [0, 1])
 def test_decode_stale_slots_hold_nan(layer_type):
     """Cache slots past a sequence's length may hold any bits: with NaN in
