@@ -110,6 +110,19 @@ def test_swa_prefill_ring_runs_every_output(B, S):
     _assert(c, BF, f"SWA B{B} S{S}")
 
 
+@pytest.mark.parametrize("hq,hkv,window,S", [(32, 8, 64, 4790), (16, 8, 32, 9590), (8, 8, 16, 19000)])
+def test_swa_prefill_staged_stores_other_head_groups(hq, hkv, window, S):
+    """The sliding kernel's staged TMA-store epilogue (16 or more tiles per
+    CTA) with 4, 2 and 1 query heads per KV group: a tile is then 32, 64 or 128
+    positions of those heads, and each warp stores its 32 rows as a box of
+    32 / heads positions. Ragged sequence ends; every row of a subset of
+    heads, both batches."""
+    spec = synthetic.mimo_layer(1, hq=hq, swa_kv=hkv, window=window)
+    c, _, _ = check_prefill(spec, 2, S, BF, seed=hq + S, heads=range(0, hq, max(1, hq // 8)))
+    _assert(c, BF, f"SWA Hq{hq} Hkv{hkv} W{window} B2 S{S}")
+    assert mimo.mimo_attn_get_device_error() == 0
+
+
 def test_swa_prefill_full_size_every_output():
     """Single SWA layer, B1 S4096 Hq64 Hkv8 qk192 v128 r64 W128: every output."""
     spec = synthetic.SWA_PREFILL.layers[0]
