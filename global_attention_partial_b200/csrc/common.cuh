@@ -278,15 +278,6 @@ __device__ __forceinline__ void tma_load_4d(void *smem_dst, const CUtensorMap *m
         : "memory");
 }
 
-// Prefetch of one 4-D box into L2 (no shared memory, no completion).
-__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-                 : "memory");
-}
-
 // 4-D tiled store of one box from shared memory (written by this CTA's
 // threads, fenced to the async proxy first) into global memory; completion
 // is tracked by the issuing thread's bulk groups. Out-of-range rows are not
