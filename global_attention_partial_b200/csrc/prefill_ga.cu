@@ -381,23 +381,33 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_ga_kernel(const __grid_co
             for (int c = 0; c < kBlockN; ++c)
                 mxv[c & 3] = fmaxf(mxv[c & 3], x[c]);
             const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])) * p.scale_log2;
-            if (mx > m_ref + kRescaleThreshold || (m_ref == -INFINITY && mx > -INFINITY)) {
-                // New reference max; O already holds P*V of tiles < j (in-order MMAs).
-                const float corr = (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - mx);
-                if (j > 0 && m_ref != -INFINITY) {
+            // A row moves its reference max when the tile's max exceeds it by
+            // more than the threshold; corr rescales what was summed against
+            // the old one. O already holds P*V of tiles < j (in-order MMAs).
+            // The TMEM load and store are warp-collective (.sync.aligned), so
+            // the whole warp rescales whenever one of its rows moved (the
+            // others by 1), 16 columns at a time.
+            const bool move = mx > m_ref + kRescaleThreshold || (m_ref == -INFINITY && mx > -INFINITY);
+            if (__any_sync(0xffffffffu, move)) {
+                const float corr = !move ? 1.f : (m_ref == -INFINITY ? 0.f : fast_exp2(m_ref - mx));
+                if (j > 0 && __any_sync(0xffffffffu, move && m_ref != -INFINITY)) {
+                    const float f = (m_ref == -INFINITY) ? 1.f : corr;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < kDv; c0 += 16) {
+                        uint32_t r[16];
+                        tmem_ld16(o_addr + c0, r);
+                        tmem_wait_ld_only();
+                        tmem_tie(r);
 #pragma unroll
-                    for (int c0 = 0; c0 < kDv; c0 += 32) {
-                        uint32_t r[32];
-                        tmem_ld32(o_addr + c0, r);
-                        tmem_wait_ld(r);
-#pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            r[c] = __float_as_uint(__uint_as_float(r[c]) * corr);
-                        tmem_st32(o_addr + c0, r);
+                        for (int c = 0; c < 16; ++c)
+                            r[c] = __float_as_uint(__uint_as_float(r[c]) * f);
+                        tmem_st16(o_addr + c0, r);
                     }
                 }
-                l_sum *= corr;
-                m_ref = mx;
+                if (move) {
+                    l_sum *= corr;
+                    m_ref = mx;
+                }
             }
             const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
             const float sc = p.scale_log2;

@@ -329,27 +329,32 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             for (int c = 0; c < kBlockN; ++c)
                 mxv[c & 3] = fmaxf(mxv[c & 3], x[c]);
             const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3]));
-            if (mx > m_ref + kRescaleThreshold || (m_ref == -INFINITY && mx > -INFINITY)) {
-                // New reference max: rescale the running sum, and O once an
-                // earlier P*V has landed in it.
-                const float corr = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mx);
-                if (j > 0 && m_ref != -INFINITY) {
-                    if (!mbar_wait(&bars->o_done, (uint32_t)(j - 1) & 1u, abort_flag, p.err)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-#pragma unroll
-                    for (int c0 = 0; c0 < kDv; c0 += 32) {
-                        uint32_t r[32];
-                        tmem_ld32(lane_base + kColO + c0, r);
-                        tmem_wait_ld(r);
-#pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            r[c] = __float_as_uint(__uint_as_float(r[c]) * corr);
-                        tmem_st32(lane_base + kColO + c0, r);
-                    }
+            // A row moves its reference max when the tile's max exceeds it by
+            // more than the threshold; corr rescales the running sum, and O
+            // once an earlier P*V has landed in it.
+            const bool move = mx > m_ref + kRescaleThreshold || (m_ref == -INFINITY && mx > -INFINITY);
+            const float corr = !move ? 1.f : (m_ref == -INFINITY ? 0.f : exp2f(m_ref - mx));
+            // The TMEM load and store are warp-collective (.sync.aligned): the
+            // whole warp rescales whenever one of its rows moved (the others by 1).
+            if (j > 0 && __any_sync(0xffffffffu, move && m_ref != -INFINITY)) {
+                if (!mbar_wait(&bars->o_done, (uint32_t)(j - 1) & 1u, abort_flag, p.err)) {
+                    ok = false;
+                    break;
                 }
+                tc_fence_after();
+                const float f = (m_ref == -INFINITY) ? 1.f : corr;
+#pragma unroll
+                for (int c0 = 0; c0 < kDv; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(lane_base + kColO + c0, r);
+                    tmem_wait_ld(r);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        r[c] = __float_as_uint(__uint_as_float(r[c]) * f);
+                    tmem_st32(lane_base + kColO + c0, r);
+                }
+            }
+            if (move) {
                 l_sum *= corr;
                 m_ref = mx;
             }
