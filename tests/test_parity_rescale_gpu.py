@@ -114,7 +114,8 @@ def test_prefill_with_spike_keys(layer_type):
 def test_decode_with_spike_keys(layer_type):
     """Decode over caches holding the spikes: the per-tile lazy rescale and,
     on global layers, a combine of splits whose maxima differ by ~10 nats
-    (the block straddles the 2048-key split boundary)."""
+    (the block straddles the 2048-key split boundary). In sequence 1 the new
+    token is the spike."""
     spec = synthetic.mimo_layer(layer_type)
     lens = [2000, 2100, 2300, 2301, 3400, 3501, 3700, 4100] if layer_type == 0 else [2000, 2301, 3502, 3600]
     B = len(lens)
@@ -137,6 +138,10 @@ def test_decode_with_spike_keys(layer_type):
                     kc[b, p % W] = 0.0
                     kc[b, p % W, :, DIM] = PEAK_VALUE if p == PEAK else BLOCK_VALUE
     kn[..., DIM] = 0.0
+    # one sequence whose new token is itself a spike (its key is rotated and
+    # written by the kernel before use)
+    kn[1] = 0.0
+    kn[1, :, DIM] = PEAK_VALUE
     kc0, vc0 = kc.clone(), vc.clone()
     out = mimo.decode(lib_layer(spec, sinks), q, kn, vn, kv_lens.cuda(), kc, vc)
     torch.cuda.synchronize()
@@ -151,6 +156,61 @@ def test_decode_with_spike_keys(layer_type):
                                     f64(vc0[b, :, kv]), L, spec.rotary_dim, spec.theta, spec.layer_type,
                                     spec.window, 1 / math.sqrt(spec.qk_dim),
                                     None if sinks is None else f64(sinks[hs]), vs)
+            gpu.append(f64(out[b, hs]))
+            want.append(o)
+    c = compare(np.concatenate(gpu), np.concatenate(want))
+    assert c.ok(BF), f"max_abs={c.max_abs:.3e} mean_abs={c.mean_abs:.3e} over {c.n}"
+
+
+SINKS = (-math.inf, -30.0, 0.0, 12.0, 30.0)
+
+
+def _extreme_sinks(spec):
+    return torch.tensor([SINKS[h % len(SINKS)] for h in range(spec.num_q_heads)], dtype=torch.float32,
+                        device="cuda")
+
+
+def test_swa_prefill_extreme_sinks():
+    """Sink logits of -inf (no sink), -30, 0, +12 and +30 nats: the sink may
+    take all but ~e^-25 of the mass, or none. Every output of a ragged
+    sequence, all heads."""
+    spec = synthetic.mimo_layer(1)
+    B, S = 1, 700
+    q, k, v, _ = synthetic.prefill_inputs(spec, B, S, seed=47, layer=1, dtype=BF, device="cuda")
+    sinks = _extreme_sinks(spec)
+    out = mimo.prefill(lib_layer(spec, sinks), q, k, v)
+    torch.cuda.synchronize()
+    assert mimo.mimo_attn_get_device_error() == 0
+    ref = oracle_prefill(spec, q, k, v, sinks, {(0, h): list(range(S)) for h in range(spec.num_q_heads)})
+    gpu, want = [], []
+    for (b, h), (rr, o) in ref.items():
+        gpu.append(f64(out[b, rr, h, :]))
+        want.append(o)
+    c = compare(np.concatenate(gpu), np.concatenate(want))
+    assert c.ok(BF), f"max_abs={c.max_abs:.3e} mean_abs={c.mean_abs:.3e} over {c.n}"
+
+
+def test_swa_decode_extreme_sinks():
+    spec = synthetic.mimo_layer(1)
+    lens = [1, 2, 64, 65, 128, 129, 700]
+    B, cap = len(lens), spec.window
+    kv_lens = torch.tensor(lens, dtype=torch.int32)
+    q, kn, vn, kc, vc, _ = synthetic.decode_inputs(spec, B, cap, kv_lens, seed=53, layer=1, dtype=BF,
+                                                   device="cuda")
+    sinks = _extreme_sinks(spec)
+    kc0, vc0 = kc.clone(), vc.clone()
+    out = mimo.decode(lib_layer(spec, sinks), q, kn, vn, kv_lens.cuda(), kc, vc)
+    torch.cuda.synchronize()
+    assert mimo.mimo_attn_get_device_error() == 0
+    G = spec.num_q_heads // spec.num_kv_heads
+    vs = oracle.v_scale(spec.hidden_size, spec.num_q_heads, spec.v_dim)
+    gpu, want = [], []
+    for b, L in enumerate(lens):
+        for kv in range(spec.num_kv_heads):
+            hs = slice(kv * G, (kv + 1) * G)
+            o, _, _ = oracle.decode(f64(q[b, hs]), f64(kn[b, kv]), f64(vn[b, kv]), f64(kc0[b, :, kv]),
+                                    f64(vc0[b, :, kv]), L, spec.rotary_dim, spec.theta, spec.layer_type,
+                                    spec.window, 1 / math.sqrt(spec.qk_dim), f64(sinks[hs]), vs)
             gpu.append(f64(out[b, hs]))
             want.append(o)
     c = compare(np.concatenate(gpu), np.concatenate(want))
