@@ -215,3 +215,101 @@ def test_swa_decode_extreme_sinks():
             want.append(o)
     c = compare(np.concatenate(gpu), np.concatenate(want))
     assert c.ok(BF), f"max_abs={c.max_abs:.3e} mean_abs={c.mean_abs:.3e} over {c.n}"
+
+
+def _compare_rows(spec, out, q, k, v, sinks, rows, heads):
+    ref = oracle_prefill(spec, q, k, v, sinks, {(0, h): rows for h in heads})
+    gpu, want = [], []
+    for (b, h), (rr, o) in ref.items():
+        gpu.append(f64(out[b, rr, h, :]))
+        want.append(o)
+    return compare(np.concatenate(gpu), np.concatenate(want))
+
+
+def test_single_tile_prefill_with_spike_keys():
+    """An odd query-group size (12 query heads over 4 KV heads) takes the
+    single-tile tensor-core kernel, whose online softmax has the same lazy
+    rescale."""
+    spec = synthetic.mimo_layer(0, hq=12, ga_kv=4)
+    B, S = 1, 4096 + 37
+    q, k, v, _ = synthetic.prefill_inputs(spec, B, S, seed=59, layer=0, dtype=BF, device="cuda")
+    _plant(q, k, key_axis=1)
+    out = mimo.prefill(lib_layer(spec, None), q, k, v)
+    torch.cuda.synchronize()
+    assert mimo.mimo_attn_get_device_error() == 0
+    rows = sorted({0, 128, 1899, 1900, 1901, 2047, 2048, 2299, 2300, 3499, 3500, 3501, 4000, S - 1})
+    c = _compare_rows(spec, out, q, k, v, None, rows, (0, 2, 3, 5, 11))
+    assert c.ok(BF), f"max_abs={c.max_abs:.3e} mean_abs={c.mean_abs:.3e} over {c.n}"
+
+
+def test_decode_fp8_with_spike_keys():
+    """The fp8 (E4M3) decode over the planted global-layer cache. The keys are
+    stored at k_scale 1/2 so the spikes stay representable (124 and 207 become
+    the codes 256 and 416, i.e. 128 and 208)."""
+    from tests.test_parity_fp8_gpu import _encode_on_device
+    spec = synthetic.mimo_layer(0)
+    k_scale, v_scale = 0.5, 1.0 / 32
+    lens = [2000, 2100, 2301, 3501, 3700, 4100]
+    B, cap = len(lens), 4100
+    kv_lens = torch.tensor(lens, dtype=torch.int32)
+    q, kn, vn, kc, vc, _ = synthetic.decode_inputs(spec, B, cap, kv_lens, seed=61, layer=0, dtype=BF, device="cuda")
+    _plant(q, kc, key_axis=1)
+    kn[..., DIM] = 0.0
+    kn[1] = 0.0
+    kn[1, :, DIM] = PEAK_VALUE
+    kc8 = torch.stack([_encode_on_device(kc[b], k_scale) for b in range(B)])
+    vc8 = torch.stack([_encode_on_device(vc[b], v_scale) for b in range(B)])
+    kc0, vc0 = kc8.clone(), vc8.clone()
+    out = mimo.decode_fp8kv(lib_layer(spec, None), q, kn, vn, kv_lens.cuda(), kc8, vc8, k_scale, v_scale)
+    torch.cuda.synchronize()
+    assert mimo.mimo_attn_get_device_error() == 0
+    G = spec.num_q_heads // spec.num_kv_heads
+    vs = oracle.v_scale(spec.hidden_size, spec.num_q_heads, spec.v_dim)
+    gpu, want = [], []
+    for b, L in enumerate(lens):
+        for kv in range(spec.num_kv_heads):
+            hs = slice(kv * G, (kv + 1) * G)
+            o, _, _ = oracle.decode_fp8kv(f64(q[b, hs]), f64(kn[b, kv]), f64(vn[b, kv]), kc0[b, :, kv].cpu().numpy(),
+                                          vc0[b, :, kv].cpu().numpy(), L, spec.rotary_dim, spec.theta, 0,
+                                          spec.window, 1 / math.sqrt(spec.qk_dim), None, vs, k_scale, v_scale)
+            gpu.append(f64(out[b, hs]))
+            want.append(o)
+    c = compare(np.concatenate(gpu), np.concatenate(want))
+    assert c.ok(BF), f"max_abs={c.max_abs:.3e} mean_abs={c.mean_abs:.3e} over {c.n}"
+
+
+def test_prefill_continuing_cache_with_spike_keys():
+    """A global-layer chunk after a cache that holds the spike block, with
+    the single spike inside the chunk: the kernel reads the cache with a key
+    offset per sequence."""
+    spec = synthetic.mimo_layer(0)
+    past, S = [2500, 1950], 1100
+    B = len(past)
+    cap = max(past) + S + 5
+    q, k, v, kc, vc, _ = synthetic.cached_prefill_inputs(spec, B, S, cap, seed=67, layer=0, dtype=BF, device="cuda")
+    q[..., DIM] = 1.0
+    k[..., DIM] = 0.0
+    kc[..., DIM] = 0.0
+    for b, P in enumerate(past):
+        for p0 in range(*BLOCK):           # block positions: in the cache or in the chunk
+            if p0 < P:
+                kc[b, p0] = 0.0
+                kc[b, p0, :, DIM] = BLOCK_VALUE
+            elif p0 - P < S:
+                k[b, p0 - P] = 0.0
+                k[b, p0 - P, :, DIM] = BLOCK_VALUE
+        if 0 <= PEAK - P < S:
+            k[b, PEAK - P] = 0.0
+            k[b, PEAK - P, :, DIM] = PEAK_VALUE
+    kc0, vc0 = kc.clone(), vc.clone()
+    out = mimo.prefill_cached(lib_layer(spec, None), q, k, v, torch.tensor(past, dtype=torch.int32, device="cuda"),
+                              kc, vc, max_past_len=max(past))
+    torch.cuda.synchronize()
+    assert mimo.mimo_attn_get_device_error() == 0
+    heads = [0, 1, 30, 63]
+    ref, _, _ = oracle.prefill_cached_layer(
+        f64(q), f64(k), f64(v), f64(kc0), f64(vc0), past, layer_type=0, num_kv_heads=spec.num_kv_heads,
+        rotary_dim=spec.rotary_dim, theta=spec.theta, window=spec.window, sinks=None,
+        hidden_size=spec.hidden_size, heads=heads)
+    c = compare(f64(out)[:, :, heads].reshape(-1), ref[:, :, heads].reshape(-1))
+    assert c.ok(BF), f"max_abs={c.max_abs:.3e} mean_abs={c.mean_abs:.3e} over {c.n}"
