@@ -137,6 +137,10 @@ def status_string(status: int) -> str:
 def _ptr(t: Optional[torch.Tensor]):
     if t is None:
         return None
+    if isinstance(t, torch.Tensor) and not t.is_cuda:
+        # every pointer of the C ABI is a device pointer: a host address would
+        # reach a kernel as a bad address
+        raise ValueError("tensors passed to the library must be on a CUDA device")
     if not t.is_contiguous():
         raise ValueError("tensors passed to the library must be contiguous")
     return ctypes.c_void_p(t.data_ptr())
@@ -161,6 +165,8 @@ def make_layer(layer_type: int, num_q_heads: int, num_kv_heads: int, qk_dim: int
                sinks: Optional[torch.Tensor] = None, softmax_scale: float = 0.0) -> mimo_attn_layer:
     """Fills the C struct; `sinks` is a device fp32 tensor [Hq] or None (the
     struct keeps its pointer, so keep the tensor alive while the struct is used)."""
+    if isinstance(sinks, torch.Tensor) and not (sinks.is_cuda and sinks.dtype == torch.float32 and sinks.is_contiguous()):
+        raise ValueError("sinks must be a contiguous fp32 tensor on a CUDA device")
     return mimo_attn_layer(int(layer_type), int(num_q_heads), int(num_kv_heads), int(qk_dim),
                            int(v_dim), int(rotary_dim), int(window), int(hidden_size),
                            float(rope_theta), float(softmax_scale),

@@ -297,3 +297,15 @@ def test_python_conveniences_check_dtypes(lib):
                           torch.zeros((1, 128, 8, 128), dtype=torch.uint8), 1.0, 1.0)
     with pytest.raises(ValueError):
         mimo.quantize_fp8(torch.zeros(8, dtype=torch.float32), 1.0)
+
+
+def test_python_binding_refuses_host_tensors(lib):
+    """Every pointer of the C ABI is a device pointer: the binding refuses
+    tensors in host memory (and host sink logits) before any call."""
+    import torch
+    spec_q = torch.zeros((1, 16, 64, 192), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        mimo.prefill(layer(), spec_q, torch.zeros((1, 16, 8, 192), dtype=torch.bfloat16),
+                     torch.zeros((1, 16, 8, 128), dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        mimo.make_layer(mimo.SWA, 64, 8, 192, 128, 64, 128, 1e4, 4096, torch.zeros(64, dtype=torch.float32))
