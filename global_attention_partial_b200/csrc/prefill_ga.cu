@@ -355,17 +355,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_ga_kernel(const __grid_co
             tc_fence_after();
             float x[kBlockN];
             {
-                uint32_t r[kBlockN / 16][16];
+                uint32_t r[kBlockN / 32][32];
 #pragma unroll
-                for (int c = 0; c < kBlockN / 16; ++c)
-                    tmem_ld16(s_addr + 16 * c, r[c]);
+                for (int c = 0; c < kBlockN / 32; ++c)
+                    tmem_ld32(s_addr + 32 * c, r[c]);
                 tmem_wait_ld_only();
 #pragma unroll
-                for (int c = 0; c < kBlockN / 16; ++c) {
+                for (int c = 0; c < kBlockN / 32; ++c) {
                     tmem_tie(r[c]);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        x[16 * c + e] = __uint_as_float(r[c][e]);  // raw scores; scale folded below
+                    for (int e = 0; e < 32; ++e)
+                        x[32 * c + e] = __uint_as_float(r[c][e]);  // raw scores; scale folded below
                 }
             }
             const int k0 = j * kBlockN;
@@ -413,16 +413,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_ga_kernel(const __grid_co
             const float sc = p.scale_log2;
             float rsv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c0 = 0; c0 < kBlockN; c0 += 16) {
-                uint32_t r[8];
+            for (int c0 = 0; c0 < kBlockN; c0 += 64) {
+                uint32_t r[32];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < 32; ++c) {
                     const float e0 = fast_exp2(fmaf(x[c0 + 2 * c], sc, -m_use));
                     const float e1 = fast_exp2(fmaf(x[c0 + 2 * c + 1], sc, -m_use));
                     rsv[c & 3] += e0 + e1;
                     r[c] = pack_bf16x2(e0, e1);
                 }
-                tmem_st8(s_addr + c0 / 2, r);
+                tmem_st32(s_addr + c0 / 2, r);
             }
             l_sum += (rsv[0] + rsv[1]) + (rsv[2] + rsv[3]);
             tmem_wait_st();
