@@ -106,12 +106,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_ga_kernel(const __grid_co
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Heaviest causal tiles first.
-    const int pt = p.num_p_tiles - 1 - (int)blockIdx.x;
-    const int pair = (int)blockIdx.y;   // kv head * (G/2) + pair within the group
-    const int b = (int)blockIdx.z;
-    const int kvh = pair / (p.G / 2);
-    const int hA = kvh * p.G + 2 * (pair % (p.G / 2));
+    // Launch order (x fastest): the query-head pairs of one KV head, then the
+    // position tiles with the heaviest causal range first, then (KV head,
+    // batch). The CTAs resident together read one K/V stream, and every
+    // group's heaviest tiles start with the group, not at the end of the grid.
+    const int pt = p.num_p_tiles - 1 - (int)blockIdx.y;
+    const int hkv = p.num_pairs / (p.G / 2);
+    const int kvh = (int)blockIdx.z % hkv;
+    const int b = (int)blockIdx.z / hkv;
+    const int hA = kvh * p.G + 2 * (int)blockIdx.x;
     const int p0 = pt * kBlockM;
     const int q_last = min(p0 + kBlockM, p.S) - 1;
     // Query i is the token at key index past + i (past = 0 for a plain prefill).
@@ -513,7 +516,9 @@ cudaError_t launch_prefill_ga(const LayerArgs &L, const PrefillArgs &a, cudaStre
     cudaError_t e = prepare_kernel_once(prefill_ga_kernel, kSmemBytes, prepared, kLaunchRegs);
     if (e != cudaSuccess)
         return e;
-    dim3 grid(p.num_p_tiles, p.num_pairs, a.B);
+    if (p.num_p_tiles > 65535 || (long long)L.Hkv * a.B > 65535)
+        return cudaErrorInvalidValue;
+    dim3 grid(L.G / 2, p.num_p_tiles, L.Hkv * a.B);
     prefill_ga_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p);
     return cudaGetLastError();
 }
