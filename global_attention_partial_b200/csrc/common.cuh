@@ -553,13 +553,6 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src,
                  : "memory");
 }
 
-// Arrives on `bar` (without raising its pending count) once every cp.async
-// this thread issued so far has landed.
-__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar)
-{
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 __device__ __forceinline__ void cp_async_commit()
 {
     asm volatile("cp.async.commit_group;" ::: "memory");
